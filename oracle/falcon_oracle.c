@@ -1,0 +1,382 @@
+/*
+ * falcon_oracle.c -- TEST INFRASTRUCTURE ONLY. Not part of the product path.
+ *
+ * A plain, slow, fp64 CPU oracle for the forward pass of the Falcon fast-weight
+ * memory ("Fast Weight Attention for Continual Learning"). Only the test suite,
+ * the package smoke check and the CPU-baseline leg of the benchmark call it.
+ * It shares no code, header, table or helper with the CUDA library; the two
+ * meet only through the seeded input generator, which holds none of the
+ * method's arithmetic.
+ *
+ * What the method computes, as stated in the authors' abstract (Hugging Face
+ * paper page, ai.info and hotpaper.ai pages for "Fast Weight Attention for
+ * Continual Learning"):
+ *   - each head keeps a fixed-size state S (d_v x d_k) and the state transition
+ *     is an online learning rule;
+ *   - under read-after-write semantics the example written at step t is the
+ *     prefix-aligned pair (x_t, y_t) = (phi(k_{t-1}), v_t);
+ *   - normalised first-order updates of a squared-error regression objective
+ *     give Falcon-1 (scalar NLMS) and Falcon-3 (sliding-window mini-batch); the
+ *     negative inner-product objective gives the "A" variants;
+ *   - recurrent, masked-parallel and chunk-parallel forms exist, with a
+ *     numerically stable positive-decay renormalisation.
+ * The normalised step size is the Kaczmarz/NLMS one, written out explicitly in
+ * the Kaczmarz Linear Attention abstract on the thelatestinai.com page
+ * "Fast Weight Attention for Continual Learning": beta = eta / (||key||^2 + eps).
+ *
+ * Readings taken where the pages are silent (each is also listed in the
+ * design notes):
+ *   R1 read after write: o_t = S_t q_t.
+ *   R2 decay before the step, residual at the decayed state:
+ *        Sbar = alpha_t S_{t-1};   Falcon-1: S_t = Sbar - beta_t (Sbar x_t - y_t) x_t^T.
+ *   R3 alpha_t, eta_t belong to write step t.
+ *   R4 phi = identity; q is not mapped.
+ *   R5 beta_t = eta_t / (||x_t||^2 + eps); Falcon-3 uses the window's summed
+ *      squared key norms; if the denominator is 0 (zero key and eps = 0) the
+ *      step is a no-op (beta = 0).
+ *   R6 x_1 = k_prev when a cache is given, else 0 (no write at the first step).
+ *   R7 Falcon-3 window W_t = {max(1, t-w+1) .. t}; all residuals of one step use
+ *      the same decayed state (a simultaneous mini-batch gradient step).
+ *   R8 Falcon-1A / Falcon-3A: gradient step of -y^T S x with the same beta:
+ *        S_t = alpha_t S_{t-1} + beta_t sum_{j in W_t} y_j x_j^T.
+ *   R9 positive-decay renormalisation: only decay factors exp(g_i - g_j) with
+ *      i >= j are ever formed, so each factor lies in (0, 1]; nothing is divided
+ *      by a cumulative product of alphas.
+ *
+ * Indices below are 0-based: pair j has x_j = k_{j-1} (j >= 1), x_0 = k_prev
+ * or 0, and y_j = v_j.
+ *
+ * Layout: q, k (B,H,T,dk); v, o (B,H,T,dv); alpha, eta (B,H,T);
+ *         S0, S_out (B,H,dv,dk) with S[i][c] the weight from key coordinate c
+ *         to value coordinate i; k_prev, k_last (B,H,dk). All row-major fp64.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define OR_RULE_1 1
+#define OR_RULE_1A 2
+#define OR_RULE_3 3
+#define OR_RULE_3A 4
+
+#define OR_OK 0
+#define OR_EINVAL -1
+#define OR_ENOMEM -2
+
+static int rule_ok(int rule) {
+    return rule == OR_RULE_1 || rule == OR_RULE_1A || rule == OR_RULE_3 || rule == OR_RULE_3A;
+}
+
+/* The regression family (Falcon-1, Falcon-3) versus the inner-product family. */
+static int is_regression(int rule) { return rule == OR_RULE_1 || rule == OR_RULE_3; }
+
+/* Falcon-1 and Falcon-1A write one pair per step; Falcon-3 and -3A a window. */
+static int eff_window(int rule, int window) {
+    return (rule == OR_RULE_3 || rule == OR_RULE_3A) ? window : 1;
+}
+
+static double dotd(const double *a, const double *b, int n) {
+    double s = 0.0;
+    for (int i = 0; i < n; ++i) s += a[i] * b[i];
+    return s;
+}
+
+/* x_j: the key half of pair j (prefix-aligned pair of the abstract; reading R6). */
+static void pair_key(double *x, const double *kh, const double *kprev_h, long j, int dk) {
+    if (j >= 1)
+        memcpy(x, kh + (size_t)(j - 1) * dk, sizeof(double) * dk);
+    else if (j == 0 && kprev_h)
+        memcpy(x, kprev_h, sizeof(double) * dk);
+    else
+        memset(x, 0, sizeof(double) * dk);
+}
+
+/* Normalised step size (Kaczmarz Linear Attention abstract; reading R5). */
+static double step_size(double eta, double norm_sum, double eps) {
+    double den = norm_sum + eps;
+    return den > 0.0 ? eta / den : 0.0;
+}
+
+static int check_args(int rule, int B, int H, int T, int dk, int dv, int window,
+                      const double *q, const double *k, const double *v,
+                      const double *alpha, const double *eta) {
+    if (!rule_ok(rule) || B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return 0;
+    if ((rule == OR_RULE_3 || rule == OR_RULE_3A) && window < 1) return 0;
+    if ((size_t)B * H * T > 0 && (!q || !k || !v || !alpha || !eta)) return 0;
+    return 1;
+}
+
+/* ------------------------------------------------------------------------
+ * Recurrent form, one head ("step-by-step (recurrent)" form of the ai.info
+ * overview, "Methodology in Plain English"; update rules of the abstract).
+ * Literally per token:
+ *   Sbar = alpha_t S
+ *   beta = eta_t / (sum_{j in W_t} ||x_j||^2 + eps)
+ *   regression:     S = Sbar - beta * sum_j (Sbar x_j - y_j) x_j^T
+ *   inner product:  S = Sbar + beta * sum_j y_j x_j^T
+ *   o_t = S q_t
+ * ------------------------------------------------------------------------ */
+static int recurrent_head(int rule, int T, int dk, int dv, const double *q, const double *k,
+                          const double *v, const double *alpha, const double *eta, double eps,
+                          int w, const double *S0, const double *kprev, double *o,
+                          double *S_out, double *k_last) {
+    double *S = (double *)calloc((size_t)dv * dk, sizeof(double));
+    double *X = (double *)malloc(sizeof(double) * (size_t)w * dk);
+    double *R = (double *)malloc(sizeof(double) * (size_t)w * dv);
+    if (!S || !X || !R) {
+        free(S); free(X); free(R);
+        return OR_ENOMEM;
+    }
+    if (S0) memcpy(S, S0, sizeof(double) * (size_t)dv * dk);
+    const int regression = is_regression(rule);
+
+    for (long t = 0; t < T; ++t) {
+        const double a = alpha[t];
+        for (size_t i = 0; i < (size_t)dv * dk; ++i) S[i] *= a; /* Sbar = alpha_t S */
+
+        double nsum = 0.0;
+        for (int m = 0; m < w; ++m) {
+            pair_key(X + (size_t)m * dk, k, kprev, t - m, dk);
+            nsum += dotd(X + (size_t)m * dk, X + (size_t)m * dk, dk);
+        }
+        const double beta = step_size(eta[t], nsum, eps);
+
+        if (regression) {
+            /* all residuals at the same decayed state (reading R7) */
+            for (int m = 0; m < w; ++m) {
+                const long j = t - m;
+                for (int i = 0; i < dv; ++i) {
+                    const double yi = (j >= 0) ? v[(size_t)j * dv + i] : 0.0;
+                    R[(size_t)m * dv + i] = dotd(S + (size_t)i * dk, X + (size_t)m * dk, dk) - yi;
+                }
+            }
+            for (int m = 0; m < w; ++m)
+                for (int i = 0; i < dv; ++i) {
+                    const double ri = beta * R[(size_t)m * dv + i];
+                    for (int c = 0; c < dk; ++c) S[(size_t)i * dk + c] -= ri * X[(size_t)m * dk + c];
+                }
+        } else {
+            for (int m = 0; m < w; ++m) {
+                const long j = t - m;
+                if (j < 0) continue;
+                for (int i = 0; i < dv; ++i) {
+                    const double yi = beta * v[(size_t)j * dv + i];
+                    for (int c = 0; c < dk; ++c) S[(size_t)i * dk + c] += yi * X[(size_t)m * dk + c];
+                }
+            }
+        }
+        /* read after write (reading R1) */
+        for (int i = 0; i < dv; ++i) o[(size_t)t * dv + i] = dotd(S + (size_t)i * dk, q + (size_t)t * dk, dk);
+    }
+    if (S_out) memcpy(S_out, S, sizeof(double) * (size_t)dv * dk);
+    if (k_last) {
+        if (T > 0) memcpy(k_last, k + (size_t)(T - 1) * dk, sizeof(double) * dk);
+        else if (kprev) memcpy(k_last, kprev, sizeof(double) * dk);
+        else memset(k_last, 0, sizeof(double) * dk);
+    }
+    free(S); free(X); free(R);
+    return OR_OK;
+}
+
+/* ------------------------------------------------------------------------
+ * Chunk-parallel form, one head (chunk-parallel and masked-parallel forms of
+ * the abstract, with positive-decay renormalisation; reading R9).
+ *
+ * Unrolling the recurrence over one block of steps s = 0..n-1 that starts from
+ * state S_c: every step writes pseudo-values u_{s,m} (one per window slot m,
+ * pair j = c0 + s - m):
+ *   S_after_s = exp(g_s) S_c + sum_{s' <= s} sum_m exp(g_s - g_s') u_{s',m} x_{s'-m}^T
+ * where g_s = sum_{s'' <= s} log alpha is the block-local cumulative log decay.
+ * Substituting into the step rule gives, for the regression family, the unit
+ * lower-triangular system
+ *   u_{s,m} + beta_s sum_{s' < s} sum_m' exp(g_s - g_s') (x_{s-m} . x_{s'-m'}) u_{s',m'}
+ *       = beta_s (y_{s-m} - exp(g_s) S_c x_{s-m}),
+ * and u_{s,m} = beta_s y_{s-m} for the inner-product family. Then
+ *   o_{c0+i} = exp(g_i) S_c q_i + sum_{s' <= i} sum_m exp(g_i - g_s') (q_i . x_{s'-m}) u_{s',m}
+ *   S_{c+1}  = exp(g_{n-1}) S_c + sum_{s'} sum_m exp(g_{n-1} - g_s') u_{s',m} x_{s'-m}^T.
+ * Every decay factor formed has a non-positive exponent. With block = T this is
+ * the masked-parallel form (one T-step block, global cumulative log decay).
+ * ------------------------------------------------------------------------ */
+static int blocked_head(int rule, int T, int dk, int dv, const double *q, const double *k,
+                        const double *v, const double *alpha, const double *eta, double eps,
+                        int w, int C, const double *S0, const double *kprev, double *o,
+                        double *S_out, double *k_last) {
+    const size_t Emax = (size_t)C * w;
+    double *S = (double *)calloc((size_t)dv * dk, sizeof(double));
+    double *Xe = (double *)malloc(sizeof(double) * Emax * dk);
+    double *Ye = (double *)malloc(sizeof(double) * Emax * dv);
+    double *U = (double *)malloc(sizeof(double) * Emax * dv);
+    double *beta = (double *)malloc(sizeof(double) * (size_t)C);
+    double *g = (double *)malloc(sizeof(double) * (size_t)C);
+    if (!S || !Xe || !Ye || !U || !beta || !g) {
+        free(S); free(Xe); free(Ye); free(U); free(beta); free(g);
+        return OR_ENOMEM;
+    }
+    if (S0) memcpy(S, S0, sizeof(double) * (size_t)dv * dk);
+    const int regression = is_regression(rule);
+
+    for (long c0 = 0; c0 < T; c0 += C) {
+        const int n = (int)((T - c0) < C ? (T - c0) : C);
+        const int E = n * w;
+        /* expanded rows e = s*w + m hold pair j = c0 + s - m */
+        for (int s = 0; s < n; ++s)
+            for (int m = 0; m < w; ++m) {
+                const int e = s * w + m;
+                const long j = c0 + s - m;
+                pair_key(Xe + (size_t)e * dk, k, kprev, j, dk);
+                if (j >= 0) memcpy(Ye + (size_t)e * dv, v + (size_t)j * dv, sizeof(double) * dv);
+                else memset(Ye + (size_t)e * dv, 0, sizeof(double) * dv);
+            }
+        double acc = 0.0;
+        for (int s = 0; s < n; ++s) {
+            double nsum = 0.0;
+            for (int m = 0; m < w; ++m) {
+                const double *xe = Xe + (size_t)(s * w + m) * dk;
+                nsum += dotd(xe, xe, dk);
+            }
+            beta[s] = step_size(eta[c0 + s], nsum, eps);
+            acc += log(alpha[c0 + s]);
+            g[s] = acc;
+        }
+        /* pseudo-values */
+        for (int e = 0; e < E; ++e) {
+            const int s = e / w;
+            const double *xe = Xe + (size_t)e * dk;
+            double *ue = U + (size_t)e * dv;
+            if (regression) {
+                const double gs = exp(g[s]);
+                for (int i = 0; i < dv; ++i)
+                    ue[i] = beta[s] * (Ye[(size_t)e * dv + i] - gs * dotd(S + (size_t)i * dk, xe, dk));
+                /* forward substitution through the strictly lower block part */
+                for (int e2 = 0; e2 < s * w; ++e2) {
+                    const int s2 = e2 / w;
+                    const double l = beta[s] * exp(g[s] - g[s2]) * dotd(xe, Xe + (size_t)e2 * dk, dk);
+                    const double *u2 = U + (size_t)e2 * dv;
+                    for (int i = 0; i < dv; ++i) ue[i] -= l * u2[i];
+                }
+            } else {
+                for (int i = 0; i < dv; ++i) ue[i] = beta[s] * Ye[(size_t)e * dv + i];
+            }
+        }
+        /* outputs, read after write: the inclusive (s' <= i) sum */
+        for (int i = 0; i < n; ++i) {
+            const long t = c0 + i;
+            const double *qt = q + (size_t)t * dk;
+            double *ot = o + (size_t)t * dv;
+            const double gi = exp(g[i]);
+            for (int r = 0; r < dv; ++r) ot[r] = gi * dotd(S + (size_t)r * dk, qt, dk);
+            for (int e2 = 0; e2 < (i + 1) * w; ++e2) {
+                const int s2 = e2 / w;
+                const double p = exp(g[i] - g[s2]) * dotd(qt, Xe + (size_t)e2 * dk, dk);
+                const double *u2 = U + (size_t)e2 * dv;
+                for (int r = 0; r < dv; ++r) ot[r] += p * u2[r];
+            }
+        }
+        /* state passing */
+        const double gl = g[n - 1];
+        const double dl = exp(gl);
+        for (size_t idx = 0; idx < (size_t)dv * dk; ++idx) S[idx] *= dl;
+        for (int e2 = 0; e2 < E; ++e2) {
+            const int s2 = e2 / w;
+            const double f = exp(gl - g[s2]);
+            const double *u2 = U + (size_t)e2 * dv;
+            const double *x2 = Xe + (size_t)e2 * dk;
+            for (int r = 0; r < dv; ++r) {
+                const double fr = f * u2[r];
+                for (int c = 0; c < dk; ++c) S[(size_t)r * dk + c] += fr * x2[c];
+            }
+        }
+    }
+    if (S_out) memcpy(S_out, S, sizeof(double) * (size_t)dv * dk);
+    if (k_last) {
+        if (T > 0) memcpy(k_last, k + (size_t)(T - 1) * dk, sizeof(double) * dk);
+        else if (kprev) memcpy(k_last, kprev, sizeof(double) * dk);
+        else memset(k_last, 0, sizeof(double) * dk);
+    }
+    free(S); free(Xe); free(Ye); free(U); free(beta); free(g);
+    return OR_OK;
+}
+
+typedef struct {
+    int rule, B, H, T, dk, dv, w, C;
+    const double *q, *k, *v, *alpha, *eta, *S0, *k_prev;
+    double eps;
+    double *o, *S_out, *k_last;
+} job_t;
+
+static int run_heads(const job_t *J, int blocked, int threads) {
+    const long BH = (long)J->B * J->H;
+    int status = OR_OK;
+    if (threads < 1) threads = 1;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1) num_threads(threads)
+#endif
+    for (long bh = 0; bh < BH; ++bh) {
+        const size_t T = (size_t)J->T;
+        const double *S0h = J->S0 ? J->S0 + (size_t)bh * J->dv * J->dk : NULL;
+        const double *kph = J->k_prev ? J->k_prev + (size_t)bh * J->dk : NULL;
+        double *Soh = J->S_out ? J->S_out + (size_t)bh * J->dv * J->dk : NULL;
+        double *klh = J->k_last ? J->k_last + (size_t)bh * J->dk : NULL;
+        int rc;
+        if (blocked)
+            rc = blocked_head(J->rule, J->T, J->dk, J->dv, J->q + bh * T * J->dk, J->k + bh * T * J->dk,
+                              J->v + bh * T * J->dv, J->alpha + bh * T, J->eta + bh * T, J->eps, J->w,
+                              J->C, S0h, kph, J->o + bh * T * J->dv, Soh, klh);
+        else
+            rc = recurrent_head(J->rule, J->T, J->dk, J->dv, J->q + bh * T * J->dk, J->k + bh * T * J->dk,
+                                J->v + bh * T * J->dv, J->alpha + bh * T, J->eta + bh * T, J->eps, J->w,
+                                S0h, kph, J->o + bh * T * J->dv, Soh, klh);
+        if (rc != OR_OK) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            status = rc;
+        }
+    }
+    return status;
+}
+
+/* Exported entry points (fp64 host arrays; threads = OpenMP threads over (b,h)). */
+
+int falcon_oracle_recurrent(int rule, int B, int H, int T, int dk, int dv, const double *q,
+                            const double *k, const double *v, const double *alpha,
+                            const double *eta, double eps, int window, const double *S0,
+                            const double *k_prev, double *o, double *S_out, double *k_last,
+                            int threads) {
+    if (!check_args(rule, B, H, T, dk, dv, window, q, k, v, alpha, eta)) return OR_EINVAL;
+    if ((size_t)B * H * T > 0 && !o) return OR_EINVAL;
+    job_t J = {rule, B, H, T, dk, dv, eff_window(rule, window), 1, q, k, v, alpha, eta, S0, k_prev,
+               eps, o, S_out, k_last};
+    return run_heads(&J, 0, threads);
+}
+
+int falcon_oracle_chunk(int rule, int B, int H, int T, int dk, int dv, const double *q,
+                        const double *k, const double *v, const double *alpha, const double *eta,
+                        double eps, int window, int chunk, const double *S0, const double *k_prev,
+                        double *o, double *S_out, double *k_last, int threads) {
+    if (!check_args(rule, B, H, T, dk, dv, window, q, k, v, alpha, eta) || chunk < 1) return OR_EINVAL;
+    if ((size_t)B * H * T > 0 && !o) return OR_EINVAL;
+    job_t J = {rule, B, H, T, dk, dv, eff_window(rule, window), chunk, q, k, v, alpha, eta, S0,
+               k_prev, eps, o, S_out, k_last};
+    return run_heads(&J, 1, threads);
+}
+
+/* Masked-parallel form: the whole sequence as one block (global cumulative log decay). */
+int falcon_oracle_masked(int rule, int B, int H, int T, int dk, int dv, const double *q,
+                         const double *k, const double *v, const double *alpha, const double *eta,
+                         double eps, int window, const double *S0, const double *k_prev, double *o,
+                         double *S_out, double *k_last, int threads) {
+    return falcon_oracle_chunk(rule, B, H, T, dk, dv, q, k, v, alpha, eta, eps, window,
+                               T > 0 ? T : 1, S0, k_prev, o, S_out, k_last, threads);
+}
+
+int falcon_oracle_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
