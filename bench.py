@@ -1,0 +1,476 @@
+#!/usr/bin/env python
+"""Benchmark of the Falcon fast-weight forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl falcon|reference]
+
+One step = one chunk-parallel forward pass (falcon_fwd_chunk: prep, chunk-local
+solve and state propagation, fused in one kernel) of Falcon-1 over the
+workload B8 H16 T4096 d128, chunk 64, bf16 q/k/v, fp32 state (synthetic seeded
+inputs resident in HBM; 549.5 MB per step, larger than the 126 MB L2, so no
+flush is needed between steps). The same run also times the single-token
+decode step (256 sequences x 32 heads, 128x128 fp32 state, 1000 repeated
+steps) and reports its HBM GB/s, and the fp32 recurrent form on its small
+workload.
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent
+batch (weak scaling, no collective on the data path); the timed region is
+bracketed by barriers and the max over ranks is taken.
+
+--impl reference times the fp64 CPU oracle (the only reference this method
+has) on a bounded sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Falcon-1 chunk fwd tokens/s & % roofline (B8 H16 T4K d128); decode GB/s"
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+CHUNK_KERNEL_SOURCES = ["chunk_kernel.cuh", "chunk_mma.cuh", "common.cuh"]
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, "delta_rule_linear_falcon_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, files):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(kernel)
+    if not rec or rec.get("source_sha256_16") != kernel_source_hash(files):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.ok = False
+        self._stop = threading.Event()
+        self._th = None
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            self.N = N
+            h = None
+            try:
+                import torch
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                h = N.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            except Exception:
+                h = N.nvmlDeviceGetHandleByIndex(device_index)
+            self.h = h
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report no clocks rather than guess
+            self.err = repr(e)
+
+    def _run(self):
+        N = self.N
+        while not self._stop.is_set():
+            try:
+                self.samples.append(N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM))
+                try:
+                    r = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    r = N.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        self._stop.clear()
+        if self.ok:
+            self._th = threading.Thread(target=self._run, daemon=True)
+            self._th.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._th:
+            self._th.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "NVML unavailable"}
+        busy = [s for s in self.samples]
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(busy),
+                "source": "NVML, sampled every 2 ms during the timed regions"}
+
+
+# ----------------------------------------------------------------------------- workload sizes
+
+def chunk_algorithmic_bytes(B, H, T, dk, dv, io_bytes=2):
+    """Bytes the forward pass must move at minimum: read q, k, v, alpha, eta once,
+    write o, the final state and the continuation key once."""
+    n = B * H * T
+    return (n * (2 * dk + dv) * io_bytes + n * 2 * 4 + n * dv * io_bytes
+            + B * H * dv * dk * 4 + B * H * dk * io_bytes)
+
+
+def chunk_algorithmic_flops(B, H, T, dk, dv, window=1):
+    """Recurrent-form FLOPs: (3 + 4w) dk dv per token-head (7 dk dv for Falcon-1)."""
+    return (3 + 4 * window) * dk * dv * B * H * T
+
+
+def decode_algorithmic_bytes(N, H, dk, dv, io_bytes=2):
+    nh = N * H
+    return (nh * dv * dk * 4 * 2          # state read + write
+            + nh * (2 * dk + dv) * io_bytes  # q, k, v
+            + nh * dk * io_bytes * 2       # k_prev read + write
+            + nh * 2 * 4                   # alpha, eta
+            + nh * dv * io_bytes)          # o
+
+
+# ----------------------------------------------------------------------------- distributed
+
+class Dist:
+    def __init__(self, gpus: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            import torch
+            self.pg.barrier(device_ids=[self.local])
+            torch.cuda.synchronize()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- GPU arms
+
+def bench_chunk(args, D: Dist, clk):
+    import torch
+    from delta_rule_linear_falcon_b200 import falcon as F
+    from delta_rule_linear_falcon_b200 import inputs as I
+
+    s = I.make_seq(I.RULE_1, args.batch, 16, 4096, 128, 128, seed=1 + 1000 * D.rank, io_dtype="bf16",
+                   normalise_qk=True, alpha_mu=4.0, chunk=64)
+    B, H, T, dk, dv = s.shape
+    dev = torch.device("cuda", D.local)
+    hq, hk, hv = (torch.from_numpy(x).to(torch.bfloat16).pin_memory() for x in (s.q, s.k, s.v))
+    ha, he = (torch.from_numpy(x).pin_memory() for x in (s.alpha, s.eta))
+    q, k, v, a, e = (x.to(dev) for x in (hq, hk, hv, ha, he))
+    o = torch.empty((B, H, T, dv), dtype=torch.bfloat16, device=dev)
+    S = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    kl = torch.empty((B, H, dk), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        F.falcon_fwd_chunk(q, k, v, a, e, rule=1, eps=s.eps, chunk=64, o=o, S_out=S, k_last=kl,
+                           stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    D.barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    D.barrier()
+    total_ms = D.max(t0.elapsed_time(t1))
+    kern_ms = statistics.mean(a_.elapsed_time(b_) for a_, b_ in ev)
+    assert F.falcon_check_device_errors(stream) == F.FALCON_OK
+    assert torch.isfinite(o.float()).all().item()
+
+    # end to end through the same C-ABI call from pinned host buffers
+    ho = torch.empty((B, H, T, dv), dtype=torch.bfloat16).pin_memory()
+    hS = torch.empty((B, H, dv, dk), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        for dst, src in ((q, hq), (k, hk), (v, hv), (a, ha), (e, he)):
+            dst.copy_(src, non_blocking=True)
+        step()
+        ho.copy_(o, non_blocking=True)
+        hS.copy_(S, non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        e2e_step()
+    torch.cuda.synchronize()
+    D.barrier()
+    n_e2e = max(1, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with clk:
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    D.barrier()
+    e2e_ms = D.max(e0.elapsed_time(e1)) / n_e2e
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, ha, he))
+    d2h = ho.numel() * ho.element_size() + hS.numel() * hS.element_size()
+    return dict(s=s, total_ms=total_ms, kern_ms=kern_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h)
+
+
+def bench_decode(args, D: Dist, clk):
+    import torch
+    from delta_rule_linear_falcon_b200 import falcon as F
+    from delta_rule_linear_falcon_b200 import inputs as I
+
+    d = I.workload_decode(seed=4 + 1000 * D.rank)
+    dev = torch.device("cuda", D.local)
+    S = torch.from_numpy(d.S).to(dev)
+    kp = torch.from_numpy(d.k_prev).to(torch.bfloat16).to(dev)
+    P = d.q.shape[0]
+    toks = [tuple(torch.from_numpy(x[p]).to(dt).to(dev) for x, dt in
+                  ((d.q, torch.bfloat16), (d.k, torch.bfloat16), (d.v, torch.bfloat16),
+                   (d.alpha, torch.float32), (d.eta, torch.float32))) for p in range(P)]
+    N, H, dv, dk = S.shape
+    o = torch.empty((N, H, dv), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for i in range(max(args.warmup, 3)):
+        F.falcon_decode_step(S, kp, *toks[i % P], rule=1, eps=d.eps, o=o, stream=stream)
+    torch.cuda.synchronize()
+    D.barrier()
+    n = args.decode_steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with clk:
+        t0.record(stream)
+        for i in range(n):
+            F.falcon_decode_step(S, kp, *toks[i % P], rule=1, eps=d.eps, o=o, stream=stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    D.barrier()
+    ms = D.max(t0.elapsed_time(t1)) / n
+    assert F.falcon_check_device_errors(stream) == F.FALCON_OK
+    assert torch.isfinite(S).all().item()
+    return dict(N=N, H=H, dk=dk, dv=dv, ms=ms, steps=n)
+
+
+def bench_recurrent(args, D: Dist):
+    import torch
+    from delta_rule_linear_falcon_b200 import falcon as F
+    from delta_rule_linear_falcon_b200 import inputs as I
+
+    s = I.workload_recurrent_small()
+    dev = torch.device("cuda", D.local)
+    q, k, v, a, e = (torch.from_numpy(x).to(dev) for x in (s.q, s.k, s.v, s.alpha, s.eta))
+    stream = torch.cuda.current_stream(dev)
+    run = lambda: F.falcon_fwd_recurrent(q, k, v, a, e, rule=1, eps=s.eps, stream=stream)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(20):
+        run()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / 20
+    B, H, T, dk, dv = s.shape
+    return {"workload": s.name, "ms_per_call": round(ms, 4),
+            "tokens_per_s": round(B * T / (ms * 1e-3), 1), "note": "latency bound, parity workload"}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def cpu_oracle_sample(heads: int, T: int = 4096, threads=None):
+    """Time the fp64 oracle (recurrent form, OpenMP over heads) on `heads` heads of the
+    chunk workload (b = 0, h = 0..heads-1, all T tokens). Returns (tokens/s, seconds, cores)."""
+    import oracle
+    from delta_rule_linear_falcon_b200 import inputs as I
+    s = I.make_seq(I.RULE_1, 1, heads, T, 128, 128, seed=1, io_dtype="bf16", normalise_qk=True,
+                   alpha_mu=4.0)
+    cores = threads or os.cpu_count() or 1
+    t = time.perf_counter()
+    oracle.recurrent(I.RULE_1, s.q, s.k, s.v, s.alpha, s.eta, s.eps, threads=cores)
+    dt = time.perf_counter() - t
+    # tokens of the workload are (b, t) positions carrying 16 heads each
+    return heads * T / 16.0 / dt, dt, min(cores, heads)
+
+
+# ----------------------------------------------------------------------------- main
+
+def run_reference(args):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    heads = 4
+    cores = os.cpu_count() or 1
+    vals = []
+    for _ in range(args.warmup):
+        cpu_oracle_sample(heads, threads=cores)
+    for _ in range(args.steps):
+        tps, dt, used = cpu_oracle_sample(heads, threads=cores)
+        vals.append((tps, dt, used))
+    tps = statistics.median(v[0] for v in vals)
+    ms = statistics.median(v[1] for v in vals) * 1e3
+    used = vals[0][2]
+    sample = (f"{heads} of 128 heads x 4096 tokens of the B8 H16 T4096 d128 workload per step, "
+              f"fp64 recurrent oracle, OpenMP over heads")
+    line = {"impl": "reference", "metric": METRIC, "value": round(tps, 1), "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": base_config(args),
+            "cpu_baseline": {"value": round(tps, 1), "unit": "tokens/s", "cores": used, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(tps, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def base_config(args):
+    B = args.batch
+    return {"workload": f"falcon1_chunk_bf16_B{B}H16T4096d128_chunk64", "rule": "falcon1",
+            "B": B, "H": 16, "T": 4096, "dk": 128, "dv": 128, "chunk": 64,
+            "global_batch": B * args.gpus, "seq_len": 4096,
+            "parallelism": f"dp{args.gpus} (independent sequences per rank, no collective)",
+            "l2": "inputs larger than L2 (549.5 MB per step at B8 vs 126 MB), no flush"}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["falcon", "reference"], default="falcon")
+    ap.add_argument("--batch", type=int, default=8,
+                    help="batch of the chunk workload (8 = the benchmark; smaller only for profiler captures)")
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    from delta_rule_linear_falcon_b200 import falcon as F
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    F.lib()  # fails loudly if the library is missing
+    D = Dist(args.gpus)
+    torch.cuda.set_device(D.local)
+    clk = ClockSampler(D.local)
+
+    ch = bench_chunk(args, D, clk)
+    dec = bench_decode(args, D, clk)
+    rec = bench_recurrent(args, D) if D.rank == 0 else None
+
+    s = ch["s"]
+    B, H, T, dk, dv = s.shape
+    hbm, tf, src = peaks()
+    tokens = B * T * D.world
+    ms = ch["total_ms"] / args.steps
+    value = tokens / (ms * 1e-3)
+    nbytes = chunk_algorithmic_bytes(B, H, T, dk, dv)
+    flops = chunk_algorithmic_flops(B, H, T, dk, dv)
+    achieved = nbytes / (ch["kern_ms"] * 1e-3) / 1e9
+    t_roof = max(nbytes / (hbm * 1e9), flops / (tf * 1e12))
+    traffic = recorded_traffic("chunk_fwd_kernel", CHUNK_KERNEL_SOURCES)
+    dbytes = decode_algorithmic_bytes(dec["N"], dec["H"], dec["dk"], dec["dv"])
+    dgbs = dbytes / (dec["ms"] * 1e-3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": D.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": base_config(args),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "traffic": traffic,
+                     "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else src,
+                     "algorithmic_bytes_per_launch": nbytes, "kernel": "chunk_fwd_kernel",
+                     "kernel_ms": round(ch["kern_ms"], 4)},
+        "north_star_roofline": {"flops": flops, "bytes": nbytes, "t_roofline_us": round(t_roof * 1e6, 2),
+                                "frac": round(t_roof / (ch["kern_ms"] * 1e-3), 4),
+                                "tflops": round(flops / (ch["kern_ms"] * 1e-3) / 1e12, 2),
+                                "definition": "max(FLOPs/bf16 peak, bytes/HBM peak) / kernel time, "
+                                              "FLOPs = recurrent-form count 7 dk dv per token-head"},
+        "e2e": {"value": round(tokens / (ch["e2e_ms"] * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": ch["h2d"], "d2h_bytes_per_step": ch["d2h"],
+                "ms_per_step": round(ch["e2e_ms"], 3)},
+        "clocks": clk.summary(),
+        "gpu_launches": args.steps,
+        "decode": {"workload": f"falcon1_decode_N{dec['N']}H{dec['H']}d{dec['dk']}", "value": round(dgbs, 1),
+                   "unit": "GB/s", "ms_per_step": round(dec["ms"], 4), "steps": dec["steps"],
+                   "gpu_launches": dec["steps"],
+                   "roofline": {"bound": "hbm", "achieved": round(dgbs, 1), "peak": hbm, "unit": "GB/s",
+                                "frac": round(dgbs / hbm, 4),
+                                "traffic": recorded_traffic("decode_kernel", ["decode.cu", "common.cuh"]),
+                                "algorithmic_bytes_per_launch": dbytes}},
+    }
+    if rec is not None:
+        line["recurrent"] = rec
+    if D.rank == 0 and D.world == 1:
+        heads = 8
+        tps, dt, used = cpu_oracle_sample(heads)
+        line["cpu_baseline"] = {"value": round(tps, 1), "unit": "tokens/s", "cores": used, "kind": "oracle",
+                                "sample": f"{heads} of 128 heads x 4096 tokens, fp64 recurrent oracle "
+                                          f"({dt:.1f} s)"}
+    if D.rank == 0:
+        print(json.dumps(line), flush=True)
+    D.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,51 @@
+// launch.h -- internal launch interface between the C ABI shell (api.cu) and
+// the kernel translation units. Not installed; callers use include/falcon.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace falcon {
+
+struct RecParams {
+    int B, H, T, dk, dv, window;  // window = 1 for Falcon-1/1A
+    bool regression, io_bf16;
+    const void *q, *k, *v, *k_prev;
+    const float *alpha, *eta, *S0;
+    float eps;
+    void *o, *k_last;
+    float *S_out;
+    int *err;
+};
+
+struct DecodeParams {
+    int N, H, dk, dv;
+    bool regression, io_bf16;
+    float *S;
+    void *k_prev;
+    const void *q, *k, *v;
+    const float *alpha, *eta;
+    float eps;
+    void *o;
+    int *err;
+};
+
+struct ChunkParams {
+    int B, H, T, dk, dv;
+    int window;      // pairs per step (1 for Falcon-1/1A)
+    int tok_per_blk; // tokens per block; rows per block = tok_per_blk * window <= 64
+    bool regression, io_bf16;
+    const void *q, *k, *v, *k_prev;
+    const float *alpha, *eta, *S0;
+    float eps;
+    void *o, *k_last;
+    float *S_out;
+    int *err;
+};
+
+size_t recurrent_smem_bytes(int dk, int dv, int window);
+cudaError_t launch_recurrent(const RecParams &p, cudaStream_t s);
+cudaError_t launch_decode(const DecodeParams &p, cudaStream_t s);
+cudaError_t launch_chunk(const ChunkParams &p, int num_sms, cudaStream_t s);
+
+}  // namespace falcon

@@ -23,8 +23,10 @@ head shapes with synthetic values):
 """
 from __future__ import annotations
 
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 import math
+import os
 
 import numpy as np
 
@@ -57,26 +59,35 @@ def uniform01(seed: int, stream: int, n: int) -> np.ndarray:
     return ((z >> np.uint64(11)).astype(np.float64) + 1.0) * (1.0 / 9007199254740992.0)
 
 
-def normal(seed: int, stream: int, n: int, chunk: int = 1 << 24) -> np.ndarray:
-    """n standard normals (float32) by Box-Muller on pairs of uniforms."""
+def _normal_block(base, p0, p1, n, out):
+    i = np.arange(2 * p0, 2 * p1, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        z = _mix(base + i * _GOLDEN)
+    u = ((z >> np.uint64(11)).astype(np.float64) + 1.0) * (1.0 / 9007199254740992.0)
+    u1, u2 = u[0::2], u[1::2]
+    r = np.sqrt(-2.0 * np.log(u1))
+    th = 2.0 * math.pi * u2
+    pair = np.empty(2 * (p1 - p0), dtype=np.float64)
+    pair[0::2] = r * np.cos(th)
+    pair[1::2] = r * np.sin(th)
+    lo = 2 * p0
+    hi = min(n, 2 * p1)
+    out[lo:hi] = pair[: hi - lo]
+
+
+def normal(seed: int, stream: int, n: int, chunk: int = 1 << 21) -> np.ndarray:
+    """n standard normals (float32) by Box-Muller on pairs of uniforms. Element i
+    depends only on (seed, stream, i); blocks are drawn on host threads."""
     out = np.empty(n, dtype=np.float32)
     npair = (n + 1) // 2
     base = _stream_base(seed, stream)
-    for p0 in range(0, npair, chunk):
-        p1 = min(npair, p0 + chunk)
-        i = np.arange(2 * p0, 2 * p1, dtype=np.uint64)
-        with np.errstate(over="ignore"):
-            z = _mix(base + i * _GOLDEN)
-        u = ((z >> np.uint64(11)).astype(np.float64) + 1.0) * (1.0 / 9007199254740992.0)
-        u1, u2 = u[0::2], u[1::2]
-        r = np.sqrt(-2.0 * np.log(u1))
-        th = 2.0 * math.pi * u2
-        pair = np.empty(2 * (p1 - p0), dtype=np.float64)
-        pair[0::2] = r * np.cos(th)
-        pair[1::2] = r * np.sin(th)
-        lo = 2 * p0
-        hi = min(n, 2 * p1)
-        out[lo:hi] = pair[: hi - lo]
+    blocks = [(p0, min(npair, p0 + chunk)) for p0 in range(0, npair, chunk)]
+    if len(blocks) <= 1:
+        for p0, p1 in blocks:
+            _normal_block(base, p0, p1, n, out)
+        return out
+    with ThreadPoolExecutor(max_workers=min(len(blocks), os.cpu_count() or 1)) as ex:
+        list(ex.map(lambda b: _normal_block(base, b[0], b[1], n, out), blocks))
     return out
 
 
@@ -88,10 +99,10 @@ def sigmoid_normal(seed: int, stream: int, n: int, mu: float) -> np.ndarray:
 def round_bf16(x: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bf16 (ties to even); returns float32."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    b = x.view(np.uint32).astype(np.uint64)
-    lsb = (b >> np.uint64(16)) & np.uint64(1)
-    b = (b + np.uint64(0x7FFF) + lsb) & np.uint64(0xFFFF0000)
-    out = b.astype(np.uint32).view(np.float32)
+    b = x.view(np.uint32)
+    lsb = (b >> np.uint32(16)) & np.uint32(1)
+    # finite values cannot carry out of 32 bits (largest finite pattern 0xFF7FFFFF)
+    out = ((b + np.uint32(0x7FFF) + lsb) & np.uint32(0xFFFF0000)).view(np.float32)
     return np.where(np.isnan(x), x, out).reshape(x.shape)
 
 

@@ -1,0 +1,182 @@
+/*
+ * falcon.h -- C ABI of libfalcon, the forward pass of the Falcon fast-weight
+ * memory on NVIDIA B200 (sm_100a).
+ *
+ * The method ("Fast Weight Attention for Continual Learning", authors'
+ * abstract): every head keeps a state S of d_v x d_k numbers. At step t the
+ * state is written with the prefix-aligned pair (x_t, y_t) = (phi(k_{t-1}), v_t)
+ * by a gated, normalised first-order update, and it is read after the write:
+ * o_t = S_t q_t. phi is the identity here.
+ *
+ *   Falcon-1  (scalar NLMS, squared-error regression):
+ *       Sbar = alpha_t S_{t-1};  beta_t = eta_t / (||x_t||^2 + eps)
+ *       S_t  = Sbar - beta_t (Sbar x_t - y_t) x_t^T
+ *   Falcon-3  (sliding-window mini-batch over the last w pairs, one step):
+ *       beta_t = eta_t / (sum_{j in W_t} ||x_j||^2 + eps)
+ *       S_t  = Sbar - beta_t sum_{j in W_t} (Sbar x_j - y_j) x_j^T
+ *   Falcon-1A / Falcon-3A (negative inner-product objective):
+ *       S_t  = Sbar + beta_t sum_{j in W_t} y_j x_j^T
+ * The step size is the Kaczmarz/NLMS one (Kaczmarz Linear Attention abstract,
+ * thelatestinai.com page "Fast Weight Attention for Continual Learning").
+ * W_t = {max(1, t-w+1) .. t} (1-based). x_1 = k_prev when a cache is given,
+ * else 0 (no write at the first step). A pair whose denominator
+ * ||x||^2 + eps is 0 writes nothing (beta = 0). alpha in (0, 1] and eta >= 0
+ * are preconditions; they are not checked per element.
+ *
+ * Conventions shared by every entry point:
+ *  - All tensors are dense, row-major, contiguous, in DEVICE memory owned by
+ *    the caller. The library never allocates, frees or synchronises (except
+ *    falcon_check_device_errors, which synchronises the given stream).
+ *  - q, k: (B,H,T,d_k); v, o: (B,H,T,d_v); alpha, eta: (B,H,T) fp32;
+ *    S0, S_out: (B,H,d_v,d_k) fp32 with S[i][c] the weight from key
+ *    coordinate c to value coordinate i; k_prev, k_last: (B,H,d_k).
+ *    q, k, v, o, k_prev and k_last share io_dtype (fp32 or bf16).
+ *  - Every pointer must be 16-byte aligned except alpha and eta (4 bytes).
+ *  - Calls are asynchronous on `stream` (0 = the legacy default stream).
+ *    Shape, pointer, alignment and dtype checks run on the host before any
+ *    launch; a failed check launches nothing and returns
+ *    FALCON_ERR_INVALID_ARG or FALCON_ERR_UNSUPPORTED.
+ *  - A launch failure returns FALCON_ERR_CUDA (the CUDA error is left for
+ *    cudaGetLastError to report).
+ *  - No exception crosses this boundary.
+ */
+#ifndef FALCON_H_
+#define FALCON_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define FALCON_API __attribute__((visibility("default")))
+#else
+#define FALCON_API
+#endif
+
+/* Same underlying type as cudaStream_t. */
+typedef struct CUstream_st *falcon_stream_t;
+
+typedef enum {
+    FALCON_OK = 0,
+    FALCON_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, bad enum   */
+    FALCON_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels implement      */
+    FALCON_ERR_WORKSPACE = 3,   /* workspace smaller than falcon_workspace_size()    */
+    FALCON_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed              */
+    FALCON_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up                */
+} falcon_status_t;
+
+typedef enum {
+    FALCON_RULE_1 = 1,  /* Falcon-1: scalar NLMS                                  */
+    FALCON_RULE_1A = 2, /* Falcon-1A: normalised additive (inner-product) write   */
+    FALCON_RULE_3 = 3,  /* Falcon-3: sliding-window mini-batch (window w)         */
+    FALCON_RULE_3A = 4  /* Falcon-3A: windowed inner-product write (window w)     */
+} falcon_rule_t;
+
+typedef enum { FALCON_F32 = 0, FALCON_BF16 = 1 } falcon_dtype_t;
+
+/* Arguments of the two sequence entry points. Integer fields hold the enums
+ * above. */
+typedef struct {
+    int rule;           /* falcon_rule_t                                             */
+    int io_dtype;       /* falcon_dtype_t of q, k, v, k_prev, k_last and o            */
+    int B, H, T;        /* batch, heads, tokens (T >= 0)                              */
+    int dk, dv;         /* key/query and value widths                                 */
+    const void *q;      /* (B,H,T,dk)                                                 */
+    const void *k;      /* (B,H,T,dk)                                                 */
+    const void *v;      /* (B,H,T,dv)                                                 */
+    const float *alpha; /* (B,H,T) decay gate, preconditions 0 < alpha <= 1           */
+    const float *eta;   /* (B,H,T) step gate, precondition eta >= 0                   */
+    float eps;          /* >= 0, added to the (window) squared key norm                */
+    int window;         /* Falcon-3/3A window w >= 1; ignored by Falcon-1/1A           */
+    int chunk;          /* chunk-parallel block: 16, 32 or 64 pseudo-value rows        */
+    const float *S0;    /* (B,H,dv,dk) initial state, or NULL for zero                 */
+    const void *k_prev; /* (B,H,dk) key cached before this segment, or NULL (x_1 = 0) */
+    void *o;            /* (B,H,T,dv) output, written                                  */
+    float *S_out;       /* (B,H,dv,dk) final state, or NULL                            */
+    void *k_last;       /* (B,H,dk) last key (the cache for a continuation), or NULL   */
+} falcon_args_t;
+
+/*
+ * Bytes of device workspace falcon_fwd_chunk needs for these arguments
+ * (0 when it needs none). Returns 0 for invalid arguments as well; the call
+ * itself reports those.
+ */
+FALCON_API size_t falcon_workspace_size(const falcon_args_t *args);
+
+/*
+ * falcon_fwd_chunk -- chunk-parallel forward pass with positive-decay
+ * renormalisation (authors' abstract of "Fast Weight Attention for Continual
+ * Learning"; ai.info overview, section Methodology in Plain English, which
+ * describes the blocked form).
+ *
+ * Per block of pseudo-value rows the kernel forms the decay-weighted key Gram
+ * and query-key tiles, solves the unit lower-triangular system of the block
+ * (Falcon-1/3), applies it to the residuals against the state carried in from
+ * the previous block, writes the block's outputs and passes the fp32 state on.
+ * Decay factors are only ever formed as exp(g_i - g_j) with i >= j on a
+ * block-local cumulative log decay, so each lies in (0, 1].
+ *
+ * Supported: dk, dv in {32, 64, 128}; chunk in {16, 32, 64}; Falcon-3/3A need
+ * 1 <= window <= chunk and process floor(chunk / window) tokens per block.
+ * Tensor-core products take bf16 operands with fp32 accumulation and an fp32
+ * state, whatever io_dtype is; use falcon_fwd_recurrent for fp32-accurate work.
+ * `workspace` may be NULL when falcon_workspace_size() is 0.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+FALCON_API falcon_status_t falcon_fwd_chunk(const falcon_args_t *args, void *workspace,
+                                 size_t workspace_bytes, falcon_stream_t stream);
+
+/*
+ * falcon_fwd_recurrent -- recurrent form (authors' abstract; ai.info overview,
+ * section Methodology in Plain English): the literal per-token recurrence
+ * with an fp32 state and fp32 arithmetic. One CTA per (b, h) walks t = 1..T.
+ * Supported: 1 <= dk, dv <= 128; window <= 64 for Falcon-3/3A; `chunk` is
+ * ignored. Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+FALCON_API falcon_status_t falcon_fwd_recurrent(const falcon_args_t *args, falcon_stream_t stream);
+
+/*
+ * falcon_decode_step -- one token of the recurrence for N independent
+ * sequences x H heads, in place: the recurrent form applied to a single step,
+ * the incremental state update that the ai.info overview of "Fast Weight
+ * Attention for Continual Learning" lists for streaming inference (section
+ * Why This Matters).
+ *
+ *   x = k_prev; beta = eta / (||x||^2 + eps); Sbar = alpha S
+ *   Falcon-1:  S <- Sbar - beta (Sbar x - v) x^T     Falcon-1A: S <- Sbar + beta v x^T
+ *   o = S q;   k_prev <- k
+ *
+ * S (N,H,dv,dk) fp32 and k_prev (N,H,dk) io_dtype are read and written in
+ * place; q, k (N,H,dk), v (N,H,dv) io_dtype; alpha, eta (N,H) fp32;
+ * o (N,H,dv) io_dtype is written. The buffers of one call must not overlap.
+ * Supported: rule Falcon-1 or Falcon-1A (Falcon-3/3A need a window of past
+ * pairs and return UNSUPPORTED); dk in {32, 64, 128}; 1 <= dv <= 256.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+FALCON_API falcon_status_t falcon_decode_step(int rule, int io_dtype, int N, int H, int dk, int dv,
+                                   float *S, void *k_prev, const void *q, const void *k,
+                                   const void *v, const float *alpha, const float *eta,
+                                   float eps, void *o, falcon_stream_t stream);
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+FALCON_API const char *falcon_status_string(falcon_status_t status);
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device error
+ * word (set by a kernel that detected an inconsistent launch, or by a bounded
+ * wait that gave up). Returns FALCON_OK, FALCON_ERR_TIMEOUT, FALCON_ERR_CUDA
+ * (a CUDA error surfaced while synchronising) or FALCON_ERR_INVALID_ARG
+ * (a kernel rejected its launch geometry).
+ */
+FALCON_API falcon_status_t falcon_check_device_errors(falcon_stream_t stream);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+FALCON_API int falcon_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FALCON_H_ */

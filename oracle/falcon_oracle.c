@@ -110,8 +110,8 @@ static int check_args(int rule, int B, int H, int T, int dk, int dv, int window,
 }
 
 /* ------------------------------------------------------------------------
- * Recurrent form, one head ("step-by-step (recurrent)" form of the ai.info
- * overview, "Methodology in Plain English"; update rules of the abstract).
+ * Recurrent form, one head (authors' abstract; ai.info overview, section
+ * Methodology in Plain English; update rules of the abstract).
  * Literally per token:
  *   Sbar = alpha_t S
  *   beta = eta_t / (sum_{j in W_t} ||x_j||^2 + eps)
