@@ -165,37 +165,58 @@ def decode_algorithmic_bytes(N, H, dk, dv, io_bytes=2):
 # ----------------------------------------------------------------------------- distributed
 
 class Dist:
-    def __init__(self, gpus: int):
+    """One process per GPU (torchrun env). NCCL on GPUs; gloo for CPU tests.
+    Only the timing reduction and barriers cross ranks: no data-path collective."""
+
+    def __init__(self, backend: str = "nccl"):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
         self.pg = None
         if self.world > 1:
             import datetime
-            import torch
             import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            kw = {}
+            if backend == "nccl":
+                import torch
+                torch.cuda.set_device(self.local)
+                kw["device_id"] = torch.device("cuda", self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
             self.pg = dist
 
     def barrier(self):
         if self.pg:
-            import torch
-            self.pg.barrier(device_ids=[self.local])
-            torch.cuda.synchronize()
+            if self.backend == "nccl":
+                import torch
+                self.pg.barrier(device_ids=[self.local])
+                torch.cuda.synchronize()
+            else:
+                self.pg.barrier()
 
     def max(self, x: float) -> float:
         if not self.pg:
             return x
         import torch
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dev = "cuda" if self.backend == "nccl" else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
     def close(self):
         if self.pg:
             self.pg.destroy_process_group()
+            self.pg = None
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own independent batch (weak scaling)."""
+    return base_seed + 1000 * rank
+
+
+def weak_scaling_value(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job throughput: units processed by all ranks / slowest rank's time."""
+    return units_per_rank * world / (max_ms * 1e-3)
 
 
 # ----------------------------------------------------------------------------- GPU arms
@@ -205,7 +226,7 @@ def bench_chunk(args, D: Dist, clk):
     from delta_rule_linear_falcon_b200 import falcon as F
     from delta_rule_linear_falcon_b200 import inputs as I
 
-    s = I.make_seq(I.RULE_1, args.batch, 16, 4096, 128, 128, seed=1 + 1000 * D.rank, io_dtype="bf16",
+    s = I.make_seq(I.RULE_1, args.batch, 16, args.seq_len, 128, 128, seed=rank_seed(1, D.rank), io_dtype="bf16",
                    normalise_qk=True, alpha_mu=4.0, chunk=64)
     B, H, T, dk, dv = s.shape
     dev = torch.device("cuda", D.local)
@@ -277,7 +298,7 @@ def bench_decode(args, D: Dist, clk):
     from delta_rule_linear_falcon_b200 import falcon as F
     from delta_rule_linear_falcon_b200 import inputs as I
 
-    d = I.workload_decode(seed=4 + 1000 * D.rank)
+    d = I.workload_decode(N=args.decode_seqs, seed=rank_seed(4, D.rank))
     dev = torch.device("cuda", D.local)
     S = torch.from_numpy(d.S).to(dev)
     kp = torch.from_numpy(d.k_prev).to(torch.bfloat16).to(dev)
@@ -334,19 +355,44 @@ def bench_recurrent(args, D: Dist):
 
 # ----------------------------------------------------------------------------- CPU oracle
 
+_SAMPLE_CACHE = {}
+
+
+def _oracle_sample_inputs(heads: int, T: int):
+    from delta_rule_linear_falcon_b200 import inputs as I
+    key = (heads, T)
+    if key not in _SAMPLE_CACHE:
+        _SAMPLE_CACHE[key] = I.make_seq(I.RULE_1, 1, heads, T, 128, 128, seed=1, io_dtype="bf16",
+                                        normalise_qk=True, alpha_mu=4.0)
+    return _SAMPLE_CACHE[key]
+
+
 def cpu_oracle_sample(heads: int, T: int = 4096, threads=None):
     """Time the fp64 oracle (recurrent form, OpenMP over heads) on `heads` heads of the
     chunk workload (b = 0, h = 0..heads-1, all T tokens). Returns (tokens/s, seconds, cores)."""
     import oracle
     from delta_rule_linear_falcon_b200 import inputs as I
-    s = I.make_seq(I.RULE_1, 1, heads, T, 128, 128, seed=1, io_dtype="bf16", normalise_qk=True,
-                   alpha_mu=4.0)
+    s = _oracle_sample_inputs(heads, T)
     cores = threads or os.cpu_count() or 1
     t = time.perf_counter()
     oracle.recurrent(I.RULE_1, s.q, s.k, s.v, s.alpha, s.eta, s.eps, threads=cores)
     dt = time.perf_counter() - t
     # tokens of the workload are (b, t) positions carrying 16 heads each
     return heads * T / 16.0 / dt, dt, min(cores, heads)
+
+
+def cpu_baseline(min_seconds: float = 10.0, heads: int = 64):
+    """The oracle as it stands on the host cores: repeated passes over `heads` of the 128
+    heads of the B8 H16 T4096 d128 workload until at least `min_seconds` of work."""
+    total_t, total_tok, passes = 0.0, 0.0, 0
+    while total_t < min_seconds:
+        tps, dt, used = cpu_oracle_sample(heads)
+        total_t += dt
+        total_tok += tps * dt
+        passes += 1
+    return {"value": round(total_tok / total_t, 1), "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "sample": f"{passes} passes x {heads} of 128 heads x 4096 tokens of the B8 H16 T4096 d128 "
+                      f"workload, fp64 recurrent oracle, OpenMP over heads ({total_t:.1f} s)"}
 
 
 # ----------------------------------------------------------------------------- main
@@ -380,12 +426,13 @@ def run_reference(args):
 
 
 def base_config(args):
-    B = args.batch
-    return {"workload": f"falcon1_chunk_bf16_B{B}H16T4096d128_chunk64", "rule": "falcon1",
-            "B": B, "H": 16, "T": 4096, "dk": 128, "dv": 128, "chunk": 64,
-            "global_batch": B * args.gpus, "seq_len": 4096,
+    B, T = args.batch, getattr(args, "seq_len", 4096)
+    nbytes = chunk_algorithmic_bytes(B, 16, T, 128, 128)
+    return {"workload": f"falcon1_chunk_bf16_B{B}H16T{T}d128_chunk64", "rule": "falcon1",
+            "B": B, "H": 16, "T": T, "dk": 128, "dv": 128, "chunk": 64,
+            "global_batch": B * args.gpus, "seq_len": T,
             "parallelism": f"dp{args.gpus} (independent sequences per rank, no collective)",
-            "l2": "inputs larger than L2 (549.5 MB per step at B8 vs 126 MB), no flush"}
+            "l2": f"inputs larger than L2 ({nbytes / 1e6:.1f} MB per step vs 126 MB), no flush"}
 
 
 def main(argv=None):
@@ -396,7 +443,12 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["falcon", "reference"], default="falcon")
     ap.add_argument("--batch", type=int, default=8,
                     help="batch of the chunk workload (8 = the benchmark; smaller only for profiler captures)")
+    ap.add_argument("--seq-len", type=int, default=4096,
+                    help="tokens per sequence of the chunk workload (4096 = the benchmark; shorter "
+                         "only for profiler captures: same kernel configuration, fewer blocks)")
     ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--decode-seqs", type=int, default=256,
+                    help="sequences of the decode workload (256 = the benchmark)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -408,7 +460,7 @@ def main(argv=None):
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
     F.lib()  # fails loudly if the library is missing
-    D = Dist(args.gpus)
+    D = Dist("nccl")
     torch.cuda.set_device(D.local)
     clk = ClockSampler(D.local)
 
@@ -421,7 +473,7 @@ def main(argv=None):
     hbm, tf, src = peaks()
     tokens = B * T * D.world
     ms = ch["total_ms"] / args.steps
-    value = tokens / (ms * 1e-3)
+    value = weak_scaling_value(B * T, D.world, ms)
     nbytes = chunk_algorithmic_bytes(B, H, T, dk, dv)
     flops = chunk_algorithmic_flops(B, H, T, dk, dv)
     achieved = nbytes / (ch["kern_ms"] * 1e-3) / 1e9
@@ -461,11 +513,7 @@ def main(argv=None):
     if rec is not None:
         line["recurrent"] = rec
     if D.rank == 0 and D.world == 1:
-        heads = 8
-        tps, dt, used = cpu_oracle_sample(heads)
-        line["cpu_baseline"] = {"value": round(tps, 1), "unit": "tokens/s", "cores": used, "kind": "oracle",
-                                "sample": f"{heads} of 128 heads x 4096 tokens, fp64 recurrent oracle "
-                                          f"({dt:.1f} s)"}
+        line["cpu_baseline"] = cpu_baseline(min_seconds=10.0)
     if D.rank == 0:
         print(json.dumps(line), flush=True)
     D.close()
