@@ -62,7 +62,7 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
 }
 
 template <int DK, typename IO, bool REGRESSION>
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kDecThreads, 2)
 decode_kernel(DecodeParams p) {
     constexpr int VPL = DK / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -2,9 +2,10 @@
 // fp32 state (the recurrent form of "Fast Weight Attention for Continual
 // Learning": authors' abstract; ai.info overview, Methodology in Plain English).
 //
-// One CTA per (b, h). Thread i owns row i of S (d_v rows of d_k fp32 in shared
-// memory, padded stride so that the row-per-thread walk is bank-conflict
-// free). Keys and values of the last w pairs live in a ring in shared memory.
+// One CTA per (b, h). Thread i owns row i of S in registers (d_k padded to
+// DKMAX); keys and values of the last w pairs live in a ring in shared memory.
+// The inputs of step t+1 are loaded into registers while step t computes, so
+// the per-step latency is two barriers and the row arithmetic.
 // Per step t (0-based, pair j = t - m for window slot m):
 //   Sbar = alpha_t S
 //   beta = eta_t / (sum_m ||x_{t-m}||^2 + eps)
@@ -17,19 +18,16 @@
 namespace falcon {
 
 constexpr int kRecThreads = 128;
+constexpr int kRecMaxWindow = 64;
 
-template <typename IO, bool REGRESSION>
+template <typename IO, bool REGRESSION, int DKMAX>
 __global__ void __launch_bounds__(kRecThreads)
 recurrent_kernel(RecParams p) {
     extern __shared__ float smem[];
     const int dk = p.dk, dv = p.dv, W = p.window;
-    const int ldS = dk + 1;
-    float *sS = smem;                        // dv x ldS
-    float *sX = sS + (size_t)dv * ldS;       // W x dk  key ring
-    float *sY = sX + (size_t)W * dk;         // W x dv  value ring
-    float *sN = sY + (size_t)W * dv;         // W       squared key norms
-    float *sQ = sN + W;                      // dk      current query
-    float *sBeta = sQ + dk;                  // 1
+    float *sX = smem;                   // W x DKMAX key ring (zero padded)
+    float *sY = sX + (size_t)W * DKMAX; // W x dv   value ring
+    float *sQ = sY + (size_t)W * dv;    // 2 x DKMAX queries (double buffered)
 
     const int tid = threadIdx.x;
     const long bh = blockIdx.x;
@@ -42,71 +40,114 @@ recurrent_kernel(RecParams p) {
     const float *eta = p.eta + bh * (size_t)T;
     IO *o = reinterpret_cast<IO *>(p.o) + bh * (size_t)T * dv;
 
-    for (int idx = tid; idx < dv * dk; idx += kRecThreads) {
-        const int i = idx / dk, c = idx % dk;
-        sS[i * ldS + c] = p.S0 ? p.S0[bh * (size_t)dv * dk + idx] : 0.f;
+    for (int idx = tid; idx < W * (DKMAX + dv) + 2 * DKMAX; idx += kRecThreads) smem[idx] = 0.f;
+
+    const bool has_row = tid < dv;
+    float S[DKMAX];
+#pragma unroll
+    for (int c = 0; c < DKMAX; ++c)
+        S[c] = (has_row && p.S0 && c < dk) ? p.S0[(bh * (size_t)dv + tid) * dk + c] : 0.f;
+
+    // registers holding the inputs of the step about to be staged
+    auto load_x = [&](int t) -> float {   // key half of pair t, coordinate tid
+        if (tid >= dk) return 0.f;
+        if (t >= 1) return Io<IO>::ld(k, (size_t)(t - 1) * dk + tid);
+        return kp ? Io<IO>::ld(kp, tid) : 0.f;
+    };
+    float xr = 0.f, qr = 0.f, yr = 0.f, ar = 1.f, er = 0.f;
+    if (T > 0) {
+        xr = load_x(0);
+        qr = tid < dk ? Io<IO>::ld(q, tid) : 0.f;
+        yr = has_row ? Io<IO>::ld(v, tid) : 0.f;
+        ar = alpha[0];
+        er = eta[0];
     }
-    for (int idx = tid; idx < W * (dk + dv + 1); idx += kRecThreads) sX[idx] = 0.f;  // ring + norms
     __syncthreads();
 
+    int slot = 0;
     for (int t = 0; t < T; ++t) {
-        const int slot = t % W;
-        // (A) stage pair t = (x_t, y_t) and the query
-        for (int c = tid; c < dk; c += kRecThreads) {
-            float x;
-            if (t >= 1) x = Io<IO>::ld(k, (size_t)(t - 1) * dk + c);
-            else x = kp ? Io<IO>::ld(kp, c) : 0.f;
-            sX[slot * dk + c] = x;
-            sQ[c] = Io<IO>::ld(q, (size_t)t * dk + c);
+        // (A) stage pair t and q_t, then start loading step t+1
+        if (tid < dk) {
+            sX[slot * DKMAX + tid] = xr;
+            sQ[(t & 1) * DKMAX + tid] = qr;
         }
-        for (int i = tid; i < dv; i += kRecThreads) sY[slot * dv + i] = Io<IO>::ld(v, (size_t)t * dv + i);
-        __syncthreads();
-        // (B) squared norm of x_t and the step size over the window
-        if (tid < 32) {
-            float s = 0.f;
-            for (int c = tid; c < dk; c += 32) s += sX[slot * dk + c] * sX[slot * dk + c];
-            s = warp_sum(s);
-            if (tid == 0) {
-                sN[slot] = s;
-                const int nw = t + 1 < W ? t + 1 : W;
-                float ns = 0.f;
-                for (int m = 0; m < nw; ++m) ns += sN[(t - m) % W];
-                sBeta[0] = step_size(eta[t], ns, p.eps);
-            }
+        if (has_row) sY[slot * dv + tid] = yr;
+        const float a = ar, e = er;
+        if (t + 1 < T) {
+            xr = load_x(t + 1);
+            qr = tid < dk ? Io<IO>::ld(q, (size_t)(t + 1) * dk + tid) : 0.f;
+            yr = has_row ? Io<IO>::ld(v, (size_t)(t + 1) * dv + tid) : 0.f;
+            ar = alpha[t + 1];
+            er = eta[t + 1];
         }
         __syncthreads();
-        // (C) row updates and the read after the write
-        const float a = alpha[t];
-        const float beta = sBeta[0];
+
+        // (B) window step size (every thread computes it from the ring)
         const int nw = t + 1 < W ? t + 1 : W;
-        for (int i = tid; i < dv; i += kRecThreads) {
-            float *Si = sS + i * ldS;
-            float coef[64];
-            if (REGRESSION) {
-                for (int m = 0; m < nw; ++m) {
-                    const float *x = sX + ((t - m) % W) * dk;
-                    float r = 0.f;
-                    for (int c = 0; c < dk; ++c) r += Si[c] * x[c];
-                    coef[m] = beta * (a * r - sY[((t - m) % W) * dv + i]);  // beta (Sbar x - y)
-                }
-            } else {
-                for (int m = 0; m < nw; ++m) coef[m] = -beta * sY[((t - m) % W) * dv + i];
+        float ns = 0.f;
+        {
+            int sl = slot;
+            for (int m = 0; m < nw; ++m) {
+                const float *x = sX + sl * DKMAX;
+#pragma unroll 8
+                for (int c = 0; c < DKMAX; ++c) ns += x[c] * x[c];
+                sl = sl == 0 ? W - 1 : sl - 1;
             }
-            float out = 0.f;
-            for (int c = 0; c < dk; ++c) {
-                float s = a * Si[c];
-                for (int m = 0; m < nw; ++m) s -= coef[m] * sX[((t - m) % W) * dk + c];
-                Si[c] = s;
-                out += s * sQ[c];
-            }
-            Io<IO>::st(o, (size_t)t * dv + i, out);
         }
+        const float beta = step_size(e, ns, p.eps);
+
+        // (C) row update and the read after the write
+        if (has_row) {
+#pragma unroll
+            for (int c = 0; c < DKMAX; ++c) S[c] *= a;  // Sbar
+            if (W == 1) {
+                const float *x = sX;  // slot 0
+                float r = 0.f;
+#pragma unroll
+                for (int c = 0; c < DKMAX; ++c) r += S[c] * x[c];
+                const float coef = REGRESSION ? beta * (r - sY[tid]) : -beta * sY[tid];
+#pragma unroll
+                for (int c = 0; c < DKMAX; ++c) S[c] -= coef * x[c];
+            } else {
+                float coef[kRecMaxWindow];
+                int sl = slot;
+                for (int m = 0; m < nw; ++m) {
+                    const float *x = sX + sl * DKMAX;
+                    if (REGRESSION) {
+                        float r = 0.f;
+#pragma unroll
+                        for (int c = 0; c < DKMAX; ++c) r += S[c] * x[c];
+                        coef[m] = beta * (r - sY[sl * dv + tid]);
+                    } else {
+                        coef[m] = -beta * sY[sl * dv + tid];
+                    }
+                    sl = sl == 0 ? W - 1 : sl - 1;
+                }
+                sl = slot;
+                for (int m = 0; m < nw; ++m) {
+                    const float *x = sX + sl * DKMAX;
+                    const float cm = coef[m];
+#pragma unroll
+                    for (int c = 0; c < DKMAX; ++c) S[c] -= cm * x[c];
+                    sl = sl == 0 ? W - 1 : sl - 1;
+                }
+            }
+            const float *qq = sQ + (t & 1) * DKMAX;
+            float out = 0.f;
+#pragma unroll
+            for (int c = 0; c < DKMAX; ++c) out += S[c] * qq[c];
+            Io<IO>::st(o, (size_t)t * dv + tid, out);
+        }
+        slot = slot + 1 == W ? 0 : slot + 1;
         __syncthreads();
     }
 
-    if (p.S_out)
-        for (int idx = tid; idx < dv * dk; idx += kRecThreads)
-            p.S_out[bh * (size_t)dv * dk + idx] = sS[(idx / dk) * ldS + idx % dk];
+    if (p.S_out && has_row) {
+        float *So = p.S_out + (bh * (size_t)dv + tid) * dk;
+#pragma unroll
+        for (int c = 0; c < DKMAX; ++c)
+            if (c < dk) So[c] = S[c];
+    }
     if (p.k_last) {
         IO *kl = reinterpret_cast<IO *>(p.k_last) + bh * (size_t)dk;
         for (int c = tid; c < dk; c += kRecThreads) {
@@ -118,14 +159,17 @@ recurrent_kernel(RecParams p) {
     }
 }
 
+static int dk_max(int dk) { return dk <= 32 ? 32 : (dk <= 64 ? 64 : 128); }
+
 size_t recurrent_smem_bytes(int dk, int dv, int window) {
-    return sizeof(float) * ((size_t)dv * (dk + 1) + (size_t)window * (dk + dv + 1) + dk + 1);
+    const int D = dk_max(dk);
+    return sizeof(float) * ((size_t)window * (D + dv) + 2 * D);
 }
 
-template <typename IO, bool REG>
+template <typename IO, bool REG, int DKMAX>
 static cudaError_t launch_rec(const RecParams &p, cudaStream_t s) {
     const size_t smem = recurrent_smem_bytes(p.dk, p.dv, p.window);
-    auto kern = recurrent_kernel<IO, REG>;
+    auto kern = recurrent_kernel<IO, REG, DKMAX>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long grid = (long)p.B * p.H;
@@ -134,10 +178,20 @@ static cudaError_t launch_rec(const RecParams &p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+template <typename IO, bool REG>
+static cudaError_t launch_rec_dk(const RecParams &p, cudaStream_t s) {
+    switch (dk_max(p.dk)) {
+        case 32: return launch_rec<IO, REG, 32>(p, s);
+        case 64: return launch_rec<IO, REG, 64>(p, s);
+        default: return launch_rec<IO, REG, 128>(p, s);
+    }
+}
+
 cudaError_t launch_recurrent(const RecParams &p, cudaStream_t s) {
+    if (p.dk > 128 || p.dv > kRecThreads || p.window > kRecMaxWindow || p.window < 1) return cudaErrorInvalidValue;
     const bool reg = p.regression;
-    if (p.io_bf16) return reg ? launch_rec<__nv_bfloat16, true>(p, s) : launch_rec<__nv_bfloat16, false>(p, s);
-    return reg ? launch_rec<float, true>(p, s) : launch_rec<float, false>(p, s);
+    if (p.io_bf16) return reg ? launch_rec_dk<__nv_bfloat16, true>(p, s) : launch_rec_dk<__nv_bfloat16, false>(p, s);
+    return reg ? launch_rec_dk<float, true>(p, s) : launch_rec_dk<float, false>(p, s);
 }
 
 }  // namespace falcon
