@@ -50,5 +50,8 @@ cudaError_t launch_chunk(const ChunkParams &p, int num_sms, cudaStream_t s);
 // tcgen05 / TMA kernel for d_k = d_v = 128, bf16 I/O, one pair per step, 64-token blocks.
 bool chunk_tc_supported(const ChunkParams &p);
 cudaError_t launch_chunk_tc(const ChunkParams &p, cudaStream_t s);
+// Warp-specialised tcgen05 kernel (same shapes, T a multiple of 4).
+bool chunk_ws_supported(const ChunkParams &p);
+cudaError_t launch_chunk_ws(const ChunkParams &p, cudaStream_t s);
 
 }  // namespace falcon
