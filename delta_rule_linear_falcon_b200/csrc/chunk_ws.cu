@@ -8,15 +8,19 @@
 // (Gram tiles, triangular solve) runs while the state-dependent chain of block
 // c runs, on separate warps that hand work over through mbarriers:
 //   warp 0      TMA producer: [X;Q] and V of each block (2 stages)
-//   warp 1      MMA issuer: (a) [X;Q]X^T -> G,P   (b) S X^T -> SX, S Q~^T -> O
-//                           (d) U^T = R^T T^T   (e) O += U^T P~^T   (f) dS = U^T X~
+//   warp 1      MMA issuer: (a) [X;Q]X^T -> G,P   (b) S [X;Q~]^T -> [SX | O] (N = 128),
+//                           (y) V^T I -> Y^T (the tensor core transposes the values;
+//                               issued right after (e),(f) of the previous block)
+//                           (d) U^T = R^T T'^T  (e) O += U^T P~^T   (f) dS = U^T X~
 //               issued as soon as their inputs are ready (critical chain first)
 //   warps 2-3   helpers: x_1 patch, key norms, step sizes, cumulative log2 decay
-//               and its tables; Q~ = diag(2^g) Q after (a); X~ = diag(2^(g_last-g)) X
-//               after (b), so the state update needs no extra scaled copy
-//   warps 4-7   local: L = diag(beta)(Gamma o G) (fp32), P~ = Gamma o P (bf16),
-//               T = (I + L)^-1 (fp32, tensor-core tf32 block products)
-//   warps 8-15  chain: R^T = diag(beta)(Y - diag(2^g) SX)^T, U^T to bf16, the fp32
+//               and its tables; Q~ = diag(2^g) Q after (a); P~ = Gamma o P from TMEM
+//               lanes 64-127 (their quarters)
+//   warps 4-7   local: L = diag(beta)(Gamma o G) (fp32) from TMEM lanes 0-63,
+//               T = (I + L)^-1 (fp32, tensor-core tf32 block products), stored as
+//               T' = T diag(beta) so the residual needs no step size
+//   warps 8-15  chain: R^T = (Y - diag(2^g) SX)^T; X~ = diag(2^(g_last-g)) X in place while
+//               (d) runs, so the state update needs no extra scaled copy; U^T to bf16; the fp32
 //               state S <- 2^g_last S + dS (in registers) and its bf16 copy, O out
 // Every decay factor is 2^(g_i - g_j) with i >= j (never a quotient of
 // cumulative products). Every wait is bounded; a timeout is recorded in the
@@ -46,15 +50,19 @@ constexpr uint32_t oP = oT + 16384;                // P~ bf16 x 2 slots (B of (e
 constexpr uint32_t oL = oP + 16384;                // L / W fp32 64 x LDF
 constexpr uint32_t oTf = oL + 64 * LDF * 4;        // T fp32 64 x LDF
 constexpr uint32_t oScal = oTf + 64 * LDF * 4;     // 3 slots x {beta, gam, f, g2}[64] + g_last[3] + misc
-constexpr uint32_t oBar = oScal + 3 * 1024 + 64;
-constexpr uint32_t kSmem = oBar + 64 * 8 + 1024;
+constexpr uint32_t oBar = oScal + 4 * 1024;        // 3 slots + 3 column-factor tables + g_last + misc
+constexpr uint32_t oI = oBar + 1024;               // 64 x 64 bf16 identity (B of (y)), 1024-aligned
+constexpr uint32_t kSmem = oI + 8192 + 1024;
 static_assert(kSmem <= 232448, "shared memory");
 
 // TMEM columns
-constexpr uint32_t cGP = 0, cSX = 64, cO = 128 /* + 64 * slot */, cUT = 256, cDS = 320, kTmemCols = 512;
+// GP | [SX_0 | O_0] | [SX_1 | O_1] | Y^T, later U^T (same columns) | dS
+constexpr uint32_t cGP = 0, cSXO = 64 /* + 128 * slot */, cUT = 320, cY = 320, cDS = 384, kTmemCols = 512;
 
 constexpr uint32_t kIdN64 = tc::idesc_bf16(128, 64, 0, 0);
+constexpr uint32_t kIdN128 = tc::idesc_bf16(128, 128, 0, 0);
 constexpr uint32_t kIdN128Bmn = tc::idesc_bf16(128, 128, 0, 1);
+constexpr uint32_t kIdN64Amn = tc::idesc_bf16(128, 64, 1, 0);
 
 // barrier indices
 enum {
@@ -62,11 +70,11 @@ enum {
     B_SFREE = 2,       // [2] (f) done -> producer
     B_XQ = 4,          // helpers -> MMA (a)
     B_ADONE = 5,       // (a) done -> helpers, local
-    B_GPFREE = 6,      // local read G/P -> MMA (a) of the next block
+    B_GPFREE = 6,      // local read G and helpers read P (2 arrivals) -> MMA (a) of the next block
     B_SCAL = 7,        // [3] helpers -> local, chain (scalar slot c % 3)
     B_QSC = 10,        // Q~ ready -> MMA (b)
     B_BDONE = 11,      // (b) done -> helpers, chain
-    B_XSC = 12,        // X~ ready -> MMA (f)
+    B_XSC = 12,        // (unused)
     B_RT = 13,         // R^T ready -> MMA (d)
     B_TRDY = 14,       // [2] T ready -> MMA (d)
     B_PRDY = 16,       // [2] P~ ready -> MMA (e)
@@ -100,10 +108,10 @@ __device__ __forceinline__ void st_chunk8(uint8_t *base, uint32_t off, const flo
 
 // Scale the 16 chunks (128 bf16) of row `r` of a two-atom, 128-row-per-atom tile by `s`.
 __device__ __forceinline__ void scale_row(uint8_t *tile, int r, float s) {
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
+#pragma unroll 1
+    for (int q = 0; q < 16; ++q) {
+        const int a = q >> 3, ch = q & 7;
+        {
             uint4 *pp = reinterpret_cast<uint4 *>(tile + a * 16384 + tc::sw128_chunk(r, ch));
             uint4 u = *pp;
             __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
@@ -114,6 +122,7 @@ __device__ __forceinline__ void scale_row(uint8_t *tile, int r, float s) {
             }
             *pp = u;
         }
+    }
 }
 
 // ---- tf32 warp MMA for the 16 x 16 blocks of the triangular solve
@@ -167,17 +176,25 @@ __device__ __forceinline__ void store16(float *C, const float (&acc)[2][4], int 
 //   W_im = -T_ii L_im (stored over L_im); T_ij = sum_{m=j}^{i-1} W_im T_mj per block diagonal.
 // Entries above the block diagonal of Tf are zero on entry and stay zero.
 __device__ __forceinline__ void solve_local(float *sL, float *sTf, int lt, int lw, int lane) {
-    if (lt < 64) {
+    if (lt < 64) {  // column j of the inverse of diagonal block b, left-looking, rows of L as float4
         const int b = lt >> 4, j = lt & 15;
         const float *Lb = sL + (16 * b) * LDF + 16 * b;
-        float x[16], acc[16];
+        float x[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+        for (int i = 0; i < 16; ++i) {
+            float l[16];
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            x[m] = m < j ? 0.f : (m == j ? 1.f : -acc[m]);
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const float4 w = *reinterpret_cast<const float4 *>(Lb + i * LDF + 4 * q4);
+                l[4 * q4] = w.x; l[4 * q4 + 1] = w.y; l[4 * q4 + 2] = w.z; l[4 * q4 + 3] = w.w;
+            }
+            float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int i = m + 1; i < 16; ++i) acc[i] += Lb[i * LDF + m] * x[m];
+            for (int m = 0; m < i; ++m) {
+                if (m & 1) a1 += l[m] * x[m];
+                else a0 += l[m] * x[m];
+            }
+            x[i] = i < j ? 0.f : (i == j ? 1.f : -(a0 + a1));
         }
         float *Tb = sTf + (16 * b) * LDF + 16 * b;
 #pragma unroll
@@ -242,8 +259,8 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     // Scalars of block c live in slot c % 3 (beta[64] gam[64] f[64] g2[64]); three slots, because the
     // helpers prepare block c+1 while the chain may still read block c-1.
     float *sScal = reinterpret_cast<float *>(sm + oScal);
-    float *sGL = sScal + 768;                              // g_last per slot
-    float *sMisc = sScal + 772;                            // helper scan carry
+    float *sGL = sScal + 960;                              // g_last per slot (after 3 x cf[64])
+    float *sMisc = sScal + 964;                            // helper scan carry
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + B_COUNT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
@@ -255,7 +272,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     constexpr int D = 128;
 
     if (tid == 0) {
-        for (int i = 0; i < B_COUNT; ++i) tc::mbar_init(&bars[i], 1);
+        for (int i = 0; i < B_COUNT; ++i) tc::mbar_init(&bars[i], i == B_GPFREE ? 2 : 1);
         *abort_flag = 0;
         tc::mbar_fence_init();
     }
@@ -264,6 +281,14 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         tc::tmem_relinquish();
     }
     for (int idx = tid; idx < 64 * LDF; idx += kThreads) sTf[idx] = 0.f;
+    for (int idx = tid; idx < 64 * 8; idx += kThreads) {  // identity, row e has a 1 at column e
+        const int e = idx >> 3, ch = idx & 7;
+        float v8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v8[k] = (8 * ch + k == e) ? 1.f : 0.f;
+        st_chunk8(sm + oI, tc::sw128_chunk(e, ch), v8);
+    }
+    tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -304,98 +329,94 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     } else if (warp == 1) {
         // ================================================================ MMA issuer
         if (lane == 0) {
-            const uint32_t aS = tc::smem_u32(sS), aRT = tc::smem_u32(sRT);
-            int na = 0, nb = 0, nd = 0, nef = 0;
-            long long idle_since = clock64();
-            while (nef < nblk && !*abort_flag) {
-                bool prog = false;
-                // (e) + (f)
-                if (nef < (REG ? nd : nb)) {
-                    const int c = nef, s = c & 1;
-                    if (tc::mbar_try_wait(&bars[B_URDY], c & 1) &&
-                        tc::mbar_try_wait(&bars[B_PRDY + s], (c >> 1) & 1) &&
-                        tc::mbar_try_wait(&bars[B_XSC], c & 1)) {
-                        tc::fence_after_sync();
-                        const uint32_t aX = tc::smem_u32(sm + oStage + s * kStage);
-                        const uint32_t aP = tc::smem_u32(sm + oP + s * 8192);
+            // Descriptors are built once; a K step only moves the 14-bit start-address field
+            // (address >> 4), which stays below 2^14 for every operand here, so a plain add is exact.
+            const uint64_t dS = tc::sdesc(tc::smem_u32(sS), 16, 1024);
+            const uint64_t dRT = tc::sdesc(tc::smem_u32(sRT), 16, 1024);
+            const uint64_t dI = tc::sdesc(tc::smem_u32(sm + oI), 16, 1024);
+            uint64_t dX[2], dXmn[2], dV[2], dT[2], dP[2];
 #pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            tc::mma_bf16(tbase + cO + 64 * s, tc::sdesc(aRT + ks * 32, 16, 1024),
-                                         tc::sdesc(aP + ks * 32, 16, 1024), kIdN64, 1);
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            tc::mma_bf16(tbase + cDS, tc::sdesc(aRT + ks * 32, 16, 1024),
-                                         tc::sdesc(aX + ks * 2048, 16384, 1024), kIdN128Bmn, ks > 0);
-                        tc::mma_commit(&bars[B_EFDONE]);
-                        tc::mma_commit(&bars[B_PFREE + s]);
-                        tc::mma_commit(&bars[B_SFREE + s]);
-                        ++nef;
-                        prog = true;
-                    }
-                }
-                // (d)
-                if (REG && nd < nb) {
-                    const int c = nd, s = c & 1;
-                    if (tc::mbar_try_wait(&bars[B_RT], c & 1) && tc::mbar_try_wait(&bars[B_TRDY + s], (c >> 1) & 1)) {
-                        tc::fence_after_sync();
-                        const uint32_t aT = tc::smem_u32(sm + oT + s * 8192);
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            tc::mma_bf16(tbase + cUT, tc::sdesc(aRT + ks * 32, 16, 1024),
-                                         tc::sdesc(aT + ks * 32, 16, 1024), kIdN64, ks > 0);
-                        tc::mma_commit(&bars[B_DDONE]);
-                        tc::mma_commit(&bars[B_TFREE + s]);
-                        ++nd;
-                        prog = true;
-                    }
-                }
-                // (b)
-                if (nb < na) {
-                    const int c = nb, s = c & 1;
-                    if (tc::mbar_try_wait(&bars[B_QSC], c & 1) && tc::mbar_try_wait(&bars[B_SRDY], c & 1) &&
-                        (c < 2 || tc::mbar_try_wait(&bars[B_OFREE + s], ((c >> 1) + 1) & 1))) {
-                        tc::fence_after_sync();
-                        const uint32_t aX = tc::smem_u32(sm + oStage + s * kStage);
-#pragma unroll
-                        for (int ks = 0; ks < 8; ++ks) {
-                            const uint32_t ko = (ks >> 2) * 16384 + (ks & 3) * 32;
-                            tc::mma_bf16(tbase + cSX, tc::sdesc(aS + ko, 16, 1024), tc::sdesc(aX + ko, 16, 1024),
-                                         kIdN64, ks > 0);
-                        }
-#pragma unroll
-                        for (int ks = 0; ks < 8; ++ks) {
-                            const uint32_t ko = (ks >> 2) * 16384 + (ks & 3) * 32;
-                            tc::mma_bf16(tbase + cO + 64 * s, tc::sdesc(aS + ko, 16, 1024),
-                                         tc::sdesc(aX + 8192 + ko, 16, 1024), kIdN64, ks > 0);
-                        }
-                        tc::mma_commit(&bars[B_BDONE]);
-                        ++nb;
-                        prog = true;
-                    }
-                }
-                // (a)
-                if (na < nblk) {
-                    const int c = na, s = c & 1;
-                    if (tc::mbar_try_wait(&bars[B_XQ], c & 1) &&
-                        (c < 1 || tc::mbar_try_wait(&bars[B_GPFREE], (c - 1) & 1))) {
-                        tc::fence_after_sync();
-                        const uint32_t aX = tc::smem_u32(sm + oStage + s * kStage);
-#pragma unroll
-                        for (int ks = 0; ks < 8; ++ks) {
-                            const uint32_t ko = (ks >> 2) * 16384 + (ks & 3) * 32;
-                            tc::mma_bf16(tbase + cGP, tc::sdesc(aX + ko, 16, 1024), tc::sdesc(aX + ko, 16, 1024),
-                                         kIdN64, ks > 0);
-                        }
-                        tc::mma_commit(&bars[B_ADONE]);
-                        ++na;
-                        prog = true;
-                    }
-                }
-                if (prog) {
-                    idle_since = clock64();
-                } else if (clock64() - idle_since > kWaitBudget) {
+            for (int st = 0; st < 2; ++st) {
+                const uint32_t a = tc::smem_u32(sm + oStage + st * kStage);
+                dX[st] = tc::sdesc(a, 16, 1024);            // [X;Q] K-major (also X as N=64 / N=128 B)
+                dXmn[st] = tc::sdesc(a, 16384, 1024);       // X as an MN-major B (dk atoms 16 KB apart)
+                dV[st] = tc::sdesc(a + 32768, 8192, 1024);  // V as an MN-major A (dv atoms 8 KB apart)
+                dT[st] = tc::sdesc(tc::smem_u32(sm + oT + st * 8192), 16, 1024);
+                dP[st] = tc::sdesc(tc::smem_u32(sm + oP + st * 8192), 16, 1024);
+            }
+            auto kmaj = [](int ks) -> uint64_t { return (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4); };
+            auto wait = [&](int b, uint32_t parity) -> bool {
+                if (!tc::mbar_wait(&bars[b], parity, abort_flag, kWaitBudget)) {
                     *abort_flag = 1;
+                    return false;
                 }
+                return true;
+            };
+            // (a): [X;Q] X^T -> G (lanes 0-63), P (lanes 64-127)
+            auto issue_a = [&](int c) {
+                const uint64_t d = dX[c & 1];
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) tc::mma_bf16(tbase + cGP, d + kmaj(ks), d + kmaj(ks), kIdN64, ks > 0);
+                tc::mma_commit(&bars[B_ADONE]);
+            };
+            // (y): Y^T = V^T I (V read as an MN-major A operand of the stage tile)
+            auto issue_y = [&](int c) {
+                const uint64_t d = dV[c & 1];
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16(tbase + cY, d + (uint64_t)(ks * 128), dI + (uint64_t)(ks * 2), kIdN64Amn, ks > 0);
+            };
+            // Program order per block c (each wait parks this thread until its inputs are ready):
+            //   (b)_c, then (a)_{c+1} (runs while the chain forms R_c), (d)_c, (e)(f)_c, then (y)_{c+1}
+            //   (its columns are free once U^T_c has been read, which (e)(f)_c's inputs imply).
+            bool ok = nblk > 0 && wait(B_XQ, 0);
+            if (ok) {
+                issue_a(0);
+                issue_y(0);
+            }
+            for (int c = 0; c < nblk && ok; ++c) {
+                const int s = c & 1;
+                // (b): S [X; Q~]^T in one N = 128 pass -> [SX | O] of slot s
+                if (!(ok = wait(B_QSC, c & 1) && wait(B_SRDY, c & 1) &&
+                           (c < 2 || wait(B_OFREE + s, ((c >> 1) + 1) & 1))))
+                    break;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    tc::mma_bf16(tbase + cSXO + 128 * s, dS + kmaj(ks), dX[s] + kmaj(ks), kIdN128, ks > 0);
+                tc::mma_commit(&bars[B_BDONE]);
+                // (a) of the next block
+                if (c + 1 < nblk) {
+                    if (!(ok = wait(B_XQ, (c + 1) & 1) && wait(B_GPFREE, c & 1))) break;
+                    tc::fence_after_sync();
+                    issue_a(c + 1);
+                }
+                // (d): U^T = R^T T'^T
+                if (REG) {
+                    if (!(ok = wait(B_RT, c & 1) && wait(B_TRDY + s, (c >> 1) & 1))) break;
+                    tc::fence_after_sync();
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        tc::mma_bf16(tbase + cUT, dRT + (uint64_t)(ks * 2), dT[s] + (uint64_t)(ks * 2), kIdN64, ks > 0);
+                    tc::mma_commit(&bars[B_DDONE]);
+                    tc::mma_commit(&bars[B_TFREE + s]);
+                }
+                // (e) O += U^T P~^T and (f) dS = U^T X~
+                if (!(ok = wait(B_URDY, c & 1) && wait(B_PRDY + s, (c >> 1) & 1))) break;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16(tbase + cSXO + 128 * s + 64, dRT + (uint64_t)(ks * 2), dP[s] + (uint64_t)(ks * 2),
+                                 kIdN64, 1);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16(tbase + cDS, dRT + (uint64_t)(ks * 2), dXmn[s] + (uint64_t)(ks * 128), kIdN128Bmn,
+                                 ks > 0);
+                tc::mma_commit(&bars[B_EFDONE]);
+                tc::mma_commit(&bars[B_PFREE + s]);
+                tc::mma_commit(&bars[B_SFREE + s]);
+                // (y) of the next block (its tiles landed before xq_ready of that block)
+                if (c + 1 < nblk) issue_y(c + 1);
             }
             // drain every MMA issued so far
             tc::mma_commit(&bars[B_FINAL]);
@@ -457,6 +478,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             named_bar(1, 64);
             const float gl = sc[192 + nval - 1];
             sc[128 + ht] = exp2f(gl - la);
+            sScal[3 * 256 + 64 * u + ht] = exp2f(sc[192 + (ht | 15)] - la);
             if (leader) sGL[u] = gl;
             named_bar(1, 64);
             if (leader) {
@@ -472,34 +494,12 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             if (c + 1 < nblk) load_gates(c + 1);  // in flight while block c's Q is scaled
             uint8_t *stg = sm + oStage + s * kStage;
             const float *sc = sScal + (c % 3) * 256;
-            // Q~ = diag(2^g) Q once (a) no longer needs Q
             if (!(ok = role_wait(&bars[B_ADONE], c & 1, leader, 1, 64))) break;
-            scale_row(stg, 64 + ht, sc[64 + ht]);
-            tc::fence_proxy_async();
-            named_bar(1, 64);
-            if (leader) mbar_arrive(&bars[B_QSC]);
-            // next block's prep overlaps this block's chain
-            if (c + 1 < nblk && !(ok = prep(c + 1))) break;
-            // X~ = diag(2^(g_last - g)) X once (b) no longer needs X
-            if (!(ok = role_wait(&bars[B_BDONE], c & 1, leader, 1, 64))) break;
-            scale_row(stg, ht, sc[128 + ht]);
-            tc::fence_proxy_async();
-            named_bar(1, 64);
-            if (leader) mbar_arrive(&bars[B_XSC]);
-        }
-    } else if (warp < 8) {
-        // ================================================================ local (128 threads)
-        const int lt = tid - 128, lw = warp - 4;
-        const int r = 32 * lw + lane;      // TMEM lane: G row (r < 64) or P row r - 64
-        const bool leader = lt == 0;
-        const uint32_t tl = tbase + ((uint32_t)(32 * lw) << 16);
-        for (int c = 0; c < nblk; ++c) {
-            const int s = c & 1;
-            if (!role_wait(&bars[B_ADONE], c & 1, leader, 2, 128)) break;
-            if (!role_wait(&bars[B_SCAL + c % 3], (c / 3) & 1, leader, 2, 128)) break;
+            // P of query row i = ht from TMEM lanes 64..127 (this pair of warps' quarters), released at once
             tc::fence_after_sync();
             float v[64];
             {
+                const uint32_t tl = tbase + ((uint32_t)(64 + 32 * (warp - 2)) << 16);
                 float h0[32], h1[32];
                 tc::tmem_ld32(tl + cGP, h0);
                 tc::tmem_ld32(tl + cGP + 32, h1);
@@ -507,45 +507,112 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 for (int j = 0; j < 32; ++j) { v[j] = h0[j]; v[32 + j] = h1[j]; }
             }
             tc::fence_before_sync();
-            named_bar(2, 128);
-            if (leader) mbar_arrive(&bars[B_GPFREE]);
+            // Q~ = diag(2^g) Q once (a) no longer needs Q
+            scale_row(stg, 64 + ht, sc[64 + ht]);
+            tc::fence_proxy_async();
+            named_bar(1, 64);
+            if (leader) {
+                mbar_arrive(&bars[B_GPFREE]);
+                mbar_arrive(&bars[B_QSC]);
+            }
+            // next block's prep overlaps this block's chain (and unblocks (a) of the next block)
+            if (c + 1 < nblk && !(ok = prep(c + 1))) break;
+            // P~ = Gamma o P into P~ slot s, once (e) of block c-2 has released it
+            if (c >= 2 && !(ok = role_wait(&bars[B_PFREE + s], ((c >> 1) + 1) & 1, leader, 1, 64))) break;
+            {
+                const float *g2 = sc + 192, *cf = sScal + 3 * 256 + 64 * (c % 3);
+                const int i = ht, rb = i >> 4;
+                const float gri = g2[i];
+                float fac[4], gd[16];
+#pragma unroll
+                for (int jb = 0; jb < 4; ++jb) {
+                    const float f = exp2f(fminf(gri - g2[16 * jb + 15], 0.f));
+                    fac[jb] = jb < rb ? f : 0.f;
+                }
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const int j = 16 * rb + k;
+                    const float f = exp2f(fminf(gri - g2[j], 0.f));
+                    gd[k] = j <= i ? f : 0.f;
+                }
+                uint8_t *sP = sm + oP + s * 8192;
+#pragma unroll
+                for (int jb = 0; jb < 4; ++jb) {
+                    const bool below = jb < rb, diag = jb == rb;
+                    float pv[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const int j = 16 * jb + k;
+                        const float gm = below ? fac[jb] * cf[j] : (diag ? gd[k] : 0.f);
+                        pv[k] = gm * v[j];
+                    }
+                    st_chunk8(sP, tc::sw128_chunk(i, 2 * jb), pv);
+                    st_chunk8(sP, tc::sw128_chunk(i, 2 * jb + 1), pv + 8);
+                }
+                tc::fence_proxy_async();
+                named_bar(1, 64);
+                if (leader) mbar_arrive(&bars[B_PRDY + s]);
+            }
+        }
+    } else if (warp < 8) {
+        // ================================================================ local (128 threads)
+        const int lt = tid - 128, lw = warp - 4;
+        const int r = 32 * lw + lane;      // TMEM lane: G row for lw < 2 (P rows belong to the helpers)
+        const bool leader = lt == 0;
+        const uint32_t tl = tbase + ((uint32_t)(32 * lw) << 16);
+        for (int c = 0; c < nblk; ++c) {
+            const int s = c & 1;
+            if (!role_wait(&bars[B_ADONE], c & 1, leader, 2, 128)) break;
+            if (!role_wait(&bars[B_SCAL + c % 3], (c / 3) & 1, leader, 2, 128)) break;
+            tc::fence_after_sync();
             const float *sc = sScal + (c % 3) * 256;
-            if (r < 64) {
+            if (lw < 2) {                                   // G rows r = 0..63 -> L (regression family)
+                float v[64];
+                {
+                    float h0[32], h1[32];
+                    tc::tmem_ld32(tl + cGP, h0);
+                    tc::tmem_ld32(tl + cGP + 32, h1);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) { v[j] = h0[j]; v[32 + j] = h1[j]; }
+                }
+                tc::fence_before_sync();
                 if (REG) {
-                    const float be = sc[r], ge = sc[192 + r];
+                    // Decay factors 2^(g_r - g_j), j < r: below the 16x16 diagonal blocks they factor
+                    // through the last index of column block jb, 2^(g_r - g_{16jb+15}) * cf[j] with
+                    // cf[j] = 2^(g_{16jb+15} - g_j) (a helper table), both in (0, 1]; inside the
+                    // diagonal block they are formed directly. Selects only, no divergent branches.
+                    const float *g2 = sc + 192, *cf = sScal + 3 * 256 + 64 * (c % 3);
+                    const int rb = r >> 4;
+                    const float gri = g2[r], be = sc[r];
+                    float fac[4], gd[16];
+#pragma unroll
+                    for (int jb = 0; jb < 4; ++jb) {
+                        const float f = exp2f(fminf(gri - g2[16 * jb + 15], 0.f));
+                        fac[jb] = jb < rb ? be * f : 0.f;
+                    }
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const int j = 16 * rb + k;
+                        const float f = exp2f(fminf(gri - g2[j], 0.f));
+                        gd[k] = j < r ? be * f : 0.f;
+                    }
                     float *Lr = sL + r * LDF;
 #pragma unroll
                     for (int j0 = 0; j0 < 64; j0 += 4) {
-                        float4 w;
-                        w.x = j0 + 0 < r ? be * exp2f(ge - sc[192 + j0 + 0]) * v[j0 + 0] : 0.f;
-                        w.y = j0 + 1 < r ? be * exp2f(ge - sc[192 + j0 + 1]) * v[j0 + 1] : 0.f;
-                        w.z = j0 + 2 < r ? be * exp2f(ge - sc[192 + j0 + 2]) * v[j0 + 2] : 0.f;
-                        w.w = j0 + 3 < r ? be * exp2f(ge - sc[192 + j0 + 3]) * v[j0 + 3] : 0.f;
-                        *reinterpret_cast<float4 *>(Lr + j0) = w;
+                        float w4[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int j = j0 + k, jb = j >> 4;
+                            const float gm = jb < rb ? fac[jb] * cf[j] : (jb == rb ? gd[j & 15] : 0.f);
+                            w4[k] = gm * v[j];
+                        }
+                        *reinterpret_cast<float4 *>(Lr + j0) = make_float4(w4[0], w4[1], w4[2], w4[3]);
                     }
                 }
-            } else {
-                const int i = r - 64;
-                // the P~ slot is free once (e) of block c-2 is done
-                bool okp = c < 2 || tc::mbar_wait(&bars[B_PFREE + s], ((c >> 1) + 1) & 1, abort_flag, kWaitBudget);
-                if (!okp) *abort_flag = 1;
-                const float gi = sc[192 + i];
-                uint8_t *sP = sm + oP + s * 8192;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    float pv[8];
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const int j = 8 * ch + k;
-                        pv[k] = j <= i ? exp2f(gi - sc[192 + j]) * v[j] : 0.f;
-                    }
-                    st_chunk8(sP, tc::sw128_chunk(i, ch), pv);
-                }
-                tc::fence_proxy_async();
             }
             named_bar(2, 128);
+            if (leader) mbar_arrive(&bars[B_GPFREE]);
             if (*abort_flag) break;
-            if (leader) mbar_arrive(&bars[B_PRDY + s]);
             if (REG) {
                 solve_local(sL, sTf, lt, lw, lane);
                 if (c >= 2 && !role_wait(&bars[B_TFREE + s], ((c >> 1) + 1) & 1, leader, 2, 128)) break;
@@ -555,7 +622,9 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 for (int cc = 0; cc < 4; ++cc) {
                     const float4 x0 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + 8 * (ch0 + cc));
                     const float4 x1 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + 8 * (ch0 + cc) + 4);
-                    const float t8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                    const float *bcol = sScal + (c % 3) * 256 + 8 * (ch0 + cc);  // beta of columns
+                    const float t8[8] = {x0.x * bcol[0], x0.y * bcol[1], x0.z * bcol[2], x0.w * bcol[3],
+                                         x1.x * bcol[4], x1.y * bcol[5], x1.z * bcol[6], x1.w * bcol[7]};
                     st_chunk8(sT, tc::sw128_chunk(rr, ch0 + cc), t8);
                 }
                 tc::fence_proxy_async();
@@ -592,26 +661,49 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             tc::fence_after_sync();
             const float *sc = sScal + (c % 3) * 256;
             const float gl = sGL[c % 3];
-            // R^T (or U^T) from S X^T and the values
-            {
-                float v[32], rv[32];
-                tc::tmem_ld32(tl + cSX + 32 * hf, v);
-                const uint8_t *Vt = sm + oStage + s * kStage + 32768 + (row >> 6) * 8192;
-                const int dc = row & 63;
+            // R^T = Y^T - SX diag(2^g) (regression) or U^T = Y^T diag(beta) (inner product),
+            // 16 columns at a time, both operands from TMEM
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int e = 32 * hf + j;
-                    const float y = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
-                        Vt + (e >> 3) * 1024 + (e & 7) * 128 + ((((dc >> 3) ^ (e & 7))) << 4) + (dc & 7) * 2));
-                    rv[j] = REG ? sc[e] * (y - sc[64 + e] * v[j]) : sc[e] * y;
-                }
+            for (int hh = 0; hh < 2; ++hh) {
+                float y[16], v[16], rv[16];
+                const int e0 = 32 * hf + 16 * hh;
+                tc::tmem_ld16(tl + cY + e0, y);
+                if (REG) tc::tmem_ld16(tl + cSXO + 128 * s + e0, v);
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) st_chunk8(sRT, tc::sw128_chunk(row, 4 * hf + cc), rv + 8 * cc);
+                for (int j = 0; j < 16; ++j)
+                    rv[j] = REG ? y[j] - sc[64 + e0 + j] * v[j] : sc[e0 + j] * y[j];
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc)
+                    st_chunk8(sRT, tc::sw128_chunk(row, 4 * hf + 2 * hh + cc), rv + 8 * cc);
             }
             tc::fence_proxy_async();
             tc::fence_before_sync();
             named_bar(3, 256);
-            if (leader) mbar_arrive(&bars[REG ? B_RT : B_URDY]);
+            if (REG && leader) mbar_arrive(&bars[B_RT]);
+            // X~ = diag(2^(g_last - g)) X in place (X is no longer needed unscaled once (b) is done),
+            // so that (f) forms sum_e 2^(g_last - g_e) u_e x_e^T directly; done while (d) runs.
+            {
+                const int xr = ct >> 2, part = ct & 3;
+                uint8_t *xt = sm + oStage + s * kStage + (part >> 1) * 16384;
+                const float f = sc[128 + xr];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    uint4 *pp = reinterpret_cast<uint4 *>(xt + tc::sw128_chunk(xr, 4 * (part & 1) + k));
+                    uint4 u = *pp;
+                    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        const float2 x2 = __bfloat1622float2(h[q2]);
+                        h[q2] = __floats2bfloat162_rn(x2.x * f, x2.y * f);
+                    }
+                    *pp = u;
+                }
+            }
+            if (!REG) {
+                tc::fence_proxy_async();
+                named_bar(3, 256);
+                if (leader) mbar_arrive(&bars[B_URDY]);
+            }
             if (REG) {
                 if (!(ok = role_wait(&bars[B_DDONE], c & 1, leader, 3, 256))) break;
                 tc::fence_after_sync();
@@ -646,12 +738,20 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             // outputs of this block (off the critical chain)
             {
                 float v[32];
-                tc::tmem_ld32(tl + cO + 64 * s + 32 * hf, v);
-                __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.o) + ((size_t)bh * T + t0) * D + row;
+                tc::tmem_ld32(tl + cSXO + 128 * s + 64 + 32 * hf, v);
+                // lane pairs (2k, 2k+1) hold neighbouring value rows: the even lane stores the pair for
+                // even tokens, the odd lane for odd tokens, as 4-byte bf16x2 stores
+                const bool odd = lane & 1;
+                __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.o) + ((size_t)bh * T + t0) * D + (row & ~1);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int i = 32 * hf + j;
-                    if (i < nval) o[(size_t)i * D] = __float2bfloat16_rn(v[j]);
+                for (int j = 0; j < 32; j += 2) {
+                    const float mine = odd ? v[j + 1] : v[j];
+                    const float give = odd ? v[j] : v[j + 1];
+                    const float other = __shfl_xor_sync(0xffffffffu, give, 1);
+                    const int i = 32 * hf + j + (odd ? 1 : 0);
+                    const float lo = odd ? other : mine, hi = odd ? mine : other;
+                    if (i < nval)
+                        *reinterpret_cast<uint32_t *>(o + (size_t)i * D) = pack_bf16x2(lo, hi);
                 }
             }
             tc::fence_before_sync();
