@@ -2,26 +2,32 @@
 // d_k = d_v = 128, bf16 I/O, one pair per step (Falcon-1, Falcon-1A), 64-token
 // blocks. The block algebra is the chunk-parallel form with positive-decay
 // renormalisation of "Fast Weight Attention for Continual Learning" (authors'
-// abstract), written out in chunk_kernel.cuh.
+// abstract), written out in chunk_kernel.cuh, regrouped so that the state
+// recurrence crosses only two tensor-core steps per block. With g the block-local
+// cumulative log2 decay, beta the step sizes, T = (I + L)^-1 and
+//   T' = T diag(beta),  T_f = diag(2^(g_last - g)) T',  A = T_f^T X,  B' = P~ T'
+// (all independent of the state), one block is
+//   R'^T = Y^T - (S X^T) diag(2^g)                          (regression; Y^T for inner product)
+//   O^T  = S Q~^T + R'^T B'^T,   S <- 2^g_last S + R'^T A.
+// For the inner-product rule T = I, so T_f and T' are diagonal and no solve runs.
 //
-// One CTA of 512 threads per (b, h). The state-independent work of block c+1
-// (Gram tiles, triangular solve) runs while the state-dependent chain of block
-// c runs, on separate warps that hand work over through mbarriers:
-//   warp 0      TMA producer: [X;Q] and V of each block (2 stages)
-//   warp 1      MMA issuer: (a) [X;Q]X^T -> G,P   (b) S [X;Q~]^T -> [SX | O] (N = 128),
-//                           (y) V^T I -> Y^T (the tensor core transposes the values;
-//                               issued right after (e),(f) of the previous block)
-//                           (d) U^T = R^T T'^T  (e) O += U^T P~^T   (f) dS = U^T X~
-//               issued as soon as their inputs are ready (critical chain first)
-//   warps 2-3   helpers: x_1 patch, key norms, step sizes, cumulative log2 decay
-//               and its tables; Q~ = diag(2^g) Q after (a); P~ = Gamma o P from TMEM
-//               lanes 64-127 (their quarters)
+// One CTA of 512 threads per (b, h); the state-independent work of later blocks
+// runs on other warps while the state chain of block c runs:
+//   warp 0      TMA producer: [X;Q] of each block into a 3-slot ring (the solve runs two
+//               blocks ahead), V into a 2-slot ring
+//   warp 1      MMA issuer (one thread):
+//                 (a)  [X;Q] X^T -> G (lanes 0-63), P (lanes 64-127)
+//                 (A)  A^T = X^T T_f   and  (B')  B' = [P~; *] T'        (state independent)
+//                 (b)  [S X^T | S Q~^T] with S (bf16) read from tensor memory
+//                 (e') O^T += R'^T B'^T   (f') dS = R'^T A   with R'^T (bf16) from tensor memory
+//               The chain's groups go first; the state-independent ones of later blocks are issued
+//               right behind them, so they run while the chain warps work on the results.
+//   warps 2-3   helpers: x_1 patch, key norms, step sizes, cumulative log2 decay and its
+//               tables; P~ = Gamma o P from TMEM lanes 64-127; Q~ = diag(2^g) Q
 //   warps 4-7   local: L = diag(beta)(Gamma o G) (fp32) from TMEM lanes 0-63,
-//               T = (I + L)^-1 (fp32, tensor-core tf32 block products), stored as
-//               T' = T diag(beta) so the residual needs no step size
-//   warps 8-15  chain: R^T = (Y - diag(2^g) SX)^T; X~ = diag(2^(g_last-g)) X in place while
-//               (d) runs, so the state update needs no extra scaled copy; U^T to bf16; the fp32
-//               state S <- 2^g_last S + dS (in registers) and its bf16 copy, O out
+//               T = (I + L)^-1 (fp32, tensor-core tf32 block products), T_f and T' in bf16
+//   warps 8-15  chain: A^T, B' from TMEM to shared memory; R'^T (bf16 into TMEM); the fp32
+//               state S <- 2^g_last S + dS (in registers) and its bf16 copy in TMEM; O out
 // Every decay factor is 2^(g_i - g_j) with i >= j (never a quotient of
 // cumulative products). Every wait is bounded; a timeout is recorded in the
 // device error word and all roles unwind.
@@ -39,58 +45,74 @@ constexpr int kThreads = 512;
 constexpr int kBlk = 64;
 constexpr long long kWaitBudget = 1ll << 31;  // SM clocks, about 1 s
 constexpr int LDF = 68;                       // fp32 solve buffers: 16-byte rows, conflict-free A fragments
+constexpr int kChainWarps = 8;
 
 // shared memory (bytes from a 1024-aligned base)
-constexpr uint32_t kStage = 49152;                 // [X;Q] 2 atoms x 128 rows + V 2 atoms x 64 rows
-constexpr uint32_t oStage = 0;                     // 2 stages
-constexpr uint32_t oS = 2 * kStage;                // S bf16: 2 atoms x 128 rows (A of (b))
-constexpr uint32_t oRT = oS + 32768;               // R^T then U^T: 1 atom x 128 rows
-constexpr uint32_t oT = oRT + 16384;               // T bf16 x 2 slots (B of (d))
-constexpr uint32_t oP = oT + 16384;                // P~ bf16 x 2 slots (B of (e))
-constexpr uint32_t oL = oP + 16384;                // L / W fp32 64 x LDF
+constexpr uint32_t kXQ = 32768;                    // [X;Q]: 2 atoms (d 0-63, 64-127) x 128 rows (X 0-63, Q 64-127)
+constexpr uint32_t kVst = 16384;                   // V: 2 atoms (v 0-63, 64-127) x 64 rows
+constexpr uint32_t oXQ = 0;                        // 3 slots
+constexpr uint32_t oV = oXQ + 3 * kXQ;             // 2 slots
+constexpr uint32_t oTF = oV + 2 * kVst;            // T_f bf16, 64 x 64 row-major (MN-major B of (A))
+constexpr uint32_t oTP = oTF + 8192;               // T' bf16 (MN-major B of (B'))
+constexpr uint32_t oPB = oTP + 8192;               // rows 0-63 P~ (A of (B')), rows 64-127 B' (B of (e'))
+constexpr uint32_t oA = oPB + 16384;               // A^T bf16, 128 rows (d) x 64 (i) (B of (f'))
+constexpr uint32_t oL = oA + 16384;                // L / W fp32 64 x LDF
 constexpr uint32_t oTf = oL + 64 * LDF * 4;        // T fp32 64 x LDF
-constexpr uint32_t oScal = oTf + 64 * LDF * 4;     // 3 slots x {beta, gam, f, g2}[64] + g_last[3] + misc
-constexpr uint32_t oBar = oScal + 4 * 1024;        // 3 slots + 3 column-factor tables + g_last + misc
-constexpr uint32_t oI = oBar + 1024;               // 64 x 64 bf16 identity (B of (y)), 1024-aligned
-constexpr uint32_t kSmem = oI + 8192 + 1024;
+constexpr uint32_t oScal = oTf + 64 * LDF * 4;     // 4 slots x {beta, 2^g, 2^(g_last-g), g}[64], 4 x cf[64], g_last[4], misc
+constexpr uint32_t oBar = oScal + 4096 + 1024 + 256;
+constexpr uint32_t kSmem = oBar + 512 + 1024;
 static_assert(kSmem <= 232448, "shared memory");
 
 // TMEM columns
-// GP | [SX_0 | O_0] | [SX_1 | O_1] | Y^T, later U^T (same columns) | dS
-constexpr uint32_t cGP = 0, cSXO = 64 /* + 128 * slot */, cUT = 320, cY = 320, cDS = 384, kTmemCols = 512;
+// GP | [SX | O] slot 0 | [SX | O] slot 1 | A^T, B' | S (bf16) then R'^T (bf16)
+// dS of block c takes the SX half of its own slot (d < 64) and the O half of the other slot (d >= 64):
+// both are free between the chain's reads of SX_c and O_{c-1} and (b) of block c+1.
+constexpr uint32_t cGP = 0, cSXO = 64 /* + 128 * slot */, cAB = 320, cSR = 448, kTmemCols = 512;
 
 constexpr uint32_t kIdN64 = tc::idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t kIdN128 = tc::idesc_bf16(128, 128, 0, 0);
-constexpr uint32_t kIdN128Bmn = tc::idesc_bf16(128, 128, 0, 1);
-constexpr uint32_t kIdN64Amn = tc::idesc_bf16(128, 64, 1, 0);
+constexpr uint32_t kIdAT = tc::idesc_bf16(128, 64, 1, 1);   // X^T (MN-major A) x T_f (MN-major B)
+constexpr uint32_t kIdBP = tc::idesc_bf16(128, 64, 0, 1);   // P~ (K-major A) x T' (MN-major B)
 
-// barrier indices
+// barrier indices (arrival count 1 unless noted)
 enum {
-    B_FULL = 0,        // [2] TMA -> helpers
-    B_SFREE = 2,       // [2] (f) done -> producer
-    B_XQ = 4,          // helpers -> MMA (a)
-    B_ADONE = 5,       // (a) done -> helpers, local
-    B_GPFREE = 6,      // local read G and helpers read P (2 arrivals) -> MMA (a) of the next block
-    B_SCAL = 7,        // [3] helpers -> local, chain (scalar slot c % 3)
-    B_QSC = 10,        // Q~ ready -> MMA (b)
-    B_BDONE = 11,      // (b) done -> helpers, chain
-    B_XSC = 12,        // (unused)
-    B_RT = 13,         // R^T ready -> MMA (d)
-    B_TRDY = 14,       // [2] T ready -> MMA (d)
-    B_PRDY = 16,       // [2] P~ ready -> MMA (e)
-    B_DDONE = 18,      // (d) done -> chain
-    B_TFREE = 19,      // [2] (d) done -> local (T slot free)
-    B_URDY = 21,       // U^T ready -> MMA (e),(f)
-    B_EFDONE = 22,     // (e),(f) done -> chain
-    B_PFREE = 23,      // [2] (e) done -> local (P~ slot free)
-    B_SRDY = 25,       // S bf16 ready -> MMA (b)
-    B_OFREE = 26,      // [2] O slot read -> MMA (b)
-    B_FINAL = 28,      // MMA drain at exit
-    B_COUNT = 29
+    B_FULLXQ = 0,      // [3] TMA [X;Q] landed -> helpers
+    B_XQFREE = 3,      // [3] (b) done -> producer
+    B_FULLV = 6,       // [2] TMA V landed -> chain
+    B_VFREE = 8,       // [2] chain read V (8 warps) -> producer
+    B_XQRDY = 10,      // [3] helpers prepared the block -> MMA (a)
+    B_ADONE = 13,      // (a) done -> helpers, local
+    B_GPFREE = 14,     // local read G and helpers read P (2 arrivals) -> MMA (a) of the next block
+    B_SCAL = 15,       // [4] scalars of slot c % 4 ready -> local, chain
+    B_SCALFREE = 19,   // [4] chain done with scalar slot (8 warps) -> helpers
+    B_QSC = 23,        // [3] Q~ ready -> MMA (b)
+    B_PRDY = 26,       // P~ ready -> MMA (B')
+    B_TRDY = 27,       // T_f, T' ready -> MMA (A), (B')
+    B_ABDONE = 28,     // (A), (B') done -> chain, local (T tiles free), helpers (P~ tile free)
+    B_EARDY = 29,      // A^T, B' in shared memory (8 warps) -> MMA (e'), (f')
+    B_BDONE = 30,      // (b) done -> chain
+    B_RT = 31,         // R'^T in TMEM (8 warps) -> MMA (e'), (f')
+    B_EFDONE = 32,     // (e'), (f') done -> chain
+    B_UNUSED = 33,
+    B_SRDY = 34,       // S bf16 in TMEM, dS read, O of the previous block read (8 warps) -> MMA (b)
+    B_FINAL = 35,      // MMA drain at exit
+    B_COUNT = 36
 };
 
 __device__ __forceinline__ void named_bar(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Named barrier that also ORs a predicate over its participants: every thread gets the same answer.
+__device__ __forceinline__ bool named_bar_or(int id, int n, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %3, 0;\n\tbar.red.or.pred p, %1, %2, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(r)
+        : "r"(id), "r"(n), "r"((uint32_t)pred)
+        : "memory");
+    return r != 0;
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
@@ -252,15 +274,15 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 const __grid_constant__ CUtensorMap tmV, ChunkParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sS = sm + oS;
-    uint8_t *sRT = sm + oRT;
+    uint8_t *sTF = sm + oTF, *sTP = sm + oTP, *sPB = sm + oPB, *sA = sm + oA;
     float *sL = reinterpret_cast<float *>(sm + oL);
     float *sTf = reinterpret_cast<float *>(sm + oTf);
-    // Scalars of block c live in slot c % 3 (beta[64] gam[64] f[64] g2[64]); three slots, because the
-    // helpers prepare block c+1 while the chain may still read block c-1.
+    // Scalars of block c live in slot c % 4: beta[64] 2^g[64] 2^(g_last-g)[64] g[64]; the helpers
+    // prepare two blocks ahead of the chain, which still reads the slot of its own block.
     float *sScal = reinterpret_cast<float *>(sm + oScal);
-    float *sGL = sScal + 960;                              // g_last per slot (after 3 x cf[64])
-    float *sMisc = sScal + 964;                            // helper scan carry
+    float *sCF = sScal + 1024;                             // 4 x cf[64]
+    float *sGL = sScal + 1280;                             // g_last per slot
+    float *sMisc = sScal + 1284;                           // helper scan carry
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + B_COUNT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
@@ -272,7 +294,11 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     constexpr int D = 128;
 
     if (tid == 0) {
-        for (int i = 0; i < B_COUNT; ++i) tc::mbar_init(&bars[i], i == B_GPFREE ? 2 : 1);
+        for (int i = 0; i < B_COUNT; ++i) {
+            const bool chain_arrivals = (i >= B_VFREE && i < B_VFREE + 2) || (i >= B_SCALFREE && i < B_SCALFREE + 4) ||
+                                        i == B_EARDY || i == B_RT || i == B_SRDY;
+            tc::mbar_init(&bars[i], chain_arrivals ? kChainWarps : (i == B_GPFREE ? 2 : 1));
+        }
         *abort_flag = 0;
         tc::mbar_fence_init();
     }
@@ -281,147 +307,178 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         tc::tmem_relinquish();
     }
     for (int idx = tid; idx < 64 * LDF; idx += kThreads) sTf[idx] = 0.f;
-    for (int idx = tid; idx < 64 * 8; idx += kThreads) {  // identity, row e has a 1 at column e
-        const int e = idx >> 3, ch = idx & 7;
-        float v8[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) v8[k] = (8 * ch + k == e) ? 1.f : 0.f;
-        st_chunk8(sm + oI, tc::sw128_chunk(e, ch), v8);
-    }
-    tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tbase = *tslot;
 
-    // Leader-polled bounded wait, made uniform across a role with its named barrier.
+    // Leader-polled bounded wait; the outcome is made uniform across the role by its named barrier.
     auto role_wait = [&](uint64_t *bar, uint32_t parity, bool leader, int bar_id, int nthr) -> bool {
-        if (leader && !tc::mbar_wait(bar, parity, abort_flag, kWaitBudget)) *abort_flag = 1;
-        named_bar(bar_id, nthr);
-        return *abort_flag == 0;
+        bool failed = false;
+        if (leader && !tc::mbar_wait(bar, parity, abort_flag, kWaitBudget)) {
+            *abort_flag = 1;
+            failed = true;
+        }
+        return !named_bar_or(bar_id, nthr, failed);
+    };
+    // Lane-0-polled bounded wait, uniform across the warp.
+    auto warp_wait = [&](uint64_t *bar, uint32_t parity) -> bool {
+        int ok = 1;
+        if (lane == 0 && !tc::mbar_wait(bar, parity, abort_flag, kWaitBudget)) {
+            *abort_flag = 1;
+            ok = 0;
+        }
+        return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    };
+    // Per-warp arrival on a barrier that counts the chain's warps (after this warp's TMEM traffic).
+    auto warp_arrive = [&](uint64_t *bar) {
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar);
     };
 
     if (warp == 0) {
         // ================================================================ TMA producer
         if (lane == 0) {
-            for (int c = 0; c < nblk; ++c) {
-                const int s = c & 1;
-                if (c >= 2 && !tc::mbar_wait(&bars[B_SFREE + s], ((c >> 1) + 1) & 1, abort_flag, kWaitBudget)) {
+            int kx = 0, kv = 0;
+            long long idle_since = clock64();
+            while ((kx < nblk || kv < nblk) && !*abort_flag) {
+                bool progress = false;
+                if (kx < nblk && (kx < 3 || tc::mbar_test(&bars[B_XQFREE + kx % 3], ((kx / 3) - 1) & 1))) {
+                    uint8_t *dst = sm + oXQ + (kx % 3) * kXQ;
+                    uint64_t *fb = &bars[B_FULLXQ + kx % 3];
+                    const int t0 = kx * kBlk;
+                    tc::mbar_arrive_expect_tx(fb, kXQ);
+                    tc::tma_load_3d(dst + 0, &tmK, 0, t0 - 1, bh, fb);
+                    tc::tma_load_3d(dst + 16384, &tmK, 64, t0 - 1, bh, fb);
+                    tc::tma_load_3d(dst + 8192, &tmQ, 0, t0, bh, fb);
+                    tc::tma_load_3d(dst + 16384 + 8192, &tmQ, 64, t0, bh, fb);
+                    ++kx;
+                    progress = true;
+                }
+                if (kv < kx && (kv < 2 || tc::mbar_test(&bars[B_VFREE + (kv & 1)], ((kv >> 1) - 1) & 1))) {
+                    uint8_t *dst = sm + oV + (kv & 1) * kVst;
+                    uint64_t *fb = &bars[B_FULLV + (kv & 1)];
+                    const int t0 = kv * kBlk;
+                    tc::mbar_arrive_expect_tx(fb, kVst);
+                    tc::tma_load_3d(dst + 0, &tmV, 0, t0, bh, fb);
+                    tc::tma_load_3d(dst + 8192, &tmV, 64, t0, bh, fb);
+                    ++kv;
+                    progress = true;
+                }
+                if (progress) idle_since = clock64();
+                else if (clock64() - idle_since > kWaitBudget) {
                     *abort_flag = 1;
                     break;
                 }
-                uint8_t *stg = sm + oStage + s * kStage;
-                const int t0 = c * kBlk;
-                uint64_t *fb = &bars[B_FULL + s];
-                tc::mbar_arrive_expect_tx(fb, kStage);
-                tc::tma_load_3d(stg + 0, &tmK, 0, t0 - 1, bh, fb);
-                tc::tma_load_3d(stg + 16384, &tmK, 64, t0 - 1, bh, fb);
-                tc::tma_load_3d(stg + 8192, &tmQ, 0, t0, bh, fb);
-                tc::tma_load_3d(stg + 24576, &tmQ, 64, t0, bh, fb);
-                tc::tma_load_3d(stg + 32768, &tmV, 0, t0, bh, fb);
-                tc::tma_load_3d(stg + 40960, &tmV, 64, t0, bh, fb);
             }
-            // drain: every armed stage must have landed before the CTA can exit
+            // drain: every armed load must have landed before the CTA can exit
             const volatile int no_abort = 0;
-            for (int c = nblk - 2 < 0 ? 0 : nblk - 2; c < nblk; ++c)
-                tc::mbar_wait(&bars[B_FULL + (c & 1)], (c >> 1) & 1, &no_abort, kWaitBudget);
+            for (int c = kx - 3 < 0 ? 0 : kx - 3; c < kx; ++c)
+                tc::mbar_wait(&bars[B_FULLXQ + c % 3], (c / 3) & 1, &no_abort, kWaitBudget);
+            for (int c = kv - 2 < 0 ? 0 : kv - 2; c < kv; ++c)
+                tc::mbar_wait(&bars[B_FULLV + (c & 1)], (c >> 1) & 1, &no_abort, kWaitBudget);
         }
     } else if (warp == 1) {
-        // ================================================================ MMA issuer
-        if (lane == 0) {
+        // ================================================================ MMA issuer (whole warp, elected lane issues)
+        {
             // Descriptors are built once; a K step only moves the 14-bit start-address field
             // (address >> 4), which stays below 2^14 for every operand here, so a plain add is exact.
-            const uint64_t dS = tc::sdesc(tc::smem_u32(sS), 16, 1024);
-            const uint64_t dRT = tc::sdesc(tc::smem_u32(sRT), 16, 1024);
-            const uint64_t dI = tc::sdesc(tc::smem_u32(sm + oI), 16, 1024);
-            uint64_t dX[2], dXmn[2], dV[2], dT[2], dP[2];
+            uint64_t dXQ[3], dXmn[3];
 #pragma unroll
-            for (int st = 0; st < 2; ++st) {
-                const uint32_t a = tc::smem_u32(sm + oStage + st * kStage);
-                dX[st] = tc::sdesc(a, 16, 1024);            // [X;Q] K-major (also X as N=64 / N=128 B)
-                dXmn[st] = tc::sdesc(a, 16384, 1024);       // X as an MN-major B (dk atoms 16 KB apart)
-                dV[st] = tc::sdesc(a + 32768, 8192, 1024);  // V as an MN-major A (dv atoms 8 KB apart)
-                dT[st] = tc::sdesc(tc::smem_u32(sm + oT + st * 8192), 16, 1024);
-                dP[st] = tc::sdesc(tc::smem_u32(sm + oP + st * 8192), 16, 1024);
+            for (int u = 0; u < 3; ++u) {
+                const uint32_t a = tc::smem_u32(sm + oXQ + u * kXQ);
+                dXQ[u] = tc::sdesc(a, 16, 1024);      // [X;Q] K-major: A and B of (a), B of (b)
+                dXmn[u] = tc::sdesc(a, 16384, 1024);  // X as an MN-major A (d atoms 16 KB apart)
             }
+            const uint64_t dTF = tc::sdesc(tc::smem_u32(sTF), 8192, 1024);   // MN-major B, one N atom
+            const uint64_t dTP = tc::sdesc(tc::smem_u32(sTP), 8192, 1024);
+            const uint64_t dPB = tc::sdesc(tc::smem_u32(sPB), 16, 1024);     // [P~; B'] K-major
+            const uint64_t dBp = tc::sdesc(tc::smem_u32(sPB + 8192), 16, 1024);
+            const uint64_t dAt = tc::sdesc(tc::smem_u32(sA), 16, 1024);
             auto kmaj = [](int ks) -> uint64_t { return (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4); };
+            // every lane waits; the outcome is made uniform across the warp
             auto wait = [&](int b, uint32_t parity) -> bool {
-                if (!tc::mbar_wait(&bars[b], parity, abort_flag, kWaitBudget)) {
-                    *abort_flag = 1;
-                    return false;
+                const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars[b], parity, abort_flag, kWaitBudget));
+                if (!ok) *abort_flag = 1;
+                return ok;
+            };
+            auto test = [&](int b, uint32_t parity) -> bool {
+                return __all_sync(0xffffffffu, tc::mbar_test(&bars[b], parity));
+            };
+            // (a) of block na as soon as its slot is prepared and the GP columns are free;
+            // returns -1 on abort, else whether it issued.
+            int na = 0;
+            auto try_a = [&](bool block) -> int {
+                if (na >= nblk) return 0;
+                const uint32_t pr = (na / 3) & 1, pg = (na - 1) & 1;
+                if (block) {
+                    if (!wait(B_XQRDY + na % 3, pr) || (na > 0 && !wait(B_GPFREE, pg))) return -1;
+                } else if (!test(B_XQRDY + na % 3, pr) || (na > 0 && !test(B_GPFREE, pg))) {
+                    return 0;
                 }
-                return true;
-            };
-            // (a): [X;Q] X^T -> G (lanes 0-63), P (lanes 64-127)
-            auto issue_a = [&](int c) {
-                const uint64_t d = dX[c & 1];
+                tc::fence_after_sync();
+                const uint64_t d = dXQ[na % 3];
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) tc::mma_bf16(tbase + cGP, d + kmaj(ks), d + kmaj(ks), kIdN64, ks > 0);
-                tc::mma_commit(&bars[B_ADONE]);
+                for (int ks = 0; ks < 8; ++ks) tc::mma_bf16_elect(tbase + cGP, d + kmaj(ks), d + kmaj(ks), kIdN64, ks > 0);
+                tc::mma_commit_elect(&bars[B_ADONE]);
+                ++na;
+                return 1;
             };
-            // (y): Y^T = V^T I (V read as an MN-major A operand of the stage tile)
-            auto issue_y = [&](int c) {
-                const uint64_t d = dV[c & 1];
+            // (A) A^T = X^T T_f and (B') B' = P~ T' of block j into the AB columns (free once the chain
+            // copied A^T, B' of block j-1 to shared memory)
+            auto issue_AB = [&](int j) -> bool {
+                if (!(wait(B_TRDY, j & 1) && wait(B_PRDY, j & 1) && (j < 1 || wait(B_EARDY, (j - 1) & 1))))
+                    return false;
+                tc::fence_after_sync();
+                const int u = j % 3;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16(tbase + cY, d + (uint64_t)(ks * 128), dI + (uint64_t)(ks * 2), kIdN64Amn, ks > 0);
+                    tc::mma_bf16_elect(tbase + cAB, dXmn[u] + (uint64_t)(ks * 128), dTF + (uint64_t)(ks * 128), kIdAT, ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16_elect(tbase + cAB + 64, dPB + (uint64_t)(ks * 2), dTP + (uint64_t)(ks * 128), kIdBP, ks > 0);
+                tc::mma_commit_elect(&bars[B_ABDONE]);
+                return true;
             };
-            // Program order per block c (each wait parks this thread until its inputs are ready):
-            //   (b)_c, then (a)_{c+1} (runs while the chain forms R_c), (d)_c, (e)(f)_c, then (y)_{c+1}
-            //   (its columns are free once U^T_c has been read, which (e)(f)_c's inputs imply).
-            bool ok = nblk > 0 && wait(B_XQ, 0);
-            if (ok) {
-                issue_a(0);
-                issue_y(0);
-            }
+            bool ok = nblk == 0 || (try_a(true) > 0 && issue_AB(0));
             for (int c = 0; c < nblk && ok; ++c) {
-                const int s = c & 1;
-                // (b): S [X; Q~]^T in one N = 128 pass -> [SX | O] of slot s
-                if (!(ok = wait(B_QSC, c & 1) && wait(B_SRDY, c & 1) &&
-                           (c < 2 || wait(B_OFREE + s, ((c >> 1) + 1) & 1))))
-                    break;
+                const int s = c & 1, u = c % 3;
+                // (b) [S X^T | S Q~^T] -> [SX | O] of slot s, S from TMEM
+                if (!(ok = wait(B_SRDY, c & 1) && wait(B_QSC + u, (c / 3) & 1))) break;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    tc::mma_bf16(tbase + cSXO + 128 * s, dS + kmaj(ks), dX[s] + kmaj(ks), kIdN128, ks > 0);
-                tc::mma_commit(&bars[B_BDONE]);
-                // (a) of the next block
-                if (c + 1 < nblk) {
-                    if (!(ok = wait(B_XQ, (c + 1) & 1) && wait(B_GPFREE, c & 1))) break;
-                    tc::fence_after_sync();
-                    issue_a(c + 1);
-                }
-                // (d): U^T = R^T T'^T
-                if (REG) {
-                    if (!(ok = wait(B_RT, c & 1) && wait(B_TRDY + s, (c >> 1) & 1))) break;
-                    tc::fence_after_sync();
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        tc::mma_bf16(tbase + cUT, dRT + (uint64_t)(ks * 2), dT[s] + (uint64_t)(ks * 2), kIdN64, ks > 0);
-                    tc::mma_commit(&bars[B_DDONE]);
-                    tc::mma_commit(&bars[B_TFREE + s]);
-                }
-                // (e) O += U^T P~^T and (f) dS = U^T X~
-                if (!(ok = wait(B_URDY, c & 1) && wait(B_PRDY + s, (c >> 1) & 1))) break;
+                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dXQ[u] + kmaj(ks), kIdN128, ks > 0);
+                tc::mma_commit_elect(&bars[B_BDONE]);
+                tc::mma_commit_elect(&bars[B_XQFREE + u]);
+                // state-independent work of later blocks runs while the chain forms R'^T
+                while (ok && na <= c + 1 && na < nblk) ok = try_a(true) >= 0;
+                if (!ok) break;
+                if (c + 1 < nblk && !(ok = issue_AB(c + 1))) break;
+                if ((ok = try_a(false) >= 0) == false) break;
+                // (e') O^T += R'^T B'^T and (f') dS = R'^T A in two N = 64 halves, R'^T from TMEM
+                if (!(ok = wait(B_RT, c & 1) && wait(B_EARDY, c & 1))) break;
                 tc::fence_after_sync();
+                const uint32_t dlo = tbase + cSXO + 128 * s, dhi = tbase + cSXO + 128 * (s ^ 1) + 64;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16(tbase + cSXO + 128 * s + 64, dRT + (uint64_t)(ks * 2), dP[s] + (uint64_t)(ks * 2),
-                                 kIdN64, 1);
+                    tc::mma_bf16_ts_elect(dlo + 64, tbase + cSR + 8 * ks, dBp + (uint64_t)(ks * 2), kIdN64, 1);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16(tbase + cDS, dRT + (uint64_t)(ks * 2), dXmn[s] + (uint64_t)(ks * 128), kIdN128Bmn,
-                                 ks > 0);
-                tc::mma_commit(&bars[B_EFDONE]);
-                tc::mma_commit(&bars[B_PFREE + s]);
-                tc::mma_commit(&bars[B_SFREE + s]);
-                // (y) of the next block (its tiles landed before xq_ready of that block)
-                if (c + 1 < nblk) issue_y(c + 1);
+                    tc::mma_bf16_ts_elect(dlo, tbase + cSR + 8 * ks, dAt + (uint64_t)(ks * 2), kIdN64, ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16_ts_elect(dhi, tbase + cSR + 8 * ks, dAt + (uint64_t)(512 + ks * 2), kIdN64, ks > 0);
+                tc::mma_commit_elect(&bars[B_EFDONE]);
+                if ((ok = try_a(false) >= 0) == false) break;
             }
+            if (!ok) *abort_flag = 1;
             // drain every MMA issued so far
-            tc::mma_commit(&bars[B_FINAL]);
+            tc::mma_commit_elect(&bars[B_FINAL]);
             const volatile int no_abort = 0;
             tc::mbar_wait(&bars[B_FINAL], 0, &no_abort, kWaitBudget);
+            __syncwarp();
         }
     } else if (warp < 4) {
         // ================================================================ helpers (64 threads)
@@ -435,14 +492,15 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             ge = t < T ? eta_h[t] : 0.f;
         };
         auto prep = [&](int c) -> bool {   // block c: x_1 patch, norms, step sizes, decay tables
-            const int s = c & 1, u = c % 3;
-            uint8_t *stg = sm + oStage + s * kStage;
-            if (!role_wait(&bars[B_FULL + s], (c >> 1) & 1, leader, 1, 64)) return false;
+            const int u3 = c % 3, u4 = c % 4;
+            uint8_t *xq = sm + oXQ + u3 * kXQ;
+            if (c >= 4 && !role_wait(&bars[B_SCALFREE + u4], ((c >> 2) - 1) & 1, leader, 1, 64)) return false;
+            if (!role_wait(&bars[B_FULLXQ + u3], (c / 3) & 1, leader, 1, 64)) return false;
             const int t0 = c * kBlk, nval = min(kBlk, T - t0);
             if (c == 0 && p.k_prev && ht < 16) {
                 const uint4 v = *reinterpret_cast<const uint4 *>(
                     reinterpret_cast<const __nv_bfloat16 *>(p.k_prev) + (size_t)bh * D + ht * 8);
-                *reinterpret_cast<uint4 *>(stg + (ht >> 3) * 16384 + (ht & 7) * 16) = v;
+                *reinterpret_cast<uint4 *>(xq + (ht >> 3) * 16384 + (ht & 7) * 16) = v;
                 tc::fence_proxy_async();
             }
             named_bar(1, 64);
@@ -451,8 +509,8 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             for (int a = 0; a < 2; ++a)
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(stg + a * 16384 + tc::sw128_chunk(ht, ch));
-                    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+                    const uint4 w = *reinterpret_cast<const uint4 *>(xq + a * 16384 + tc::sw128_chunk(ht, ch));
+                    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&w);
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const float2 f = __bfloat1622float2(h2[k]);
@@ -470,32 +528,38 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             if (ht == 31) sMisc[0] = la;
             named_bar(1, 64);
             if (ht >= 32) la += sMisc[0];
-            float *sc = sScal + u * 256;
+            float *sc = sScal + u4 * 256;
             sc[ht] = bt;
-            sc[128 + ht] = 0.f;  // placeholder, f filled below
-            sc[192 + ht] = la;
             sc[64 + ht] = exp2f(la);
+            sc[192 + ht] = la;
             named_bar(1, 64);
             const float gl = sc[192 + nval - 1];
             sc[128 + ht] = exp2f(gl - la);
-            sScal[3 * 256 + 64 * u + ht] = exp2f(sc[192 + (ht | 15)] - la);
-            if (leader) sGL[u] = gl;
+            sCF[64 * u4 + ht] = exp2f(sc[192 + (ht | 15)] - la);
+            if (leader) sGL[u4] = gl;
             named_bar(1, 64);
             if (leader) {
-                mbar_arrive(&bars[B_SCAL + u]);
-                mbar_arrive(&bars[B_XQ]);
+                mbar_arrive(&bars[B_SCAL + u4]);
+                mbar_arrive(&bars[B_XQRDY + u3]);
             }
             return true;
         };
-        if (nblk > 0) load_gates(0);
-        bool ok = nblk > 0 ? prep(0) : true;
+        bool ok = true;
+        if (nblk > 0) {
+            load_gates(0);
+            ok = prep(0);
+        }
+        if (ok && nblk > 1) {
+            load_gates(1);
+            ok = prep(1);
+        }
         for (int c = 0; c < nblk && ok; ++c) {
-            const int s = c & 1;
-            if (c + 1 < nblk) load_gates(c + 1);  // in flight while block c's Q is scaled
-            uint8_t *stg = sm + oStage + s * kStage;
-            const float *sc = sScal + (c % 3) * 256;
+            const int u3 = c % 3;
+            if (c + 2 < nblk) load_gates(c + 2);  // in flight while block c is handled
+            uint8_t *xq = sm + oXQ + u3 * kXQ;
+            const float *sc = sScal + (c % 4) * 256;
             if (!(ok = role_wait(&bars[B_ADONE], c & 1, leader, 1, 64))) break;
-            // P of query row i = ht from TMEM lanes 64..127 (this pair of warps' quarters), released at once
+            // P of query row i = ht from TMEM lanes 64..127 (this pair of warps' quarters)
             tc::fence_after_sync();
             float v[64];
             {
@@ -508,19 +572,17 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             }
             tc::fence_before_sync();
             // Q~ = diag(2^g) Q once (a) no longer needs Q
-            scale_row(stg, 64 + ht, sc[64 + ht]);
+            scale_row(xq, 64 + ht, sc[64 + ht]);
             tc::fence_proxy_async();
             named_bar(1, 64);
             if (leader) {
                 mbar_arrive(&bars[B_GPFREE]);
-                mbar_arrive(&bars[B_QSC]);
+                mbar_arrive(&bars[B_QSC + u3]);
             }
-            // next block's prep overlaps this block's chain (and unblocks (a) of the next block)
-            if (c + 1 < nblk && !(ok = prep(c + 1))) break;
-            // P~ = Gamma o P into P~ slot s, once (e) of block c-2 has released it
-            if (c >= 2 && !(ok = role_wait(&bars[B_PFREE + s], ((c >> 1) + 1) & 1, leader, 1, 64))) break;
+            // P~ = Gamma o P (inclusive), packed to bf16 while (B') of the previous block still reads the tile
+            uint32_t pk[32];
             {
-                const float *g2 = sc + 192, *cf = sScal + 3 * 256 + 64 * (c % 3);
+                const float *g2 = sc + 192, *cf = sCF + 64 * (c % 4);
                 const int i = ht, rb = i >> 4;
                 const float gri = g2[i];
                 float fac[4], gd[16];
@@ -535,24 +597,24 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                     const float f = exp2f(fminf(gri - g2[j], 0.f));
                     gd[k] = j <= i ? f : 0.f;
                 }
-                uint8_t *sP = sm + oP + s * 8192;
 #pragma unroll
-                for (int jb = 0; jb < 4; ++jb) {
-                    const bool below = jb < rb, diag = jb == rb;
-                    float pv[16];
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const int j = 16 * jb + k;
-                        const float gm = below ? fac[jb] * cf[j] : (diag ? gd[k] : 0.f);
-                        pv[k] = gm * v[j];
-                    }
-                    st_chunk8(sP, tc::sw128_chunk(i, 2 * jb), pv);
-                    st_chunk8(sP, tc::sw128_chunk(i, 2 * jb + 1), pv + 8);
+                for (int j = 0; j < 64; j += 2) {
+                    const int jb = j >> 4;
+                    const float g0 = jb < rb ? fac[jb] * cf[j] : (jb == rb ? gd[j & 15] : 0.f);
+                    const float g1 = jb < rb ? fac[jb] * cf[j + 1] : (jb == rb ? gd[(j + 1) & 15] : 0.f);
+                    pk[j >> 1] = pack_bf16x2(g0 * v[j], g1 * v[j + 1]);
                 }
-                tc::fence_proxy_async();
-                named_bar(1, 64);
-                if (leader) mbar_arrive(&bars[B_PRDY + s]);
             }
+            if (c >= 1 && !(ok = role_wait(&bars[B_ABDONE], (c - 1) & 1, leader, 1, 64))) break;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<uint4 *>(sPB + tc::sw128_chunk(ht, ch)) =
+                    make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+            tc::fence_proxy_async();
+            named_bar(1, 64);
+            if (leader) mbar_arrive(&bars[B_PRDY]);
+            // the block after next: its slot frees once (b) of block c-1 is done
+            if (c + 2 < nblk && !(ok = prep(c + 2))) break;
         }
     } else if (warp < 8) {
         // ================================================================ local (128 threads)
@@ -561,12 +623,12 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         const bool leader = lt == 0;
         const uint32_t tl = tbase + ((uint32_t)(32 * lw) << 16);
         for (int c = 0; c < nblk; ++c) {
-            const int s = c & 1;
+            const int u4 = c % 4;
             if (!role_wait(&bars[B_ADONE], c & 1, leader, 2, 128)) break;
-            if (!role_wait(&bars[B_SCAL + c % 3], (c / 3) & 1, leader, 2, 128)) break;
+            if (!role_wait(&bars[B_SCAL + u4], (c >> 2) & 1, leader, 2, 128)) break;
             tc::fence_after_sync();
-            const float *sc = sScal + (c % 3) * 256;
-            if (lw < 2) {                                   // G rows r = 0..63 -> L (regression family)
+            const float *sc = sScal + u4 * 256;
+            if (REG && lw < 2) {                            // G rows r = 0..63 -> L
                 float v[64];
                 {
                     float h0[32], h1[32];
@@ -575,71 +637,104 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 #pragma unroll
                     for (int j = 0; j < 32; ++j) { v[j] = h0[j]; v[32 + j] = h1[j]; }
                 }
-                tc::fence_before_sync();
-                if (REG) {
-                    // Decay factors 2^(g_r - g_j), j < r: below the 16x16 diagonal blocks they factor
-                    // through the last index of column block jb, 2^(g_r - g_{16jb+15}) * cf[j] with
-                    // cf[j] = 2^(g_{16jb+15} - g_j) (a helper table), both in (0, 1]; inside the
-                    // diagonal block they are formed directly. Selects only, no divergent branches.
-                    const float *g2 = sc + 192, *cf = sScal + 3 * 256 + 64 * (c % 3);
-                    const int rb = r >> 4;
-                    const float gri = g2[r], be = sc[r];
-                    float fac[4], gd[16];
+                // Decay factors 2^(g_r - g_j), j < r: below the 16x16 diagonal blocks they factor
+                // through the last index of column block jb, 2^(g_r - g_{16jb+15}) * cf[j] with
+                // cf[j] = 2^(g_{16jb+15} - g_j) (a helper table), both in (0, 1]; inside the
+                // diagonal block they are formed directly. Selects only, no divergent branches.
+                const float *g2 = sc + 192, *cf = sCF + 64 * u4;
+                const int rb = r >> 4;
+                const float gri = g2[r], be = sc[r];
+                float fac[4], gd[16];
 #pragma unroll
-                    for (int jb = 0; jb < 4; ++jb) {
-                        const float f = exp2f(fminf(gri - g2[16 * jb + 15], 0.f));
-                        fac[jb] = jb < rb ? be * f : 0.f;
+                for (int jb = 0; jb < 4; ++jb) {
+                    const float f = exp2f(fminf(gri - g2[16 * jb + 15], 0.f));
+                    fac[jb] = jb < rb ? be * f : 0.f;
+                }
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const int j = 16 * rb + k;
+                    const float f = exp2f(fminf(gri - g2[j], 0.f));
+                    gd[k] = j < r ? be * f : 0.f;
+                }
+                float *Lr = sL + r * LDF;
+#pragma unroll
+                for (int j0 = 0; j0 < 64; j0 += 4) {
+                    float w4[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int j = j0 + k, jb = j >> 4;
+                        const float gm = jb < rb ? fac[jb] * cf[j] : (jb == rb ? gd[j & 15] : 0.f);
+                        w4[k] = gm * v[j];
                     }
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const int j = 16 * rb + k;
-                        const float f = exp2f(fminf(gri - g2[j], 0.f));
-                        gd[k] = j < r ? be * f : 0.f;
-                    }
-                    float *Lr = sL + r * LDF;
-#pragma unroll
-                    for (int j0 = 0; j0 < 64; j0 += 4) {
-                        float w4[4];
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const int j = j0 + k, jb = j >> 4;
-                            const float gm = jb < rb ? fac[jb] * cf[j] : (jb == rb ? gd[j & 15] : 0.f);
-                            w4[k] = gm * v[j];
-                        }
-                        *reinterpret_cast<float4 *>(Lr + j0) = make_float4(w4[0], w4[1], w4[2], w4[3]);
-                    }
+                    *reinterpret_cast<float4 *>(Lr + j0) = make_float4(w4[0], w4[1], w4[2], w4[3]);
                 }
             }
+            tc::fence_before_sync();
             named_bar(2, 128);
             if (leader) mbar_arrive(&bars[B_GPFREE]);
-            if (*abort_flag) break;
-            if (REG) {
-                solve_local(sL, sTf, lt, lw, lane);
-                if (c >= 2 && !role_wait(&bars[B_TFREE + s], ((c >> 1) + 1) & 1, leader, 2, 128)) break;
-                uint8_t *sT = sm + oT + s * 8192;
+            if (REG) solve_local(sL, sTf, lt, lw, lane);
+            // T_f = diag(2^(g_last - g)) T diag(beta), T' = T diag(beta) once (A), (B') of c-1 are done
+            if (c >= 1 && !role_wait(&bars[B_ABDONE], (c - 1) & 1, leader, 2, 128)) break;
+            {
                 const int rr = lt >> 1, ch0 = 4 * (lt & 1);
+                const float fr = sc[128 + rr];
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
-                    const float4 x0 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + 8 * (ch0 + cc));
-                    const float4 x1 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + 8 * (ch0 + cc) + 4);
-                    const float *bcol = sScal + (c % 3) * 256 + 8 * (ch0 + cc);  // beta of columns
-                    const float t8[8] = {x0.x * bcol[0], x0.y * bcol[1], x0.z * bcol[2], x0.w * bcol[3],
-                                         x1.x * bcol[4], x1.y * bcol[5], x1.z * bcol[6], x1.w * bcol[7]};
-                    st_chunk8(sT, tc::sw128_chunk(rr, ch0 + cc), t8);
+                    const int j0 = 8 * (ch0 + cc);
+                    float t8[8], f8[8];
+                    if (REG) {
+                        const float4 x0 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + j0);
+                        const float4 x1 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + j0 + 4);
+                        t8[0] = x0.x; t8[1] = x0.y; t8[2] = x0.z; t8[3] = x0.w;
+                        t8[4] = x1.x; t8[5] = x1.y; t8[6] = x1.z; t8[7] = x1.w;
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) t8[k] = (j0 + k == rr) ? 1.f : 0.f;
+                    }
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        t8[k] *= sc[j0 + k];  // beta of the column
+                        f8[k] = fr * t8[k];
+                    }
+                    st_chunk8(sTP, tc::sw128_chunk(rr, ch0 + cc), t8);
+                    st_chunk8(sTF, tc::sw128_chunk(rr, ch0 + cc), f8);
                 }
-                tc::fence_proxy_async();
-                named_bar(2, 128);
-                if (leader) mbar_arrive(&bars[B_TRDY + s]);
             }
+            tc::fence_proxy_async();
+            named_bar(2, 128);
+            if (leader) mbar_arrive(&bars[B_TRDY]);
         }
     } else {
         // ================================================================ chain (256 threads)
         const int ct = tid - 256;
         const int qd = warp & 3, hf = (warp - 8) >> 2;
-        const int row = 32 * qd + lane;    // TMEM lane = value row
-        const bool leader = ct == 0;
+        const int row = 32 * qd + lane;    // TMEM lane = value row (and key row d of A^T)
         const uint32_t tl = tbase + ((uint32_t)(32 * qd) << 16);
-        float S[64];
+        float S[64];                       // fp32 state, row `row`, columns 64 hf ..
+        auto store_S = [&]() {             // bf16 pairs of this thread's 64 columns -> TMEM A operand
+            uint32_t pk[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(S[2 * j], S[2 * j + 1]);
+            tc::tmem_st32(tl + cSR + 32 * hf, pk);
+        };
+        // O^T of block c (TMEM slot c & 1) to global memory: lane pairs (2k, 2k+1) hold neighbouring
+        // value rows; the even lane stores the pair for even tokens, the odd lane for odd tokens.
+        auto store_out = [&](int c) {
+            const int t0 = c * kBlk, nval = min(kBlk, T - t0);
+            float v[32];
+            tc::tmem_ld32(tl + cSXO + 128 * (c & 1) + 64 + 32 * hf, v);
+            const bool odd = lane & 1;
+            __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.o) + ((size_t)bh * T + t0) * D + (row & ~1);
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                const float mine = odd ? v[j + 1] : v[j];
+                const float give = odd ? v[j] : v[j + 1];
+                const float other = __shfl_xor_sync(0xffffffffu, give, 1);
+                const int i = 32 * hf + j + (odd ? 1 : 0);
+                const float lo = odd ? other : mine, hi = odd ? mine : other;
+                if (i < nval) *reinterpret_cast<uint32_t *>(o + (size_t)i * D) = pack_bf16x2(lo, hi);
+            }
+        };
         {
             const float *S0 = p.S0 ? p.S0 + ((size_t)bh * D + row) * D + 64 * hf : nullptr;
 #pragma unroll
@@ -647,116 +742,76 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 const float4 x = S0 ? *reinterpret_cast<const float4 *>(S0 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
                 S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
             }
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) st_chunk8(sS + hf * 16384, tc::sw128_chunk(row, ch), S + 8 * ch);
-            tc::fence_proxy_async();
-            named_bar(3, 256);
-            if (leader) mbar_arrive(&bars[B_SRDY]);
+            store_S();
+            warp_arrive(&bars[B_SRDY]);
         }
         bool ok = true;
         for (int c = 0; c < nblk; ++c) {
-            const int s = c & 1, t0 = c * kBlk, nval = min(kBlk, T - t0);
-            if (!(ok = role_wait(&bars[B_BDONE], c & 1, leader, 3, 256))) break;
-            if (!(ok = role_wait(&bars[B_SCAL + c % 3], (c / 3) & 1, leader, 3, 256))) break;
+            const int s = c & 1, u4 = c % 4;
+            // A^T (rows d, columns i) and B' (rows i < 64) from TMEM to their shared-memory tiles
+            if (!(ok = warp_wait(&bars[B_ABDONE], c & 1))) break;
             tc::fence_after_sync();
-            const float *sc = sScal + (c % 3) * 256;
-            const float gl = sGL[c % 3];
-            // R^T = Y^T - SX diag(2^g) (regression) or U^T = Y^T diag(beta) (inner product),
-            // 16 columns at a time, both operands from TMEM
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float y[16], v[16], rv[16];
-                const int e0 = 32 * hf + 16 * hh;
-                tc::tmem_ld16(tl + cY + e0, y);
-                if (REG) tc::tmem_ld16(tl + cSXO + 128 * s + e0, v);
-#pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    rv[j] = REG ? y[j] - sc[64 + e0 + j] * v[j] : sc[e0 + j] * y[j];
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc)
-                    st_chunk8(sRT, tc::sw128_chunk(row, 4 * hf + 2 * hh + cc), rv + 8 * cc);
-            }
-            tc::fence_proxy_async();
-            tc::fence_before_sync();
-            named_bar(3, 256);
-            if (REG && leader) mbar_arrive(&bars[B_RT]);
-            // X~ = diag(2^(g_last - g)) X in place (X is no longer needed unscaled once (b) is done),
-            // so that (f) forms sum_e 2^(g_last - g_e) u_e x_e^T directly; done while (d) runs.
             {
-                const int xr = ct >> 2, part = ct & 3;
-                uint8_t *xt = sm + oStage + s * kStage + (part >> 1) * 16384;
-                const float f = sc[128 + xr];
+                float v[32];
+                tc::tmem_ld32(tl + cAB + 32 * hf, v);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    uint4 *pp = reinterpret_cast<uint4 *>(xt + tc::sw128_chunk(xr, 4 * (part & 1) + k));
-                    uint4 u = *pp;
-                    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+                for (int cc = 0; cc < 4; ++cc) st_chunk8(sA, tc::sw128_chunk(row, 4 * hf + cc), v + 8 * cc);
+                if (qd < 2) {
+                    tc::tmem_ld32(tl + cAB + 64 + 32 * hf, v);
 #pragma unroll
-                    for (int q2 = 0; q2 < 4; ++q2) {
-                        const float2 x2 = __bfloat1622float2(h[q2]);
-                        h[q2] = __floats2bfloat162_rn(x2.x * f, x2.y * f);
-                    }
-                    *pp = u;
+                    for (int cc = 0; cc < 4; ++cc)
+                        st_chunk8(sPB + 8192, tc::sw128_chunk(row, 4 * hf + cc), v + 8 * cc);
                 }
             }
-            if (!REG) {
-                tc::fence_proxy_async();
-                named_bar(3, 256);
-                if (leader) mbar_arrive(&bars[B_URDY]);
-            }
-            if (REG) {
-                if (!(ok = role_wait(&bars[B_DDONE], c & 1, leader, 3, 256))) break;
-                tc::fence_after_sync();
-                float v[32];
-                tc::tmem_ld32(tl + cUT + 32 * hf, v);
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) st_chunk8(sRT, tc::sw128_chunk(row, 4 * hf + cc), v + 8 * cc);
-                tc::fence_proxy_async();
-                tc::fence_before_sync();
-                named_bar(3, 256);
-                if (leader) mbar_arrive(&bars[B_URDY]);
-            }
-            // state update: S <- 2^g_last S + dS, then its bf16 copy for (b) of the next block
-            if (!(ok = role_wait(&bars[B_EFDONE], c & 1, leader, 3, 256))) break;
+            tc::fence_proxy_async();
+            warp_arrive(&bars[B_EARDY]);
+            // outputs of the previous block (off the chain; their columns take dS of this block)
+            if (c >= 1) store_out(c - 1);
+            // R'^T = Y^T - SX diag(2^g) (regression) or Y^T (inner product), bf16 into TMEM
+            if (!(ok = warp_wait(&bars[B_BDONE], c & 1) && warp_wait(&bars[B_SCAL + u4], (c >> 2) & 1) &&
+                       warp_wait(&bars[B_FULLV + s], (c >> 1) & 1)))
+                break;
             tc::fence_after_sync();
             {
-                const float dl = exp2f(gl);
+                const float *sc = sScal + u4 * 256;
+                const uint8_t *sV = sm + oV + s * kVst;
+                float x[32];
+                if (REG) tc::tmem_ld32(tl + cSXO + 128 * s + 32 * hf, x);
+                uint32_t pk[16];
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    const int i = 32 * hf + j;
+                    const float y0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sV + tc::sw128_off(i, row, 64)));
+                    const float y1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sV + tc::sw128_off(i + 1, row, 64)));
+                    const float r0 = REG ? y0 - sc[64 + i] * x[j] : y0;
+                    const float r1 = REG ? y1 - sc[64 + i + 1] * x[j + 1] : y1;
+                    pk[j >> 1] = pack_bf16x2(r0, r1);
+                }
+                tc::tmem_st16(tl + cSR + 16 * hf, pk);
+            }
+            warp_arrive(&bars[B_RT]);
+            if (lane == 0) mbar_arrive(&bars[B_VFREE + s]);
+            // state update: S <- 2^g_last S + dS, then its bf16 copy for (b) of the next block
+            if (!(ok = warp_wait(&bars[B_EFDONE], c & 1))) break;
+            tc::fence_after_sync();
+            {
+                const float dl = exp2f(sGL[u4]);
+                const uint32_t cds = hf == 0 ? cSXO + 128 * s : cSXO + 128 * (s ^ 1) + 64;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float v[32];
-                    tc::tmem_ld32(tl + cDS + 64 * hf + 32 * hh, v);
+                    tc::tmem_ld32(tl + cds + 32 * hh, v);
 #pragma unroll
                     for (int j = 0; j < 32; ++j) S[32 * hh + j] = dl * S[32 * hh + j] + v[j];
                 }
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) st_chunk8(sS + hf * 16384, tc::sw128_chunk(row, ch), S + 8 * ch);
             }
-            tc::fence_proxy_async();
+            store_S();
+            warp_arrive(&bars[B_SRDY]);
+            if (lane == 0) mbar_arrive(&bars[B_SCALFREE + u4]);
+        }
+        if (ok && nblk > 0 && !*abort_flag) {
+            store_out(nblk - 1);
             tc::fence_before_sync();
-            named_bar(3, 256);
-            if (leader) mbar_arrive(&bars[B_SRDY]);
-            // outputs of this block (off the critical chain)
-            {
-                float v[32];
-                tc::tmem_ld32(tl + cSXO + 128 * s + 64 + 32 * hf, v);
-                // lane pairs (2k, 2k+1) hold neighbouring value rows: the even lane stores the pair for
-                // even tokens, the odd lane for odd tokens, as 4-byte bf16x2 stores
-                const bool odd = lane & 1;
-                __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.o) + ((size_t)bh * T + t0) * D + (row & ~1);
-#pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    const float mine = odd ? v[j + 1] : v[j];
-                    const float give = odd ? v[j] : v[j + 1];
-                    const float other = __shfl_xor_sync(0xffffffffu, give, 1);
-                    const int i = 32 * hf + j + (odd ? 1 : 0);
-                    const float lo = odd ? other : mine, hi = odd ? mine : other;
-                    if (i < nval)
-                        *reinterpret_cast<uint32_t *>(o + (size_t)i * D) = pack_bf16x2(lo, hi);
-                }
-            }
-            tc::fence_before_sync();
-            named_bar(3, 256);
-            if (leader) mbar_arrive(&bars[B_OFREE + s]);
         }
         if (ok && !*abort_flag) {
             if (p.S_out) {
