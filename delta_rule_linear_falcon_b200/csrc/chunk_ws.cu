@@ -8,7 +8,7 @@
 //   T' = T diag(beta),  T_f = diag(2^(g_last - g)) T',  A = T_f^T X,  B' = P~ T'
 // (all independent of the state), one block is
 //   R'^T = Y^T - (S X^T) diag(2^g)                          (regression; Y^T for inner product)
-//   O^T  = S Q~^T + R'^T B'^T,   S <- 2^g_last S + R'^T A.
+//   O^T  = (S Q^T) diag(2^g) + R'^T B'^T,   S <- 2^g_last S + R'^T A.
 // For the inner-product rule T = I, so T_f and T' are diagonal and no solve runs.
 //
 // One CTA of 512 threads per (b, h); the state-independent work of later blocks
@@ -18,16 +18,18 @@
 //   warp 1      MMA issuer (one thread):
 //                 (a)  [X;Q] X^T -> G (lanes 0-63), P (lanes 64-127)
 //                 (A)  A^T = X^T T_f   and  (B')  B' = [P~; *] T'        (state independent)
-//                 (b)  [S X^T | S Q~^T] with S (bf16) read from tensor memory
-//                 (e') O^T += R'^T B'^T   (f') dS = R'^T A   with R'^T (bf16) from tensor memory
+//                 (b)  [S X^T | S Q^T] with S (bf16) read from tensor memory
+//                 (e') R'^T B'^T   (f') dS = R'^T A   with R'^T (bf16) from tensor memory
 //               The chain's groups go first; the state-independent ones of later blocks are issued
 //               right behind them, so they run while the chain warps work on the results.
-//   warps 2-3   helpers: x_1 patch, key norms, step sizes, cumulative log2 decay and its
-//               tables; P~ = Gamma o P from TMEM lanes 64-127; Q~ = diag(2^g) Q
-//   warps 4-7   local: L = diag(beta)(Gamma o G) (fp32) from TMEM lanes 0-63,
+//   warps 2-3   helpers: x_1 patch, cumulative log2 decay and its tables; P~ = Gamma o P
+//               from TMEM lanes 64-127
+//   warps 4-7   local: step sizes from the key norms on the diagonal of G,
+//               L = diag(beta)(Gamma o G) (fp32) from TMEM lanes 0-63,
 //               T = (I + L)^-1 (fp32, tensor-core tf32 block products), T_f and T' in bf16
 //   warps 8-15  chain: A^T, B' from TMEM to shared memory; R'^T (bf16 into TMEM); the fp32
-//               state S <- 2^g_last S + dS (in registers) and its bf16 copy in TMEM; O out
+//               state S <- 2^g_last S + dS (in registers) and its bf16 copy in TMEM;
+//               O = 2^g o (Q S^T) + B' R' out
 // Every decay factor is 2^(g_i - g_j) with i >= j (never a quotient of
 // cumulative products). Every wait is bounded; a timeout is recorded in the
 // device error word and all roles unwind.
@@ -64,9 +66,10 @@ constexpr uint32_t kSmem = oBar + 512 + 1024;
 static_assert(kSmem <= 232448, "shared memory");
 
 // TMEM columns
-// GP | [SX | O] slot 0 | [SX | O] slot 1 | A^T, B' | S (bf16) then R'^T (bf16)
-// dS of block c takes the SX half of its own slot (d < 64) and the O half of the other slot (d >= 64):
-// both are free between the chain's reads of SX_c and O_{c-1} and (b) of block c+1.
+// GP | slot 0 | slot 1 | A^T, B' | S (bf16) then R'^T (bf16)
+// Slot c & 1 holds [S X^T | S Q^T] of block c from (b); once the chain has read S X^T, (e') puts
+// R'^T B'^T in its place. dS of block c takes all of the other slot, free between the chain's read
+// of the outputs of block c-1 and (b) of block c+1.
 constexpr uint32_t cGP = 0, cSXO = 64 /* + 128 * slot */, cAB = 320, cSR = 448, kTmemCols = 512;
 
 constexpr uint32_t kIdN64 = tc::idesc_bf16(128, 64, 0, 0);
@@ -83,11 +86,11 @@ enum {
     B_XQRDY = 10,      // [3] helpers prepared the block -> MMA (a)
     B_ADONE = 13,      // (a) done -> helpers, local
     B_GPFREE = 14,     // local read G and helpers read P (2 arrivals) -> MMA (a) of the next block
-    B_SCAL = 15,       // [4] scalars of slot c % 4 ready -> local, chain
-    B_SCALFREE = 19,   // [4] chain done with scalar slot (8 warps) -> helpers
-    B_QSC = 23,        // [3] Q~ ready -> MMA (b)
+    B_SCAL = 15,       // [4] decay scalars of slot c % 4 ready -> local, chain
+    B_SCALFREE = 19,   // [4] chain done with scalar slot, outputs stored (8 warps) -> helpers
+    B_UNUSED23 = 23,   // [3]
     B_PRDY = 26,       // P~ ready -> MMA (B')
-    B_TRDY = 27,       // T_f, T' ready -> MMA (A), (B')
+    B_TRDY = 27,       // T_f, T' (and the step sizes) ready -> MMA (A), (B')
     B_ABDONE = 28,     // (A), (B') done -> chain, local (T tiles free), helpers (P~ tile free)
     B_EARDY = 29,      // A^T, B' in shared memory (8 warps) -> MMA (e'), (f')
     B_BDONE = 30,      // (b) done -> chain
@@ -126,25 +129,6 @@ __device__ __forceinline__ void st_chunk8(uint8_t *base, uint32_t off, const flo
     pk.z = pack_bf16x2(v8[4], v8[5]);
     pk.w = pack_bf16x2(v8[6], v8[7]);
     *reinterpret_cast<uint4 *>(base + off) = pk;
-}
-
-// Scale the 16 chunks (128 bf16) of row `r` of a two-atom, 128-row-per-atom tile by `s`.
-__device__ __forceinline__ void scale_row(uint8_t *tile, int r, float s) {
-#pragma unroll 1
-    for (int q = 0; q < 16; ++q) {
-        const int a = q >> 3, ch = q & 7;
-        {
-            uint4 *pp = reinterpret_cast<uint4 *>(tile + a * 16384 + tc::sw128_chunk(r, ch));
-            uint4 u = *pp;
-            __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                float2 f = __bfloat1622float2(h[k]);
-                h[k] = __floats2bfloat162_rn(f.x * s, f.y * s);
-            }
-            *pp = u;
-        }
-    }
 }
 
 // ---- tf32 warp MMA for the 16 x 16 blocks of the triangular solve
@@ -340,36 +324,40 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     if (warp == 0) {
         // ================================================================ TMA producer
         if (lane == 0) {
+            // [X;Q] of block j, then V of block j-1: the slot of XQ_j frees at (b) of block j-3, which
+            // precedes the chain's read of V_{j-3} that frees the slot of V_{j-1}, so the blocking waits
+            // below never hold back a load that could already start.
             int kx = 0, kv = 0;
-            long long idle_since = clock64();
-            while ((kx < nblk || kv < nblk) && !*abort_flag) {
-                bool progress = false;
-                if (kx < nblk && (kx < 3 || tc::mbar_test(&bars[B_XQFREE + kx % 3], ((kx / 3) - 1) & 1))) {
-                    uint8_t *dst = sm + oXQ + (kx % 3) * kXQ;
-                    uint64_t *fb = &bars[B_FULLXQ + kx % 3];
-                    const int t0 = kx * kBlk;
+            for (int j = 0; j <= nblk && !*abort_flag; ++j) {
+                if (j < nblk) {
+                    if (j >= 3 && !tc::mbar_wait(&bars[B_XQFREE + j % 3], ((j / 3) - 1) & 1, abort_flag, kWaitBudget)) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    uint8_t *dst = sm + oXQ + (j % 3) * kXQ;
+                    uint64_t *fb = &bars[B_FULLXQ + j % 3];
+                    const int t0 = j * kBlk;
                     tc::mbar_arrive_expect_tx(fb, kXQ);
                     tc::tma_load_3d(dst + 0, &tmK, 0, t0 - 1, bh, fb);
                     tc::tma_load_3d(dst + 16384, &tmK, 64, t0 - 1, bh, fb);
                     tc::tma_load_3d(dst + 8192, &tmQ, 0, t0, bh, fb);
                     tc::tma_load_3d(dst + 16384 + 8192, &tmQ, 64, t0, bh, fb);
-                    ++kx;
-                    progress = true;
+                    kx = j + 1;
                 }
-                if (kv < kx && (kv < 2 || tc::mbar_test(&bars[B_VFREE + (kv & 1)], ((kv >> 1) - 1) & 1))) {
-                    uint8_t *dst = sm + oV + (kv & 1) * kVst;
-                    uint64_t *fb = &bars[B_FULLV + (kv & 1)];
-                    const int t0 = kv * kBlk;
+                const int jv = j - 1;
+                if (jv >= 0) {
+                    if (jv >= 2 &&
+                        !tc::mbar_wait(&bars[B_VFREE + (jv & 1)], ((jv >> 1) - 1) & 1, abort_flag, kWaitBudget)) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    uint8_t *dst = sm + oV + (jv & 1) * kVst;
+                    uint64_t *fb = &bars[B_FULLV + (jv & 1)];
+                    const int t0 = jv * kBlk;
                     tc::mbar_arrive_expect_tx(fb, kVst);
                     tc::tma_load_3d(dst + 0, &tmV, 0, t0, bh, fb);
                     tc::tma_load_3d(dst + 8192, &tmV, 64, t0, bh, fb);
-                    ++kv;
-                    progress = true;
-                }
-                if (progress) idle_since = clock64();
-                else if (clock64() - idle_since > kWaitBudget) {
-                    *abort_flag = 1;
-                    break;
+                    kv = jv + 1;
                 }
             }
             // drain: every armed load must have landed before the CTA can exit
@@ -426,10 +414,18 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 return 1;
             };
             // (A) A^T = X^T T_f and (B') B' = P~ T' of block j into the AB columns (free once the chain
-            // copied A^T, B' of block j-1 to shared memory)
-            auto issue_AB = [&](int j) -> bool {
-                if (!(wait(B_TRDY, j & 1) && wait(B_PRDY, j & 1) && (j < 1 || wait(B_EARDY, (j - 1) & 1))))
-                    return false;
+            // copied A^T, B' of block j-1 to shared memory). Returns -1 on abort, else whether it issued.
+            auto issue_AB = [&](int j, bool block) -> int {
+                if (block) {
+                    while (na <= j)
+                        if (try_a(true) < 0) return -1;
+                    if (!(wait(B_TRDY, j & 1) && wait(B_PRDY, j & 1) && (j < 1 || wait(B_EARDY, (j - 1) & 1))))
+                        return -1;
+                } else {
+                    if (na <= j && try_a(false) < 0) return -1;
+                    if (na <= j || !test(B_TRDY, j & 1) || !test(B_PRDY, j & 1) || (j >= 1 && !test(B_EARDY, (j - 1) & 1)))
+                        return 0;
+                }
                 tc::fence_after_sync();
                 const int u = j % 3;
 #pragma unroll
@@ -439,38 +435,34 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 for (int ks = 0; ks < 4; ++ks)
                     tc::mma_bf16_elect(tbase + cAB + 64, dPB + (uint64_t)(ks * 2), dTP + (uint64_t)(ks * 128), kIdBP, ks > 0);
                 tc::mma_commit_elect(&bars[B_ABDONE]);
-                return true;
+                return 1;
             };
-            bool ok = nblk == 0 || (try_a(true) > 0 && issue_AB(0));
+            bool ok = nblk == 0 || issue_AB(0, true) > 0;
             for (int c = 0; c < nblk && ok; ++c) {
                 const int s = c & 1, u = c % 3;
-                // (b) [S X^T | S Q~^T] -> [SX | O] of slot s, S from TMEM
-                if (!(ok = wait(B_SRDY, c & 1) && wait(B_QSC + u, (c / 3) & 1))) break;
+                // (b) [S X^T | S Q^T] -> slot s, S from TMEM
+                if (!(ok = wait(B_SRDY, c & 1))) break;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
                     tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dXQ[u] + kmaj(ks), kIdN128, ks > 0);
                 tc::mma_commit_elect(&bars[B_BDONE]);
                 tc::mma_commit_elect(&bars[B_XQFREE + u]);
-                // state-independent work of later blocks runs while the chain forms R'^T
-                while (ok && na <= c + 1 && na < nblk) ok = try_a(true) >= 0;
-                if (!ok) break;
-                if (c + 1 < nblk && !(ok = issue_AB(c + 1))) break;
+                // state-independent work of the next block runs while the chain forms R'^T, if it is ready
+                int ab = 0;
+                if (c + 1 < nblk && (ab = issue_AB(c + 1, false)) < 0) { ok = false; break; }
                 if ((ok = try_a(false) >= 0) == false) break;
-                // (e') O^T += R'^T B'^T and (f') dS = R'^T A in two N = 64 halves, R'^T from TMEM
+                // (e') R'^T B'^T over S X^T in slot s and (f') dS = R'^T A into slot s^1, R'^T from TMEM
                 if (!(ok = wait(B_RT, c & 1) && wait(B_EARDY, c & 1))) break;
                 tc::fence_after_sync();
-                const uint32_t dlo = tbase + cSXO + 128 * s, dhi = tbase + cSXO + 128 * (s ^ 1) + 64;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16_ts_elect(dlo + 64, tbase + cSR + 8 * ks, dBp + (uint64_t)(ks * 2), kIdN64, 1);
+                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dBp + (uint64_t)(ks * 2), kIdN64, ks > 0);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16_ts_elect(dlo, tbase + cSR + 8 * ks, dAt + (uint64_t)(ks * 2), kIdN64, ks > 0);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16_ts_elect(dhi, tbase + cSR + 8 * ks, dAt + (uint64_t)(512 + ks * 2), kIdN64, ks > 0);
+                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * (s ^ 1), tbase + cSR + 8 * ks, dAt + (uint64_t)(ks * 2), kIdN128, ks > 0);
                 tc::mma_commit_elect(&bars[B_EFDONE]);
+                if (c + 1 < nblk && ab == 0 && issue_AB(c + 1, true) < 0) { ok = false; break; }
                 if ((ok = try_a(false) >= 0) == false) break;
             }
             if (!ok) *abort_flag = 1;
@@ -484,14 +476,13 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         // ================================================================ helpers (64 threads)
         const int ht = tid - 64;           // row / token index 0..63
         const bool leader = ht == 0;
-        const float *alpha_h = p.alpha + (size_t)bh * T, *eta_h = p.eta + (size_t)bh * T;
-        float ga = 1.f, ge = 0.f;          // gates of the block prep() handles next
+        const float *alpha_h = p.alpha + (size_t)bh * T;
+        float ga = 1.f;                    // decay gate of the block prep() handles next
         auto load_gates = [&](int c) {
             const int t = c * kBlk + ht;
             ga = t < T ? alpha_h[t] : 1.f;
-            ge = t < T ? eta_h[t] : 0.f;
         };
-        auto prep = [&](int c) -> bool {   // block c: x_1 patch, norms, step sizes, decay tables
+        auto prep = [&](int c) -> bool {   // block c: x_1 patch, decay tables
             const int u3 = c % 3, u4 = c % 4;
             uint8_t *xq = sm + oXQ + u3 * kXQ;
             if (c >= 4 && !role_wait(&bars[B_SCALFREE + u4], ((c >> 2) - 1) & 1, leader, 1, 64)) return false;
@@ -503,23 +494,8 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 *reinterpret_cast<uint4 *>(xq + (ht >> 3) * 16384 + (ht & 7) * 16) = v;
                 tc::fence_proxy_async();
             }
-            named_bar(1, 64);
-            float nrm = 0.f;
-#pragma unroll
-            for (int a = 0; a < 2; ++a)
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const uint4 w = *reinterpret_cast<const uint4 *>(xq + a * 16384 + tc::sw128_chunk(ht, ch));
-                    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&w);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float2 f = __bfloat1622float2(h2[k]);
-                        nrm += f.x * f.x + f.y * f.y;
-                    }
-                }
             const bool valid = ht < nval;
             float la = valid ? log2f(ga) : 0.f;
-            const float bt = valid ? step_size(ge, nrm, p.eps) : 0.f;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const float y = __shfl_up_sync(0xffffffffu, la, off);
@@ -529,7 +505,6 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             named_bar(1, 64);
             if (ht >= 32) la += sMisc[0];
             float *sc = sScal + u4 * 256;
-            sc[ht] = bt;
             sc[64 + ht] = exp2f(la);
             sc[192 + ht] = la;
             named_bar(1, 64);
@@ -556,7 +531,6 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         for (int c = 0; c < nblk && ok; ++c) {
             const int u3 = c % 3;
             if (c + 2 < nblk) load_gates(c + 2);  // in flight while block c is handled
-            uint8_t *xq = sm + oXQ + u3 * kXQ;
             const float *sc = sScal + (c % 4) * 256;
             if (!(ok = role_wait(&bars[B_ADONE], c & 1, leader, 1, 64))) break;
             // P of query row i = ht from TMEM lanes 64..127 (this pair of warps' quarters)
@@ -571,14 +545,8 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 for (int j = 0; j < 32; ++j) { v[j] = h0[j]; v[32 + j] = h1[j]; }
             }
             tc::fence_before_sync();
-            // Q~ = diag(2^g) Q once (a) no longer needs Q
-            scale_row(xq, 64 + ht, sc[64 + ht]);
-            tc::fence_proxy_async();
             named_bar(1, 64);
-            if (leader) {
-                mbar_arrive(&bars[B_GPFREE]);
-                mbar_arrive(&bars[B_QSC + u3]);
-            }
+            if (leader) mbar_arrive(&bars[B_GPFREE]);
             // P~ = Gamma o P (inclusive), packed to bf16 while (B') of the previous block still reads the tile
             uint32_t pk[32];
             {
@@ -622,13 +590,15 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         const int r = 32 * lw + lane;      // TMEM lane: G row for lw < 2 (P rows belong to the helpers)
         const bool leader = lt == 0;
         const uint32_t tl = tbase + ((uint32_t)(32 * lw) << 16);
+        const float *eta_h = p.eta + (size_t)bh * T;
+        float ge = (lw < 2 && r < T) ? eta_h[r] : 0.f;   // step-size gate of row r, one block ahead
         for (int c = 0; c < nblk; ++c) {
             const int u4 = c % 4;
             if (!role_wait(&bars[B_ADONE], c & 1, leader, 2, 128)) break;
             if (!role_wait(&bars[B_SCAL + u4], (c >> 2) & 1, leader, 2, 128)) break;
             tc::fence_after_sync();
-            const float *sc = sScal + u4 * 256;
-            if (REG && lw < 2) {                            // G rows r = 0..63 -> L
+            float *sc = sScal + u4 * 256;
+            if (lw < 2) {                                   // G rows r = 0..63: step sizes, then L
                 float v[64];
                 {
                     float h0[32], h1[32];
@@ -637,13 +607,23 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 #pragma unroll
                     for (int j = 0; j < 32; ++j) { v[j] = h0[j]; v[32 + j] = h1[j]; }
                 }
+                // ||x_r||^2 is the diagonal entry G[r][r]: column r = 32 lw + lane of this row
+                float nrm = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) nrm += (j == lane) ? (lw == 0 ? v[j] : v[32 + j]) : 0.f;
+                const bool valid = c * kBlk + r < T;
+                const float be = valid ? step_size(ge, nrm, p.eps) : 0.f;
+                sc[r] = be;
+                const int tn = (c + 1) * kBlk + r;
+                ge = tn < T ? eta_h[tn] : 0.f;
+              if (REG) {
                 // Decay factors 2^(g_r - g_j), j < r: below the 16x16 diagonal blocks they factor
                 // through the last index of column block jb, 2^(g_r - g_{16jb+15}) * cf[j] with
                 // cf[j] = 2^(g_{16jb+15} - g_j) (a helper table), both in (0, 1]; inside the
                 // diagonal block they are formed directly. Selects only, no divergent branches.
                 const float *g2 = sc + 192, *cf = sCF + 64 * u4;
                 const int rb = r >> 4;
-                const float gri = g2[r], be = sc[r];
+                const float gri = g2[r];
                 float fac[4], gd[16];
 #pragma unroll
                 for (int jb = 0; jb < 4; ++jb) {
@@ -668,6 +648,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                     }
                     *reinterpret_cast<float4 *>(Lr + j0) = make_float4(w4[0], w4[1], w4[2], w4[3]);
                 }
+              }
             }
             tc::fence_before_sync();
             named_bar(2, 128);
@@ -717,22 +698,30 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(S[2 * j], S[2 * j + 1]);
             tc::tmem_st32(tl + cSR + 32 * hf, pk);
         };
-        // O^T of block c (TMEM slot c & 1) to global memory: lane pairs (2k, 2k+1) hold neighbouring
-        // value rows; the even lane stores the pair for even tokens, the odd lane for odd tokens.
+        // O^T of block c (TMEM slot c & 1: S Q^T scaled by 2^g per token, plus R'^T B'^T) to global
+        // memory: lane pairs (2k, 2k+1) hold neighbouring value rows; the even lane stores the pair for
+        // even tokens, the odd lane for odd tokens.
         auto store_out = [&](int c) {
             const int t0 = c * kBlk, nval = min(kBlk, T - t0);
-            float v[32];
-            tc::tmem_ld32(tl + cSXO + 128 * (c & 1) + 64 + 32 * hf, v);
             const bool odd = lane & 1;
             __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.o) + ((size_t)bh * T + t0) * D + (row & ~1);
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                const int i0 = 32 * hf + 16 * h;
+                const float *d2 = sScal + (c % 4) * 256 + 64 + i0;   // 2^g of the tokens
+                float v[16], w[16];
+                tc::tmem_ld16(tl + cSXO + 128 * (c & 1) + 64 + i0, v);
+                tc::tmem_ld16(tl + cSXO + 128 * (c & 1) + i0, w);
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-                const float mine = odd ? v[j + 1] : v[j];
-                const float give = odd ? v[j] : v[j + 1];
-                const float other = __shfl_xor_sync(0xffffffffu, give, 1);
-                const int i = 32 * hf + j + (odd ? 1 : 0);
-                const float lo = odd ? other : mine, hi = odd ? mine : other;
-                if (i < nval) *reinterpret_cast<uint32_t *>(o + (size_t)i * D) = pack_bf16x2(lo, hi);
+                for (int j = 0; j < 16; j += 2) {
+                    const float v0 = d2[j] * v[j] + w[j], v1 = d2[j + 1] * v[j + 1] + w[j + 1];
+                    const float mine = odd ? v1 : v0;
+                    const float give = odd ? v0 : v1;
+                    const float other = __shfl_xor_sync(0xffffffffu, give, 1);
+                    const int i = i0 + j + (odd ? 1 : 0);
+                    const float lo = odd ? other : mine, hi = odd ? mine : other;
+                    if (i < nval) *reinterpret_cast<uint32_t *>(o + (size_t)i * D) = pack_bf16x2(lo, hi);
+                }
             }
         };
         {
@@ -766,7 +755,12 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             tc::fence_proxy_async();
             warp_arrive(&bars[B_EARDY]);
             // outputs of the previous block (off the chain; their columns take dS of this block)
-            if (c >= 1) store_out(c - 1);
+            if (c >= 1) {
+                store_out(c - 1);
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_SCALFREE + (c - 1) % 4]);
+            }
             // R'^T = Y^T - SX diag(2^g) (regression) or Y^T (inner product), bf16 into TMEM
             if (!(ok = warp_wait(&bars[B_BDONE], c & 1) && warp_wait(&bars[B_SCAL + u4], (c >> 2) & 1) &&
                        warp_wait(&bars[B_FULLV + s], (c >> 1) & 1)))
@@ -796,7 +790,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             tc::fence_after_sync();
             {
                 const float dl = exp2f(sGL[u4]);
-                const uint32_t cds = hf == 0 ? cSXO + 128 * s : cSXO + 128 * (s ^ 1) + 64;
+                const uint32_t cds = cSXO + 128 * (s ^ 1) + 64 * hf;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float v[32];
@@ -807,7 +801,6 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             }
             store_S();
             warp_arrive(&bars[B_SRDY]);
-            if (lane == 0) mbar_arrive(&bars[B_SCALFREE + u4]);
         }
         if (ok && nblk > 0 && !*abort_flag) {
             store_out(nblk - 1);
