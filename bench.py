@@ -37,7 +37,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "Falcon-1 chunk fwd tokens/s & % roofline (B8 H16 T4K d128); decode GB/s"
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
-CHUNK_KERNEL_SOURCES = ["chunk_kernel.cuh", "chunk_mma.cuh", "common.cuh"]
+CHUNK_KERNEL_SOURCES = ["chunk_ws.cu", "tc_common.cuh", "common.cuh"]
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -478,7 +478,7 @@ def main(argv=None):
     flops = chunk_algorithmic_flops(B, H, T, dk, dv)
     achieved = nbytes / (ch["kern_ms"] * 1e-3) / 1e9
     t_roof = max(nbytes / (hbm * 1e9), flops / (tf * 1e12))
-    traffic = recorded_traffic("chunk_fwd_kernel", CHUNK_KERNEL_SOURCES)
+    traffic = recorded_traffic("chunk_ws_kernel", CHUNK_KERNEL_SOURCES)
     dbytes = decode_algorithmic_bytes(dec["N"], dec["H"], dec["dk"], dec["dv"])
     dgbs = dbytes / (dec["ms"] * 1e-3) / 1e9
 
@@ -490,7 +490,7 @@ def main(argv=None):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(achieved / hbm, 4), "traffic": traffic,
                      "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else src,
-                     "algorithmic_bytes_per_launch": nbytes, "kernel": "chunk_fwd_kernel",
+                     "algorithmic_bytes_per_launch": nbytes, "kernel": "chunk_ws_kernel",
                      "kernel_ms": round(ch["kern_ms"], 4)},
         "north_star_roofline": {"flops": flops, "bytes": nbytes, "t_roofline_us": round(t_roof * 1e6, 2),
                                 "frac": round(t_roof / (ch["kern_ms"] * 1e-3), 4),

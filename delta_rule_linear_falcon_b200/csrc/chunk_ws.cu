@@ -553,24 +553,29 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 const float *g2 = sc + 192, *cf = sCF + 64 * (c % 4);
                 const int i = ht, rb = i >> 4;
                 const float gri = g2[i];
-                float fac[4], gd[16];
+                float gd[16];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float4 g4 = *reinterpret_cast<const float4 *>(g2 + 16 * rb + 4 * q);
+                    const int j = 16 * rb + 4 * q;
+                    gd[4 * q] = j <= i ? exp2f(fminf(gri - g4.x, 0.f)) : 0.f;
+                    gd[4 * q + 1] = j + 1 <= i ? exp2f(fminf(gri - g4.y, 0.f)) : 0.f;
+                    gd[4 * q + 2] = j + 2 <= i ? exp2f(fminf(gri - g4.z, 0.f)) : 0.f;
+                    gd[4 * q + 3] = j + 3 <= i ? exp2f(fminf(gri - g4.w, 0.f)) : 0.f;
+                }
 #pragma unroll
                 for (int jb = 0; jb < 4; ++jb) {
-                    const float f = exp2f(fminf(gri - g2[16 * jb + 15], 0.f));
-                    fac[jb] = jb < rb ? f : 0.f;
-                }
+                    const float fac = jb < rb ? exp2f(fminf(gri - g2[16 * jb + 15], 0.f)) : 0.f;
+                    const bool diag = jb == rb;
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const int j = 16 * rb + k;
-                    const float f = exp2f(fminf(gri - g2[j], 0.f));
-                    gd[k] = j <= i ? f : 0.f;
-                }
-#pragma unroll
-                for (int j = 0; j < 64; j += 2) {
-                    const int jb = j >> 4;
-                    const float g0 = jb < rb ? fac[jb] * cf[j] : (jb == rb ? gd[j & 15] : 0.f);
-                    const float g1 = jb < rb ? fac[jb] * cf[j + 1] : (jb == rb ? gd[(j + 1) & 15] : 0.f);
-                    pk[j >> 1] = pack_bf16x2(g0 * v[j], g1 * v[j + 1]);
+                    for (int q = 0; q < 4; ++q) {
+                        const int j = 16 * jb + 4 * q;
+                        const float4 c4 = *reinterpret_cast<const float4 *>(cf + j);
+                        const float w0 = diag ? gd[4 * q] : fac * c4.x, w1 = diag ? gd[4 * q + 1] : fac * c4.y;
+                        const float w2 = diag ? gd[4 * q + 2] : fac * c4.z, w3 = diag ? gd[4 * q + 3] : fac * c4.w;
+                        pk[j >> 1] = pack_bf16x2(w0 * v[j], w1 * v[j + 1]);
+                        pk[(j >> 1) + 1] = pack_bf16x2(w2 * v[j + 2], w3 * v[j + 3]);
+                    }
                 }
             }
             if (c >= 1 && !(ok = role_wait(&bars[B_ABDONE], (c - 1) & 1, leader, 1, 64))) break;
@@ -620,33 +625,36 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 // Decay factors 2^(g_r - g_j), j < r: below the 16x16 diagonal blocks they factor
                 // through the last index of column block jb, 2^(g_r - g_{16jb+15}) * cf[j] with
                 // cf[j] = 2^(g_{16jb+15} - g_j) (a helper table), both in (0, 1]; inside the
-                // diagonal block they are formed directly. Selects only, no divergent branches.
+                // diagonal block they are formed directly. The solve reads only the strictly lower
+                // part, so entries on and above the diagonal are left as they come (finite, <= |G|).
                 const float *g2 = sc + 192, *cf = sCF + 64 * u4;
                 const int rb = r >> 4;
                 const float gri = g2[r];
-                float fac[4], gd[16];
+                float gd[16];
 #pragma unroll
-                for (int jb = 0; jb < 4; ++jb) {
-                    const float f = exp2f(fminf(gri - g2[16 * jb + 15], 0.f));
-                    fac[jb] = jb < rb ? be * f : 0.f;
-                }
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const int j = 16 * rb + k;
-                    const float f = exp2f(fminf(gri - g2[j], 0.f));
-                    gd[k] = j < r ? be * f : 0.f;
+                for (int q = 0; q < 4; ++q) {
+                    const float4 g4 = *reinterpret_cast<const float4 *>(g2 + 16 * rb + 4 * q);
+                    gd[4 * q] = be * exp2f(fminf(gri - g4.x, 0.f));
+                    gd[4 * q + 1] = be * exp2f(fminf(gri - g4.y, 0.f));
+                    gd[4 * q + 2] = be * exp2f(fminf(gri - g4.z, 0.f));
+                    gd[4 * q + 3] = be * exp2f(fminf(gri - g4.w, 0.f));
                 }
                 float *Lr = sL + r * LDF;
 #pragma unroll
-                for (int j0 = 0; j0 < 64; j0 += 4) {
-                    float w4[4];
+                for (int jb = 0; jb < 4; ++jb) {
+                    const float fac = be * exp2f(fminf(gri - g2[16 * jb + 15], 0.f));
+                    const bool below = jb < rb;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int j = j0 + k, jb = j >> 4;
-                        const float gm = jb < rb ? fac[jb] * cf[j] : (jb == rb ? gd[j & 15] : 0.f);
-                        w4[k] = gm * v[j];
+                    for (int q = 0; q < 4; ++q) {
+                        const int j = 16 * jb + 4 * q;
+                        const float4 c4 = *reinterpret_cast<const float4 *>(cf + j);
+                        const float w0 = below ? fac * c4.x : gd[4 * q];
+                        const float w1 = below ? fac * c4.y : gd[4 * q + 1];
+                        const float w2 = below ? fac * c4.z : gd[4 * q + 2];
+                        const float w3 = below ? fac * c4.w : gd[4 * q + 3];
+                        *reinterpret_cast<float4 *>(Lr + j) =
+                            make_float4(w0 * v[j], w1 * v[j + 1], w2 * v[j + 2], w3 * v[j + 3]);
                     }
-                    *reinterpret_cast<float4 *>(Lr + j0) = make_float4(w4[0], w4[1], w4[2], w4[3]);
                 }
               }
             }
@@ -672,9 +680,12 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 #pragma unroll
                         for (int k = 0; k < 8; ++k) t8[k] = (j0 + k == rr) ? 1.f : 0.f;
                     }
+                    const float4 b0 = *reinterpret_cast<const float4 *>(sc + j0);     // beta of the columns
+                    const float4 b1 = *reinterpret_cast<const float4 *>(sc + j0 + 4);
+                    const float bc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
-                        t8[k] *= sc[j0 + k];  // beta of the column
+                        t8[k] *= bc[k];
                         f8[k] = fr * t8[k];
                     }
                     st_chunk8(sTP, tc::sw128_chunk(rr, ch0 + cc), t8);
@@ -691,6 +702,11 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         const int qd = warp & 3, hf = (warp - 8) >> 2;
         const int row = 32 * qd + lane;    // TMEM lane = value row (and key row d of A^T)
         const uint32_t tl = tbase + ((uint32_t)(32 * qd) << 16);
+        // V tile (token rows i, value columns): element (i, row) sits at vcol + voff[i & 7] + (i >> 3) * 1024
+        const uint32_t vcol = (row >> 6) * 8192 + (row & 7) * 2;
+        uint32_t voff[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) voff[k] = k * 128 + (((((row & 63) >> 3) ^ k)) << 4);
         float S[64];                       // fp32 state, row `row`, columns 64 hf ..
         auto store_S = [&]() {             // bf16 pairs of this thread's 64 columns -> TMEM A operand
             uint32_t pk[32];
@@ -709,12 +725,17 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             for (int h = 0; h < 2; ++h) {
                 const int i0 = 32 * hf + 16 * h;
                 const float *d2 = sScal + (c % 4) * 256 + 64 + i0;   // 2^g of the tokens
-                float v[16], w[16];
+                float v[16], w[16], dg[16];
                 tc::tmem_ld16(tl + cSXO + 128 * (c & 1) + 64 + i0, v);
                 tc::tmem_ld16(tl + cSXO + 128 * (c & 1) + i0, w);
 #pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float4 d4 = *reinterpret_cast<const float4 *>(d2 + 4 * q);
+                    dg[4 * q] = d4.x; dg[4 * q + 1] = d4.y; dg[4 * q + 2] = d4.z; dg[4 * q + 3] = d4.w;
+                }
+#pragma unroll
                 for (int j = 0; j < 16; j += 2) {
-                    const float v0 = d2[j] * v[j] + w[j], v1 = d2[j + 1] * v[j + 1] + w[j + 1];
+                    const float v0 = dg[j] * v[j] + w[j], v1 = dg[j + 1] * v[j + 1] + w[j + 1];
                     const float mine = odd ? v1 : v0;
                     const float give = odd ? v0 : v1;
                     const float other = __shfl_xor_sync(0xffffffffu, give, 1);
@@ -768,18 +789,29 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             tc::fence_after_sync();
             {
                 const float *sc = sScal + u4 * 256;
-                const uint8_t *sV = sm + oV + s * kVst;
-                float x[32];
-                if (REG) tc::tmem_ld32(tl + cSXO + 128 * s + 32 * hf, x);
+                const uint8_t *sV = sm + oV + s * kVst + vcol;
                 uint32_t pk[16];
 #pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    const int i = 32 * hf + j;
-                    const float y0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sV + tc::sw128_off(i, row, 64)));
-                    const float y1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sV + tc::sw128_off(i + 1, row, 64)));
-                    const float r0 = REG ? y0 - sc[64 + i] * x[j] : y0;
-                    const float r1 = REG ? y1 - sc[64 + i + 1] * x[j + 1] : y1;
-                    pk[j >> 1] = pack_bf16x2(r0, r1);
+                for (int hh = 0; hh < 2; ++hh) {           // 16 tokens at a time
+                    const int i0 = 32 * hf + 16 * hh;
+                    float x[16], dg[16];
+                    if (REG) {
+                        tc::tmem_ld16(tl + cSXO + 128 * s + i0, x);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 d4 = *reinterpret_cast<const float4 *>(sc + 64 + i0 + 4 * q);
+                            dg[4 * q] = d4.x; dg[4 * q + 1] = d4.y; dg[4 * q + 2] = d4.z; dg[4 * q + 3] = d4.w;
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; j += 2) {
+                        const int i = i0 + j;              // token row of V: swizzle depends on i & 7 only
+                        const float y0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sV + voff[i & 7] + (i >> 3) * 1024));
+                        const float y1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sV + voff[(i + 1) & 7] + ((i + 1) >> 3) * 1024));
+                        const float r0 = REG ? y0 - dg[j] * x[j] : y0;
+                        const float r1 = REG ? y1 - dg[j + 1] * x[j + 1] : y1;
+                        pk[8 * hh + (j >> 1)] = pack_bf16x2(r0, r1);
+                    }
                 }
                 tc::tmem_st16(tl + cSR + 16 * hf, pk);
             }
