@@ -100,7 +100,6 @@ cudaError_t launch_chunk_dk128(const ChunkParams &p, int dvs, cudaStream_t s);
 
 cudaError_t launch_chunk(const ChunkParams &p, int num_sms, cudaStream_t s) {
     if (chunk_ws_supported(p)) return launch_chunk_ws(p, s);
-    if (chunk_tc_supported(p)) return launch_chunk_tc(p, s);
     const int dvs = pick_value_slice((long long)p.B * p.H, p.dv, num_sms);
     switch (p.dk) {
         case 32: return launch_chunk_dk32(p, dvs, s);

@@ -47,10 +47,7 @@ size_t recurrent_smem_bytes(int dk, int dv, int window);
 cudaError_t launch_recurrent(const RecParams &p, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, cudaStream_t s);
 cudaError_t launch_chunk(const ChunkParams &p, int num_sms, cudaStream_t s);
-// tcgen05 / TMA kernel for d_k = d_v = 128, bf16 I/O, one pair per step, 64-token blocks.
-bool chunk_tc_supported(const ChunkParams &p);
-cudaError_t launch_chunk_tc(const ChunkParams &p, cudaStream_t s);
-// Warp-specialised tcgen05 kernel (same shapes, T a multiple of 4).
+// Warp-specialised tcgen05 / TMA kernel: d_k = d_v = 128, bf16 I/O, one pair per step, 64-token blocks.
 bool chunk_ws_supported(const ChunkParams &p);
 cudaError_t launch_chunk_ws(const ChunkParams &p, cudaStream_t s);
 
