@@ -85,7 +85,7 @@ enum {
     B_VFREE = 8,       // [2] chain read V (8 warps) -> producer
     B_XQRDY = 10,      // [3] helpers prepared the block -> MMA (a)
     B_ADONE = 13,      // (a) done -> helpers, local
-    B_GPFREE = 14,     // local read G and helpers read P (2 arrivals) -> MMA (a) of the next block
+    B_GPFREE = 14,     // G read (local warps 4, 5) and P read (helpers): 3 arrivals -> MMA (a) of the next block
     B_SCAL = 15,       // [4] decay scalars of slot c % 4 ready -> local, chain
     B_SCALFREE = 19,   // [4] chain done with scalar slot, outputs stored (8 warps) -> helpers
     B_UNUSED23 = 23,   // [3]
@@ -281,7 +281,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         for (int i = 0; i < B_COUNT; ++i) {
             const bool chain_arrivals = (i >= B_VFREE && i < B_VFREE + 2) || (i >= B_SCALFREE && i < B_SCALFREE + 4) ||
                                         i == B_EARDY || i == B_RT || i == B_SRDY;
-            tc::mbar_init(&bars[i], chain_arrivals ? kChainWarps : (i == B_GPFREE ? 2 : 1));
+            tc::mbar_init(&bars[i], chain_arrivals ? kChainWarps : (i == B_GPFREE ? 3 : 1));
         }
         *abort_flag = 0;
         tc::mbar_fence_init();
@@ -612,6 +612,10 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 #pragma unroll
                     for (int j = 0; j < 32; ++j) { v[j] = h0[j]; v[32 + j] = h1[j]; }
                 }
+                // G is in registers: its columns may take (a) of the next block
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_GPFREE]);
                 // ||x_r||^2 is the diagonal entry G[r][r]: column r = 32 lw + lane of this row
                 float nrm = 0.f;
 #pragma unroll
@@ -658,9 +662,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 }
               }
             }
-            tc::fence_before_sync();
             named_bar(2, 128);
-            if (leader) mbar_arrive(&bars[B_GPFREE]);
             if (REG) solve_local(sL, sTf, lt, lw, lane);
             // T_f = diag(2^(g_last - g)) T diag(beta), T' = T diag(beta) once (A), (B') of c-1 are done
             if (c >= 1 && !role_wait(&bars[B_ABDONE], (c - 1) & 1, leader, 2, 128)) break;
