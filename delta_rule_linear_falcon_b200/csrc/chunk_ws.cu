@@ -178,8 +178,12 @@ __device__ __forceinline__ void store16(float *C, const float (&acc)[2][4], int 
 
 // T = (I + L)^-1 for strictly lower L (64 x 64 fp32) by 16 x 16 blocks, run by the
 // 128 threads of the local warpgroup (named barrier 2):
-//   diagonal blocks by forward substitution (one thread per column);
-//   W_im = -T_ii L_im (stored over L_im); T_ij = sum_{m=j}^{i-1} W_im T_mj per block diagonal.
+//   diagonal blocks T_ii by forward substitution (one thread per column);
+//   W_im = -T_ii L_im, stored over L_im by the warp that formed it;
+//   T_ij = sum_{m=j}^{i-1} W_im T_mj, with the terms spread so that the longest chain of
+//   dependent 16 x 16 products after W is three:
+//     round A: T_10, T_21, T_32 and W_20 T_00;  round B: T_20, T_31 and W_30 T_00 + W_31 T_10;
+//     round C: T_30.
 // Entries above the block diagonal of Tf are zero on entry and stay zero.
 __device__ __forceinline__ void solve_local(float *sL, float *sTf, int lt, int lw, int lane) {
     if (lt < 64) {  // column j of the inverse of diagonal block b, left-looking, rows of L as float4
@@ -207,47 +211,59 @@ __device__ __forceinline__ void solve_local(float *sL, float *sTf, int lt, int l
         for (int i = 0; i < 16; ++i) Tb[i * LDF + j] = x[i];
     }
     named_bar(2, 128);
+    auto Lb = [&](int i, int m) { return sL + (16 * i) * LDF + 16 * m; };    // L_im, then W_im
+    auto Tb = [&](int i, int m) { return sTf + (16 * i) * LDF + 16 * m; };
+    auto zero = [](float (&acc)[2][4]) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int h = 0; h < 4; ++h) acc[nt][h] = 0.f;
+    };
     // W blocks (i, m): (1,0) (2,0) (2,1) (3,0) (3,1) (3,2); warp lw takes blocks lw and lw + 4
-    float wacc[2][2][4];
-    int nw = 0;
-    int wi[2], wm[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
         const int blk = lw + 4 * k;
         if (blk < 6) {
             const int i = blk < 1 ? 1 : (blk < 3 ? 2 : 3);
             const int m = blk < 1 ? 0 : (blk < 3 ? blk - 1 : blk - 3);
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int h = 0; h < 4; ++h) wacc[k][nt][h] = 0.f;
-            mma16_acc(wacc[k], sTf + (16 * i) * LDF + 16 * i, sL + (16 * i) * LDF + 16 * m, lane);
-            wi[k] = i;
-            wm[k] = m;
-            nw = k + 1;
-        }
-    }
-    named_bar(2, 128);
-#pragma unroll
-    for (int k = 0; k < 2; ++k)
-        if (k < nw) store16(sL + (16 * wi[k]) * LDF + 16 * wm[k], wacc[k], lane, -1.f);
-    named_bar(2, 128);
-#pragma unroll
-    for (int d = 1; d < 4; ++d) {
-        const int j = lw;          // block column; warp lw computes T_{j+d, j}
-        const int i = j + d;
-        if (i < 4) {
             float acc[2][4];
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int h = 0; h < 4; ++h) acc[nt][h] = 0.f;
-            for (int m = j; m < i; ++m)
-                mma16_acc(acc, sL + (16 * i) * LDF + 16 * m, sTf + (16 * m) * LDF + 16 * j, lane);
-            store16(sTf + (16 * i) * LDF + 16 * j, acc, lane, 1.f);
+            zero(acc);
+            mma16_acc(acc, Tb(i, i), Lb(i, m), lane);
+            __syncwarp();
+            store16(Lb(i, m), acc, lane, -1.f);
         }
-        named_bar(2, 128);
     }
+    named_bar(2, 128);
+    float part[2][4];
+    zero(part);
+    if (lw < 3) {          // round A: T_{lw+1, lw} = W_{lw+1, lw} T_{lw, lw}
+        float acc[2][4];
+        zero(acc);
+        mma16_acc(acc, Lb(lw + 1, lw), Tb(lw, lw), lane);
+        store16(Tb(lw + 1, lw), acc, lane, 1.f);
+    } else {
+        mma16_acc(part, Lb(2, 0), Tb(0, 0), lane);   // W_20 T_00, finished in round B
+    }
+    named_bar(2, 128);
+    if (lw == 0) {         // round B
+        mma16_acc(part, Lb(3, 0), Tb(0, 0), lane);   // W_30 T_00 + W_31 T_10, finished in round C
+        mma16_acc(part, Lb(3, 1), Tb(1, 0), lane);
+    } else if (lw == 1) {
+        float acc[2][4];
+        zero(acc);
+        mma16_acc(acc, Lb(3, 1), Tb(1, 1), lane);
+        mma16_acc(acc, Lb(3, 2), Tb(2, 1), lane);
+        store16(Tb(3, 1), acc, lane, 1.f);
+    } else if (lw == 3) {
+        mma16_acc(part, Lb(2, 1), Tb(1, 0), lane);
+        store16(Tb(2, 0), part, lane, 1.f);
+    }
+    named_bar(2, 128);
+    if (lw == 0) {         // round C
+        mma16_acc(part, Lb(3, 2), Tb(2, 0), lane);
+        store16(Tb(3, 0), part, lane, 1.f);
+    }
+    named_bar(2, 128);
 }
 
 }  // namespace
