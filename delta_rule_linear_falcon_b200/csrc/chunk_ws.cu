@@ -178,7 +178,7 @@ __device__ __forceinline__ void store16(float *C, const float (&acc)[2][4], int 
 
 // T = (I + L)^-1 for strictly lower L (64 x 64 fp32) by 16 x 16 blocks, run by the
 // 128 threads of the local warpgroup (named barrier 2):
-//   diagonal blocks T_ii by forward substitution (one thread per column);
+//   diagonal blocks T_ii by forward substitution (one thread per column, one warp per block);
 //   W_im = -T_ii L_im, stored over L_im by the warp that formed it;
 //   T_ij = sum_{m=j}^{i-1} W_im T_mj, with the terms spread so that the longest chain of
 //   dependent 16 x 16 products after W is three:
@@ -186,8 +186,8 @@ __device__ __forceinline__ void store16(float *C, const float (&acc)[2][4], int 
 //     round C: T_30.
 // Entries above the block diagonal of Tf are zero on entry and stay zero.
 __device__ __forceinline__ void solve_local(float *sL, float *sTf, int lt, int lw, int lane) {
-    if (lt < 64) {  // column j of the inverse of diagonal block b, left-looking, rows of L as float4
-        const int b = lt >> 4, j = lt & 15;
+    if (lane < 16) {  // column j of the inverse of diagonal block b = warp, left-looking, rows of L as float4
+        const int b = lw, j = lane;
         const float *Lb = sL + (16 * b) * LDF + 16 * b;
         float x[16];
 #pragma unroll
@@ -388,13 +388,11 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         {
             // Descriptors are built once; a K step only moves the 14-bit start-address field
             // (address >> 4), which stays below 2^14 for every operand here, so a plain add is exact.
-            uint64_t dXQ[3], dXmn[3];
-#pragma unroll
-            for (int u = 0; u < 3; ++u) {
-                const uint32_t a = tc::smem_u32(sm + oXQ + u * kXQ);
-                dXQ[u] = tc::sdesc(a, 16, 1024);      // [X;Q] K-major: A and B of (a), B of (b)
-                dXmn[u] = tc::sdesc(a, 16384, 1024);  // X as an MN-major A (d atoms 16 KB apart)
-            }
+            // Slot u of the [X;Q] ring is kXQ bytes further: its descriptors are the slot-0 ones plus
+            // u * kXQ / 16 (kept arithmetic so that they stay warp-uniform, in uniform registers).
+            const uint64_t dXQ0 = tc::sdesc(tc::smem_u32(sm + oXQ), 16, 1024);      // [X;Q] K-major: (a), (b)
+            const uint64_t dXmn0 = tc::sdesc(tc::smem_u32(sm + oXQ), 16384, 1024);  // X as an MN-major A
+            auto slot_off = [](int u) -> uint64_t { return (uint64_t)(u * (kXQ >> 4)); };
             const uint64_t dTF = tc::sdesc(tc::smem_u32(sTF), 8192, 1024);   // MN-major B, one N atom
             const uint64_t dTP = tc::sdesc(tc::smem_u32(sTP), 8192, 1024);
             const uint64_t dPB = tc::sdesc(tc::smem_u32(sPB), 16, 1024);     // [P~; B'] K-major
@@ -422,7 +420,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                     return 0;
                 }
                 tc::fence_after_sync();
-                const uint64_t d = dXQ[na % 3];
+                const uint64_t d = dXQ0 + slot_off(na % 3);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) tc::mma_bf16_elect(tbase + cGP, d + kmaj(ks), d + kmaj(ks), kIdN64, ks > 0);
                 tc::mma_commit_elect(&bars[B_ADONE]);
@@ -446,7 +444,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 const int u = j % 3;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16_elect(tbase + cAB, dXmn[u] + (uint64_t)(ks * 128), dTF + (uint64_t)(ks * 128), kIdAT, ks > 0);
+                    tc::mma_bf16_elect(tbase + cAB, dXmn0 + slot_off(u) + (uint64_t)(ks * 128), dTF + (uint64_t)(ks * 128), kIdAT, ks > 0);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     tc::mma_bf16_elect(tbase + cAB + 64, dPB + (uint64_t)(ks * 2), dTP + (uint64_t)(ks * 128), kIdBP, ks > 0);
@@ -461,7 +459,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 tc::fence_after_sync();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dXQ[u] + kmaj(ks), kIdN128, ks > 0);
+                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dXQ0 + slot_off(u) + kmaj(ks), kIdN128, ks > 0);
                 tc::mma_commit_elect(&bars[B_BDONE]);
                 tc::mma_commit_elect(&bars[B_XQFREE + u]);
                 // state-independent work of the next block runs while the chain forms R'^T, if it is ready
@@ -620,6 +618,8 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             tc::fence_after_sync();
             float *sc = sScal + u4 * 256;
             if (lw < 2) {                                   // G rows r = 0..63: step sizes, then L
+                const float *g2 = sc + 192, *cf = sCF + 64 * u4;
+                const int rb = r >> 4;
                 float v[64];
                 {
                     float h0[32], h1[32];
@@ -647,8 +647,6 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 // cf[j] = 2^(g_{16jb+15} - g_j) (a helper table), both in (0, 1]; inside the
                 // diagonal block they are formed directly. The solve reads only the strictly lower
                 // part, so entries on and above the diagonal are left as they come (finite, <= |G|).
-                const float *g2 = sc + 192, *cf = sCF + 64 * u4;
-                const int rb = r >> 4;
                 const float gri = g2[r];
                 float gd[16];
 #pragma unroll
@@ -740,19 +738,18 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             const bool odd = lane & 1;
             __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.o) + ((size_t)bh * T + t0) * D + (row & ~1);
 #pragma unroll 1
-            for (int h = 0; h < 2; ++h) {
-                const int i0 = 32 * hf + 16 * h;
+            for (int h = 0; h < 4; ++h) {          // 8 tokens at a time
+                const int i0 = 32 * hf + 8 * h;
                 const float *d2 = sScal + (c % 4) * 256 + 64 + i0;   // 2^g of the tokens
-                float v[16], w[16], dg[16];
-                tc::tmem_ld16(tl + cSXO + 128 * (c & 1) + 64 + i0, v);
-                tc::tmem_ld16(tl + cSXO + 128 * (c & 1) + i0, w);
+                // the scales first, so that their shared-memory latency overlaps the TMEM loads
+                const float4 da = *reinterpret_cast<const float4 *>(d2);
+                const float4 db = *reinterpret_cast<const float4 *>(d2 + 4);
+                float v[8], w[8];
+                tc::tmem_ld8(tl + cSXO + 128 * (c & 1) + 64 + i0, v);
+                tc::tmem_ld8(tl + cSXO + 128 * (c & 1) + i0, w);
+                const float dg[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 d4 = *reinterpret_cast<const float4 *>(d2 + 4 * q);
-                    dg[4 * q] = d4.x; dg[4 * q + 1] = d4.y; dg[4 * q + 2] = d4.z; dg[4 * q + 3] = d4.w;
-                }
-#pragma unroll
-                for (int j = 0; j < 16; j += 2) {
+                for (int j = 0; j < 8; j += 2) {
                     const float v0 = dg[j] * v[j] + w[j], v1 = dg[j + 1] * v[j + 1] + w[j + 1];
                     const float mine = odd ? v1 : v0;
                     const float give = odd ? v0 : v1;
