@@ -807,25 +807,24 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 const uint8_t *sV = sm + oV + s * kVst + vcol;
                 uint32_t pk[16];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {           // 16 tokens at a time
-                    const int i0 = 32 * hf + 16 * hh;
-                    float x[16], dg[16];
-                    if (REG) {
-                        tc::tmem_ld16(tl + cSXO + 128 * s + i0, x);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const float4 d4 = *reinterpret_cast<const float4 *>(sc + 64 + i0 + 4 * q);
-                            dg[4 * q] = d4.x; dg[4 * q + 1] = d4.y; dg[4 * q + 2] = d4.z; dg[4 * q + 3] = d4.w;
-                        }
+                for (int hh = 0; hh < 4; ++hh) {           // 8 tokens at a time
+                    const int i0 = 32 * hf + 8 * hh;
+                    float x[8], dg[8];
+                    if (REG) {                             // scales first: their latency overlaps the TMEM load
+                        const float4 da = *reinterpret_cast<const float4 *>(sc + 64 + i0);
+                        const float4 db = *reinterpret_cast<const float4 *>(sc + 64 + i0 + 4);
+                        dg[0] = da.x; dg[1] = da.y; dg[2] = da.z; dg[3] = da.w;
+                        dg[4] = db.x; dg[5] = db.y; dg[6] = db.z; dg[7] = db.w;
+                        tc::tmem_ld8(tl + cSXO + 128 * s + i0, x);
                     }
 #pragma unroll
-                    for (int j = 0; j < 16; j += 2) {
+                    for (int j = 0; j < 8; j += 2) {
                         const int i = i0 + j;              // token row of V: swizzle depends on i & 7 only
                         const float y0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sV + voff[i & 7] + (i >> 3) * 1024));
                         const float y1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sV + voff[(i + 1) & 7] + ((i + 1) >> 3) * 1024));
                         const float r0 = REG ? y0 - dg[j] * x[j] : y0;
                         const float r1 = REG ? y1 - dg[j + 1] * x[j + 1] : y1;
-                        pk[8 * hh + (j >> 1)] = pack_bf16x2(r0, r1);
+                        pk[4 * hh + (j >> 1)] = pack_bf16x2(r0, r1);
                     }
                 }
                 tc::tmem_st16(tl + cSR + 16 * hf, pk);
