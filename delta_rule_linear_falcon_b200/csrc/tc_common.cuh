@@ -75,11 +75,12 @@ TC_DEV bool mbar_test(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
-// Bounded wait for the phase with the given parity. Gives up after
-// `budget_cycles` SM clocks (or at once if the CTA is already aborting) and
-// reports that by returning false.
+// Bounded wait for the phase with the given parity. A phase that is already complete (or completes
+// within the hardware's suspend window) returns at once; otherwise the wait gives up after
+// `budget_cycles` SM clocks, or as soon as the CTA is aborting, and reports that by returning false.
 TC_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, const volatile int *abort_flag,
                       long long budget_cycles) {
+    if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
