@@ -42,9 +42,14 @@
  *   R9 positive-decay renormalisation: only decay factors exp(g_i - g_j) with
  *      i >= j are ever formed, so each factor lies in (0, 1]; nothing is divided
  *      by a cumulative product of alphas.
+ *   R10 same-step association (flag OR_SAME_STEP in `rule`): the pair written at
+ *      step t is (phi(k_t), v_t), the association of Kaczmarz Linear Attention
+ *      (thelatestinai.com page, KLA abstract), which the authors' abstract names
+ *      as the alternative to the prefix-aligned pair. k_prev is then not used as
+ *      a key; k_last is still the last key.
  *
  * Indices below are 0-based: pair j has x_j = k_{j-1} (j >= 1), x_0 = k_prev
- * or 0, and y_j = v_j.
+ * or 0 (same-step association: x_j = k_j), and y_j = v_j.
  *
  * Layout: q, k (B,H,T,dk); v, o (B,H,T,dv); alpha, eta (B,H,T);
  *         S0, S_out (B,H,dv,dk) with S[i][c] the weight from key coordinate c
@@ -61,21 +66,26 @@
 #define OR_RULE_1A 2
 #define OR_RULE_3 3
 #define OR_RULE_3A 4
+#define OR_SAME_STEP 0x100 /* flag bit in `rule`: reading R10 */
 
 #define OR_OK 0
 #define OR_EINVAL -1
 #define OR_ENOMEM -2
 
+static int base_rule(int rule) { return rule & ~OR_SAME_STEP; }
+static int same_step(int rule) { return (rule & OR_SAME_STEP) != 0; }
+
 static int rule_ok(int rule) {
-    return rule == OR_RULE_1 || rule == OR_RULE_1A || rule == OR_RULE_3 || rule == OR_RULE_3A;
+    const int b = base_rule(rule);
+    return b == OR_RULE_1 || b == OR_RULE_1A || b == OR_RULE_3 || b == OR_RULE_3A;
 }
 
 /* The regression family (Falcon-1, Falcon-3) versus the inner-product family. */
-static int is_regression(int rule) { return rule == OR_RULE_1 || rule == OR_RULE_3; }
+static int is_regression(int rule) { return base_rule(rule) == OR_RULE_1 || base_rule(rule) == OR_RULE_3; }
 
 /* Falcon-1 and Falcon-1A write one pair per step; Falcon-3 and -3A a window. */
 static int eff_window(int rule, int window) {
-    return (rule == OR_RULE_3 || rule == OR_RULE_3A) ? window : 1;
+    return (base_rule(rule) == OR_RULE_3 || base_rule(rule) == OR_RULE_3A) ? window : 1;
 }
 
 static double dotd(const double *a, const double *b, int n) {
@@ -84,9 +94,15 @@ static double dotd(const double *a, const double *b, int n) {
     return s;
 }
 
-/* x_j: the key half of pair j (prefix-aligned pair of the abstract; reading R6). */
-static void pair_key(double *x, const double *kh, const double *kprev_h, long j, int dk) {
-    if (j >= 1)
+/* x_j: the key half of pair j (prefix-aligned pair of the abstract, reading R6; same-step
+ * association k_j when `same` is set, reading R10). */
+static void pair_key(double *x, const double *kh, const double *kprev_h, long j, int dk, int same) {
+    if (same) {
+        if (j >= 0)
+            memcpy(x, kh + (size_t)j * dk, sizeof(double) * dk);
+        else
+            memset(x, 0, sizeof(double) * dk);
+    } else if (j >= 1)
         memcpy(x, kh + (size_t)(j - 1) * dk, sizeof(double) * dk);
     else if (j == 0 && kprev_h)
         memcpy(x, kprev_h, sizeof(double) * dk);
@@ -104,7 +120,7 @@ static int check_args(int rule, int B, int H, int T, int dk, int dv, int window,
                       const double *q, const double *k, const double *v,
                       const double *alpha, const double *eta) {
     if (!rule_ok(rule) || B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return 0;
-    if ((rule == OR_RULE_3 || rule == OR_RULE_3A) && window < 1) return 0;
+    if ((base_rule(rule) == OR_RULE_3 || base_rule(rule) == OR_RULE_3A) && window < 1) return 0;
     if ((size_t)B * H * T > 0 && (!q || !k || !v || !alpha || !eta)) return 0;
     return 1;
 }
@@ -139,7 +155,7 @@ static int recurrent_head(int rule, int T, int dk, int dv, const double *q, cons
 
         double nsum = 0.0;
         for (int m = 0; m < w; ++m) {
-            pair_key(X + (size_t)m * dk, k, kprev, t - m, dk);
+            pair_key(X + (size_t)m * dk, k, kprev, t - m, dk, same_step(rule));
             nsum += dotd(X + (size_t)m * dk, X + (size_t)m * dk, dk);
         }
         const double beta = step_size(eta[t], nsum, eps);
@@ -226,7 +242,7 @@ static int blocked_head(int rule, int T, int dk, int dv, const double *q, const 
             for (int m = 0; m < w; ++m) {
                 const int e = s * w + m;
                 const long j = c0 + s - m;
-                pair_key(Xe + (size_t)e * dk, k, kprev, j, dk);
+                pair_key(Xe + (size_t)e * dk, k, kprev, j, dk, same_step(rule));
                 if (j >= 0) memcpy(Ye + (size_t)e * dv, v + (size_t)j * dv, sizeof(double) * dv);
                 else memset(Ye + (size_t)e * dv, 0, sizeof(double) * dv);
             }

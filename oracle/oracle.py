@@ -15,6 +15,7 @@ import threading
 import numpy as np
 
 RULE_1, RULE_1A, RULE_3, RULE_3A = 1, 2, 3, 4
+SAME_STEP = 0x100  # flag OR-ed into a rule: pair (k_t, v_t) at step t (same-step association)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "falcon_oracle.c")
