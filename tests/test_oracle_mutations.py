@@ -16,8 +16,8 @@ SRC = os.path.join(os.path.dirname(orc.__file__), "falcon_oracle.c")
 # (name, original text, mutated text) or (name, [(original, mutated), ...])
 MUTANTS = [
     ("same-step pairing (k_t instead of k_{t-1})",
-     "pair_key(X + (size_t)m * dk, k, kprev, t - m, dk);",
-     "pair_key(X + (size_t)m * dk, k, kprev, t - m + 1, dk);"),
+     "pair_key(X + (size_t)m * dk, k, kprev, t - m, dk, same_step(rule));",
+     "pair_key(X + (size_t)m * dk, k, kprev, t - m + 1, dk, same_step(rule));"),
     ("no decay in the recurrence",
      "S[i] *= a; /* Sbar = alpha_t S */", "(void)a;"),
     ("normaliser ignores the key norm",
