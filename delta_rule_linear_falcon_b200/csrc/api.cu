@@ -46,9 +46,11 @@ bool device_info(int **err, int *sms) {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
-bool rule_valid(int r) { return r >= FALCON_RULE_1 && r <= FALCON_RULE_3A; }
-bool is_regression(int r) { return r == FALCON_RULE_1 || r == FALCON_RULE_3; }
-bool is_windowed(int r) { return r == FALCON_RULE_3 || r == FALCON_RULE_3A; }
+int base_rule(int r) { return r & ~FALCON_SAME_STEP; }
+bool same_step(int r) { return (r & FALCON_SAME_STEP) != 0; }
+bool rule_valid(int r) { return base_rule(r) >= FALCON_RULE_1 && base_rule(r) <= FALCON_RULE_3A; }
+bool is_regression(int r) { return base_rule(r) == FALCON_RULE_1 || base_rule(r) == FALCON_RULE_3; }
+bool is_windowed(int r) { return base_rule(r) == FALCON_RULE_3 || base_rule(r) == FALCON_RULE_3A; }
 
 // Checks shared by the two sequence entry points.
 falcon_status_t check_seq_args(const falcon_args_t *a) {
@@ -137,6 +139,7 @@ falcon_status_t falcon_fwd_chunk(const falcon_args_t *a, void *workspace, size_t
     p.window = w;
     p.tok_per_blk = a->chunk / w;
     p.regression = is_regression(a->rule);
+    p.same_step = same_step(a->rule);
     p.io_bf16 = a->io_dtype == FALCON_BF16;
     p.q = a->q; p.k = a->k; p.v = a->v; p.k_prev = a->k_prev;
     p.alpha = a->alpha; p.eta = a->eta; p.S0 = a->S0; p.eps = a->eps;
@@ -158,6 +161,7 @@ falcon_status_t falcon_fwd_recurrent(const falcon_args_t *a, falcon_stream_t str
     RecParams p{};
     p.B = a->B; p.H = a->H; p.T = a->T; p.dk = a->dk; p.dv = a->dv; p.window = w;
     p.regression = is_regression(a->rule);
+    p.same_step = same_step(a->rule);
     p.io_bf16 = a->io_dtype == FALCON_BF16;
     p.q = a->q; p.k = a->k; p.v = a->v; p.k_prev = a->k_prev;
     p.alpha = a->alpha; p.eta = a->eta; p.S0 = a->S0; p.eps = a->eps;
@@ -190,6 +194,7 @@ falcon_status_t falcon_decode_step(int rule, int io_dtype, int N, int H, int dk,
     DecodeParams p{};
     p.N = N; p.H = H; p.dk = dk; p.dv = dv;
     p.regression = is_regression(rule);
+    p.same_step = same_step(rule);
     p.io_bf16 = io_dtype == FALCON_BF16;
     p.S = S; p.k_prev = k_prev; p.q = q; p.k = k; p.v = v;
     p.alpha = alpha; p.eta = eta; p.eps = eps; p.o = o;

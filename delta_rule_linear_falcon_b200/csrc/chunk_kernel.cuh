@@ -153,7 +153,9 @@ chunk_fwd_kernel(ChunkParams p) {
                 const int s = e / W, m = e % W;
                 const long j = (long)t0 + s - m;
                 if (s < nval) {
-                    if (j >= 1) Io<IO>::ld8(k, (size_t)(j - 1) * DK + ch * 8, x8);
+                    if (p.same_step) {                  // pair j holds k_j
+                        if (j >= 0) Io<IO>::ld8(k, (size_t)j * DK + ch * 8, x8);
+                    } else if (j >= 1) Io<IO>::ld8(k, (size_t)(j - 1) * DK + ch * 8, x8);
                     else if (j == 0 && kp) Io<IO>::ld8(kp, (size_t)ch * 8, x8);
                 }
             }

@@ -344,6 +344,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             // precedes the chain's read of V_{j-3} that frees the slot of V_{j-1}, so the blocking waits
             // below never hold back a load that could already start.
             int kx = 0, kv = 0;
+            const int kshift = p.same_step ? 0 : 1;   // prefix-aligned key rows of block j start at t0 - 1
             for (int j = 0; j <= nblk && !*abort_flag; ++j) {
                 if (j < nblk) {
                     if (j >= 3 && !tc::mbar_wait(&bars[B_XQFREE + j % 3], ((j / 3) - 1) & 1, abort_flag, kWaitBudget)) {
@@ -354,8 +355,8 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                     uint64_t *fb = &bars[B_FULLXQ + j % 3];
                     const int t0 = j * kBlk;
                     tc::mbar_arrive_expect_tx(fb, kXQ);
-                    tc::tma_load_3d(dst + 0, &tmK, 0, t0 - 1, bh, fb);
-                    tc::tma_load_3d(dst + 16384, &tmK, 64, t0 - 1, bh, fb);
+                    tc::tma_load_3d(dst + 0, &tmK, 0, t0 - kshift, bh, fb);
+                    tc::tma_load_3d(dst + 16384, &tmK, 64, t0 - kshift, bh, fb);
                     tc::tma_load_3d(dst + 8192, &tmQ, 0, t0, bh, fb);
                     tc::tma_load_3d(dst + 16384 + 8192, &tmQ, 64, t0, bh, fb);
                     kx = j + 1;
@@ -502,7 +503,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             if (c >= 4 && !role_wait(&bars[B_SCALFREE + u4], ((c >> 2) - 1) & 1, leader, 1, 64)) return false;
             if (!role_wait(&bars[B_FULLXQ + u3], (c / 3) & 1, leader, 1, 64)) return false;
             const int t0 = c * kBlk, nval = min(kBlk, T - t0);
-            if (c == 0 && p.k_prev && ht < 16) {
+            if (c == 0 && p.k_prev && !p.same_step && ht < 16) {
                 const uint4 v = *reinterpret_cast<const uint4 *>(
                     reinterpret_cast<const __nv_bfloat16 *>(p.k_prev) + (size_t)bh * D + ht * 8);
                 *reinterpret_cast<uint4 *>(xq + (ht >> 3) * 16384 + (ht & 7) * 16) = v;

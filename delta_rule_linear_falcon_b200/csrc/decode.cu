@@ -2,7 +2,8 @@
 // (sequence, head), with the fp32 state read and written in place.
 //
 // For one head, with x = k_prev (the prefix-aligned key, "Fast Weight
-// Attention for Continual Learning", authors' abstract) and y = v:
+// Attention for Continual Learning", authors' abstract; x = k for the same-step
+// association of Kaczmarz Linear Attention) and y = v:
 //   beta = eta / (||x||^2 + eps)
 //   r_i  = S_i . x,   s_i = S_i . q          (one pass over row i of S)
 //   Falcon-1:  u_i = beta (y_i - alpha r_i)   Falcon-1A:  u_i = beta y_i
@@ -76,9 +77,10 @@ decode_kernel(DecodeParams p) {
     IO *oh = reinterpret_cast<IO *>(p.o) + nh * (size_t)dv;
 
     float x[VPL], qv[VPL];
+    const IO *xs = p.same_step ? kh : kp;   // same-step association: the current key
 #pragma unroll
     for (int j = 0; j < VPL; ++j) {
-        x[j] = Io<IO>::ld(kp, lane * VPL + j);
+        x[j] = Io<IO>::ld(xs, lane * VPL + j);
         qv[j] = Io<IO>::ld(qh, lane * VPL + j);
     }
     float xx = 0.f, xq = 0.f;

@@ -10,6 +10,7 @@ namespace falcon {
 struct RecParams {
     int B, H, T, dk, dv, window;  // window = 1 for Falcon-1/1A
     bool regression, io_bf16;
+    bool same_step;               // pair (k_t, v_t) instead of (k_{t-1}, v_t)
     const void *q, *k, *v, *k_prev;
     const float *alpha, *eta, *S0;
     float eps;
@@ -21,6 +22,7 @@ struct RecParams {
 struct DecodeParams {
     int N, H, dk, dv;
     bool regression, io_bf16;
+    bool same_step;  // x = k instead of the cached k_prev
     float *S;
     void *k_prev;
     const void *q, *k, *v;
@@ -35,6 +37,7 @@ struct ChunkParams {
     int window;      // pairs per step (1 for Falcon-1/1A)
     int tok_per_blk; // tokens per block; rows per block = tok_per_blk * window <= 64
     bool regression, io_bf16;
+    bool same_step;  // pair (k_t, v_t) instead of (k_{t-1}, v_t)
     const void *q, *k, *v, *k_prev;
     const float *alpha, *eta, *S0;
     float eps;

@@ -51,6 +51,7 @@ recurrent_kernel(RecParams p) {
     // registers holding the inputs of the step about to be staged
     auto load_x = [&](int t) -> float {   // key half of pair t, coordinate tid
         if (tid >= dk) return 0.f;
+        if (p.same_step) return Io<IO>::ld(k, (size_t)t * dk + tid);
         if (t >= 1) return Io<IO>::ld(k, (size_t)(t - 1) * dk + tid);
         return kp ? Io<IO>::ld(kp, tid) : 0.f;
     };

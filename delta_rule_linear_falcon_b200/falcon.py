@@ -20,6 +20,7 @@ FALCON_OK, FALCON_ERR_INVALID_ARG, FALCON_ERR_UNSUPPORTED = 0, 1, 2
 FALCON_ERR_WORKSPACE, FALCON_ERR_CUDA, FALCON_ERR_TIMEOUT = 3, 4, 5
 FALCON_RULE_1, FALCON_RULE_1A, FALCON_RULE_3, FALCON_RULE_3A = 1, 2, 3, 4
 FALCON_F32, FALCON_BF16 = 0, 1
+FALCON_SAME_STEP = 0x100  # OR into a rule code: pair (k_t, v_t) at step t (same-step association)
 RULES = {"falcon1": FALCON_RULE_1, "falcon1a": FALCON_RULE_1A, "falcon3": FALCON_RULE_3,
          "falcon3a": FALCON_RULE_3A}
 
@@ -115,7 +116,12 @@ def _need(t, name, dtype=None):
 
 
 def _rule_code(rule) -> int:
-    return RULES[rule] if isinstance(rule, str) else int(rule)
+    """A rule name or code; FALCON_SAME_STEP may be OR-ed into a code, or a name may end in
+    '+same_step'."""
+    if isinstance(rule, str):
+        name, _, flag = rule.partition("+")
+        return RULES[name] | (FALCON_SAME_STEP if flag == "same_step" else 0)
+    return int(rule)
 
 
 def make_args(q, k, v, alpha, eta, *, rule, eps=1e-6, window=1, chunk=64, S0=None, k_prev=None,

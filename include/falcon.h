@@ -74,12 +74,22 @@ typedef enum {
     FALCON_RULE_3A = 4  /* Falcon-3A: windowed inner-product write (window w)     */
 } falcon_rule_t;
 
+/*
+ * Flag OR-ed into a rule value (the `rule` field, or the `rule` argument of
+ * falcon_decode_step): write the same-step pair (k_t, v_t) at step t, the
+ * association of Kaczmarz Linear Attention (thelatestinai.com page of "Fast Weight
+ * Attention for Continual Learning", KLA abstract), instead of the prefix-aligned
+ * pair (k_{t-1}, v_t) of the authors' abstract. k_prev is then not used as a key
+ * (k_last is still the last key, and the decode step still stores k into k_prev).
+ */
+#define FALCON_SAME_STEP 0x100
+
 typedef enum { FALCON_F32 = 0, FALCON_BF16 = 1 } falcon_dtype_t;
 
 /* Arguments of the two sequence entry points. Integer fields hold the enums
  * above. */
 typedef struct {
-    int rule;           /* falcon_rule_t                                             */
+    int rule;           /* falcon_rule_t, optionally | FALCON_SAME_STEP               */
     int io_dtype;       /* falcon_dtype_t of q, k, v, k_prev, k_last and o            */
     int B, H, T;        /* batch, heads, tokens (T >= 0)                              */
     int dk, dv;         /* key/query and value widths                                 */
@@ -92,7 +102,8 @@ typedef struct {
     int window;         /* Falcon-3/3A window w >= 1; ignored by Falcon-1/1A           */
     int chunk;          /* chunk-parallel block: 16, 32 or 64 pseudo-value rows        */
     const float *S0;    /* (B,H,dv,dk) initial state, or NULL for zero                 */
-    const void *k_prev; /* (B,H,dk) key cached before this segment, or NULL (x_1 = 0) */
+    const void *k_prev; /* (B,H,dk) key cached before this segment, or NULL (x_1 = 0);
+                           not read with FALCON_SAME_STEP                              */
     void *o;            /* (B,H,T,dv) output, written                                  */
     float *S_out;       /* (B,H,dv,dk) final state, or NULL                            */
     void *k_last;       /* (B,H,dk) last key (the cache for a continuation), or NULL   */
@@ -144,7 +155,7 @@ FALCON_API falcon_status_t falcon_fwd_recurrent(const falcon_args_t *args, falco
  * Attention for Continual Learning" lists for streaming inference (section
  * Why This Matters).
  *
- *   x = k_prev; beta = eta / (||x||^2 + eps); Sbar = alpha S
+ *   x = k_prev (x = k with FALCON_SAME_STEP); beta = eta / (||x||^2 + eps); Sbar = alpha S
  *   Falcon-1:  S <- Sbar - beta (Sbar x - v) x^T     Falcon-1A: S <- Sbar + beta v x^T
  *   o = S q;   k_prev <- k
  *
