@@ -353,6 +353,56 @@ def bench_recurrent(args, D: Dist):
             "tokens_per_s": round(B * T / (ms * 1e-3), 1), "note": "latency bound, parity workload"}
 
 
+def bench_more_chunk(args, D: Dist):
+    """Secondary chunk workloads (rank 0, device-resident inputs, CUDA events): Falcon-3 and
+    Falcon-3A (w = 4, B4 H16 T8192 d128), Falcon-1A on B1 H16 T32768 d128, and the benchmark
+    workload with the same-step flag."""
+    import torch
+    from delta_rule_linear_falcon_b200 import falcon as F
+    from delta_rule_linear_falcon_b200 import inputs as I
+
+    dev = torch.device("cuda", D.local)
+    stream = torch.cuda.current_stream(dev)
+    hbm, _, _ = peaks()
+    out = {}
+
+    def timed(s, rule, label):
+        q, k, v = (torch.from_numpy(x).to(torch.bfloat16).to(dev) for x in (s.q, s.k, s.v))
+        a, e = (torch.from_numpy(x).to(dev) for x in (s.alpha, s.eta))
+        run = lambda: F.falcon_fwd_chunk(q, k, v, a, e, rule=rule, eps=s.eps, window=s.window, chunk=64,
+                                         stream=stream)
+        for _ in range(2):
+            run()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = 5
+        t0.record(stream)
+        for _ in range(n):
+            run()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        assert F.falcon_check_device_errors(stream) == F.FALCON_OK
+        ms = t0.elapsed_time(t1) / n
+        B, H, T, dk, dv = s.shape
+        nbytes = chunk_algorithmic_bytes(B, H, T, dk, dv)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[label] = {"workload": label, "ms_per_launch": round(ms, 4),
+                      "tokens_per_s": round(B * T / (ms * 1e-3), 1), "gbs_algorithmic": round(gbs, 1),
+                      "roofline_frac": round(gbs / hbm, 4), "launches": n}
+        del q, k, v, a, e
+
+    s3 = I.workload_chunk_f3()
+    timed(s3, 3, "falcon3_w4_chunk_bf16_B4H16T8192d128")
+    timed(s3, 4, "falcon3a_w4_chunk_bf16_B4H16T8192d128")
+    del s3
+    s2 = I.workload_chunk_f1a_long()
+    timed(s2, 2, "falcon1a_chunk_bf16_B1H16T32768d128")
+    del s2
+    s1 = I.workload_chunk_f1(B=args.batch, T=args.seq_len)
+    timed(s1, 1 | F.FALCON_SAME_STEP, f"falcon1_same_step_chunk_bf16_B{args.batch}H16T{args.seq_len}d128")
+    return out
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 
 _SAMPLE_CACHE = {}
@@ -467,6 +517,7 @@ def main(argv=None):
     ch = bench_chunk(args, D, clk)
     dec = bench_decode(args, D, clk)
     rec = bench_recurrent(args, D) if D.rank == 0 else None
+    more = bench_more_chunk(args, D) if D.rank == 0 else None
 
     s = ch["s"]
     B, H, T, dk, dv = s.shape
@@ -512,6 +563,8 @@ def main(argv=None):
     }
     if rec is not None:
         line["recurrent"] = rec
+    if more is not None:
+        line["more_chunk"] = more
     if D.rank == 0 and D.world == 1:
         line["cpu_baseline"] = cpu_baseline(min_seconds=10.0)
     if D.rank == 0:
