@@ -543,7 +543,7 @@ def main(argv=None):
                      "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else src,
                      "algorithmic_bytes_per_launch": nbytes, "kernel": "chunk_ws_kernel",
                      "kernel_ms": round(ch["kern_ms"], 4)},
-        "north_star_roofline": {"flops": flops, "bytes": nbytes, "t_roofline_us": round(t_roof * 1e6, 2),
+        "roofline_flops_and_bytes": {"flops": flops, "bytes": nbytes, "t_roofline_us": round(t_roof * 1e6, 2),
                                 "frac": round(t_roof / (ch["kern_ms"] * 1e-3), 4),
                                 "tflops": round(flops / (ch["kern_ms"] * 1e-3) / 1e12, 2),
                                 "definition": "max(FLOPs/bf16 peak, bytes/HBM peak) / kernel time, "
