@@ -369,8 +369,15 @@ def bench_more_chunk(args, D: Dist):
     def timed(s, rule, label):
         q, k, v = (torch.from_numpy(x).to(torch.bfloat16).to(dev) for x in (s.q, s.k, s.v))
         a, e = (torch.from_numpy(x).to(dev) for x in (s.alpha, s.eta))
+        B, H, T, dk, dv = s.shape
+        o = torch.empty_like(v)
+        S = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+        kl = torch.empty((B, H, dk), dtype=torch.bfloat16, device=dev)
+        need = F.falcon_workspace_size(F.make_args(q, k, v, a, e, rule=rule, eps=s.eps, window=s.window,
+                                                   chunk=64, o=o, S_out=S, k_last=kl))
+        ws = torch.empty(need, dtype=torch.uint8, device=dev) if need else None
         run = lambda: F.falcon_fwd_chunk(q, k, v, a, e, rule=rule, eps=s.eps, window=s.window, chunk=64,
-                                         stream=stream)
+                                         o=o, S_out=S, k_last=kl, workspace=ws, stream=stream)
         for _ in range(2):
             run()
         torch.cuda.synchronize()
@@ -383,13 +390,14 @@ def bench_more_chunk(args, D: Dist):
         torch.cuda.synchronize()
         assert F.falcon_check_device_errors(stream) == F.FALCON_OK
         ms = t0.elapsed_time(t1) / n
-        B, H, T, dk, dv = s.shape
         nbytes = chunk_algorithmic_bytes(B, H, T, dk, dv)
         gbs = nbytes / (ms * 1e-3) / 1e9
         out[label] = {"workload": label, "ms_per_launch": round(ms, 4),
                       "tokens_per_s": round(B * T / (ms * 1e-3), 1), "gbs_algorithmic": round(gbs, 1),
-                      "roofline_frac": round(gbs / hbm, 4), "launches": n}
-        del q, k, v, a, e
+                      "roofline_frac": round(gbs / hbm, 4), "launches": n,
+                      # the sequence split of the inner-product rule: state pass, scan, chunk kernel
+                      "kernels_per_call": 3 if need else 1, "workspace_bytes": need}
+        del q, k, v, a, e, o, S, kl, ws
 
     s3 = I.workload_chunk_f3()
     timed(s3, 3, "falcon3_w4_chunk_bf16_B4H16T8192d128")

@@ -94,6 +94,21 @@ int pick_value_slice(long long bh, int dv, int num_sms) {
     return best;
 }
 
+// Launch parameters of the chunk-parallel pass from checked arguments.
+ChunkParams chunk_params(const falcon_args_t *a) {
+    ChunkParams p{};
+    p.B = a->B; p.H = a->H; p.T = a->T; p.dk = a->dk; p.dv = a->dv;
+    p.window = is_windowed(a->rule) ? a->window : 1;
+    p.tok_per_blk = a->chunk / p.window;
+    p.regression = is_regression(a->rule);
+    p.same_step = same_step(a->rule);
+    p.io_bf16 = a->io_dtype == FALCON_BF16;
+    p.q = a->q; p.k = a->k; p.v = a->v; p.k_prev = a->k_prev;
+    p.alpha = a->alpha; p.eta = a->eta; p.S0 = a->S0; p.eps = a->eps;
+    p.o = a->o; p.k_last = a->k_last; p.S_out = a->S_out;
+    return p;
+}
+
 }  // namespace
 
 cudaError_t launch_chunk_dk32(const ChunkParams &p, int dvs, cudaStream_t s);
@@ -117,37 +132,38 @@ using namespace falcon;
 
 extern "C" {
 
-size_t falcon_workspace_size(const falcon_args_t *args) {
-    (void)args;
-    return 0;  // the fused chunk kernel keeps every intermediate on chip
+size_t falcon_workspace_size(const falcon_args_t *a) {
+    if (!a || check_seq_args(a) != FALCON_OK) return 0;
+    if (!dim_supported_chunk(a->dk) || !dim_supported_chunk(a->dv)) return 0;
+    if (a->chunk != 16 && a->chunk != 32 && a->chunk != 64) return 0;
+    if ((long long)a->B * a->H == 0) return 0;
+    ChunkParams p = chunk_params(a);
+    int sms = 0;
+    if (!device_info(&p.err, &sms)) return 0;
+    return seg_plan(p, sms).bytes;
 }
 
 falcon_status_t falcon_fwd_chunk(const falcon_args_t *a, void *workspace, size_t workspace_bytes,
                                  falcon_stream_t stream) {
     falcon_status_t st = check_seq_args(a);
     if (st != FALCON_OK) return st;
-    (void)workspace;
-    if (workspace_bytes < falcon_workspace_size(a)) return FALCON_ERR_WORKSPACE;
     if (!dim_supported_chunk(a->dk) || !dim_supported_chunk(a->dv)) return FALCON_ERR_UNSUPPORTED;
     if (a->chunk != 16 && a->chunk != 32 && a->chunk != 64) return FALCON_ERR_UNSUPPORTED;
     const int w = is_windowed(a->rule) ? a->window : 1;
     if (w > a->chunk) return FALCON_ERR_UNSUPPORTED;
     if ((long long)a->B * a->H == 0) return FALCON_OK;
 
-    ChunkParams p{};
-    p.B = a->B; p.H = a->H; p.T = a->T; p.dk = a->dk; p.dv = a->dv;
-    p.window = w;
-    p.tok_per_blk = a->chunk / w;
-    p.regression = is_regression(a->rule);
-    p.same_step = same_step(a->rule);
-    p.io_bf16 = a->io_dtype == FALCON_BF16;
-    p.q = a->q; p.k = a->k; p.v = a->v; p.k_prev = a->k_prev;
-    p.alpha = a->alpha; p.eta = a->eta; p.S0 = a->S0; p.eps = a->eps;
-    p.o = a->o; p.k_last = a->k_last; p.S_out = a->S_out;
+    ChunkParams p = chunk_params(a);
     int sms = 0;
     if (!device_info(&p.err, &sms)) return FALCON_ERR_CUDA;
-    return launch_chunk(p, sms, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? FALCON_OK
-                                                                                      : FALCON_ERR_CUDA;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const SegPlan plan = seg_plan(p, sms);
+    if (plan.nseg > 1) {
+        if (!workspace || workspace_bytes < plan.bytes) return FALCON_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return FALCON_ERR_INVALID_ARG;
+        return launch_chunk_seg(p, plan, workspace, s) == cudaSuccess ? FALCON_OK : FALCON_ERR_CUDA;
+    }
+    return launch_chunk(p, sms, s) == cudaSuccess ? FALCON_OK : FALCON_ERR_CUDA;
 }
 
 falcon_status_t falcon_fwd_recurrent(const falcon_args_t *a, falcon_stream_t stream) {

@@ -54,4 +54,15 @@ cudaError_t launch_chunk(const ChunkParams &p, int num_sms, cudaStream_t s);
 bool chunk_ws_supported(const ChunkParams &p);
 cudaError_t launch_chunk_ws(const ChunkParams &p, cudaStream_t s);
 
+// Sequence split of the inner-product rule (seg_state.cu): the segments of each head run
+// as heads of their own, started from states that a parallel pass and a scan provide.
+struct SegPlan {
+    int nseg = 1;       // segments per head (1: no split)
+    int L = 0;          // tokens per segment, whole 64-token blocks
+    int piece = 0;      // tokens per piece of the state pass; divides L
+    size_t bytes = 0;   // device workspace the split needs
+};
+SegPlan seg_plan(const ChunkParams &p, int num_sms);
+cudaError_t launch_chunk_seg(const ChunkParams &p, const SegPlan &plan, void *workspace, cudaStream_t s);
+
 }  // namespace falcon

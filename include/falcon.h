@@ -110,9 +110,13 @@ typedef struct {
 } falcon_args_t;
 
 /*
- * Bytes of device workspace falcon_fwd_chunk needs for these arguments
- * (0 when it needs none). Returns 0 for invalid arguments as well; the call
- * itself reports those.
+ * Bytes of device workspace falcon_fwd_chunk needs for these arguments on the
+ * current device (0 when it needs none). Returns 0 for invalid arguments as
+ * well; the call itself reports those. Nonzero only for the sequence split of
+ * the inner-product rules described at falcon_fwd_chunk: about
+ * (B*H*T/piece + B*H*nseg) * dv*dk*4 bytes, a few tens of MB for 16 heads of
+ * 32768 tokens. The caller allocates it (16-byte aligned) and owns it; the
+ * call only uses it while its kernels run on `stream`.
  */
 FALCON_API size_t falcon_workspace_size(const falcon_args_t *args);
 
@@ -133,8 +137,19 @@ FALCON_API size_t falcon_workspace_size(const falcon_args_t *args);
  * 1 <= window <= chunk and process floor(chunk / window) tokens per block.
  * Tensor-core products take bf16 operands with fp32 accumulation and an fp32
  * state, whatever io_dtype is; use falcon_fwd_recurrent for fp32-accurate work.
+ *
+ * Sequence split (inner-product write, window 1, dk = dv = 128, bf16, chunk 64,
+ * T a multiple of 64, fewer heads than SMs): the additive write has a scalar
+ * state transition, so each head is cut into nseg segments of whole blocks;
+ * one parallel pass forms every piece's state increment
+ * sum_t 2^(G_end - G_t) beta_t y_t x_t^T and its decay, a scan gives the state
+ * at each segment start, and the segments then run as heads of their own.
+ * The result is the same up to rounding; falcon_workspace_size() says when
+ * this path is taken and how much workspace it needs.
+ *
  * `workspace` may be NULL when falcon_workspace_size() is 0.
- * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ * Errors: INVALID_ARG (also a workspace not 16-byte aligned), UNSUPPORTED,
+ * WORKSPACE (NULL or smaller than falcon_workspace_size()), CUDA.
  */
 FALCON_API falcon_status_t falcon_fwd_chunk(const falcon_args_t *args, void *workspace,
                                  size_t workspace_bytes, falcon_stream_t stream);
