@@ -154,6 +154,36 @@ FALCON_API size_t falcon_workspace_size(const falcon_args_t *args);
 FALCON_API falcon_status_t falcon_fwd_chunk(const falcon_args_t *args, void *workspace,
                                  size_t workspace_bytes, falcon_stream_t stream);
 
+/* Size of the fixed scratch array behind falcon_fwd_chunk_noalloc: 32 MiB. */
+#define FALCON_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/*
+ * falcon_fwd_chunk_noalloc -- falcon_fwd_chunk without a caller-provided
+ * workspace, for callers that cannot allocate device memory where they run
+ * the forward pass: a plugin that receives raw device pointers from a host
+ * runtime with no allocator to offer, a serving loop in which a cudaMalloc
+ * (which may synchronise the device) is not acceptable, or a process whose
+ * device memory is owned by a pool it does not control. The paper has no
+ * counterpart; this is a deployment convenience of this library.
+ *
+ * Arguments, results and errors are those of falcon_fwd_chunk. Where that call
+ * needs workspace (falcon_workspace_size() > 0), this one uses a fixed array of
+ * FALCON_NOALLOC_SCRATCH_BYTES in the library's device image instead; every
+ * GPU that loads the library holds that array until the process exits. Larger
+ * needs are rejected before anything runs with FALCON_ERR_WORKSPACE (use
+ * falcon_fwd_chunk with your own workspace then). The call allocates and frees
+ * nothing.
+ *
+ * The first call on each device resolves the array's device address (with that
+ * device current) and keeps it; make that first call before any stream
+ * capture. All calls share the one array per device: calls whose kernels can
+ * overlap on the GPU (different streams without an ordering between them,
+ * several host threads) race on it and give wrong results, so order them, for
+ * example on one stream. Nothing in the array needs clearing between calls:
+ * each call writes every byte it later reads.
+ */
+FALCON_API falcon_status_t falcon_fwd_chunk_noalloc(const falcon_args_t *args, falcon_stream_t stream);
+
 /*
  * falcon_fwd_recurrent -- recurrent form (authors' abstract; ai.info overview,
  * section Methodology in Plain English): the literal per-token recurrence
