@@ -239,11 +239,13 @@ seg_piece_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             }
             const float e = e_next;
             if (i + 1 < nst) e_next = eta_h[(i + 1) * kPBlk + tok];
+            // chunk c ^ (tok % 8) at step c: the eight rows of a 1024-byte group start their walk
+            // on eight different 16-byte positions, so a warp's loads spread over all 32 banks
             const uint4 *xr = reinterpret_cast<const uint4 *>(xa + roff);
             float nrm = 0.f;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-                const uint4 u = xr[c];
+                const uint4 u = xr[c ^ (tok & 7)];
                 nrm = sumsq_bf16x2(u.x, nrm);
                 nrm = sumsq_bf16x2(u.y, nrm);
                 nrm = sumsq_bf16x2(u.z, nrm);
@@ -254,12 +256,12 @@ seg_piece_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             uint4 *yr = reinterpret_cast<uint4 *>(ya + roff);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-                uint4 u = yr[c];
+                uint4 u = yr[c ^ (tok & 7)];
                 u.x = scale_bf16x2(u.x, w);
                 u.y = scale_bf16x2(u.y, w);
                 u.z = scale_bf16x2(u.z, w);
                 u.w = scale_bf16x2(u.w, w);
-                yr[c] = u;
+                yr[c ^ (tok & 7)] = u;
             }
             tc::fence_proxy_async();
             __syncwarp();
