@@ -159,7 +159,12 @@ def falcon_workspace_size(args: FalconArgs) -> int:
 def falcon_fwd_chunk(q, k, v, alpha, eta, *, rule, eps=1e-6, window=1, chunk=64, S0=None,
                      k_prev=None, o=None, S_out=None, k_last=None, want_state=True,
                      workspace=None, stream=None):
-    """Chunk-parallel forward pass. Returns (o, S_out, k_last)."""
+    """Chunk-parallel forward pass. Returns (o, S_out, k_last).
+
+    ``workspace`` is an optional contiguous CUDA tensor of at least
+    ``falcon_workspace_size(args)`` bytes (nonzero only where the library splits the
+    sequence of an inner-product problem with few heads); when it is needed and not
+    given, one is allocated here with torch for the call."""
     o, S_out, k_last = _outputs(k, v, o, S_out, k_last, want_state)
     args = make_args(q, k, v, alpha, eta, rule=rule, eps=eps, window=window, chunk=chunk, S0=S0,
                      k_prev=k_prev, o=o, S_out=S_out, k_last=k_last)
