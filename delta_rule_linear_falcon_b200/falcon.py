@@ -164,7 +164,9 @@ def falcon_fwd_chunk(q, k, v, alpha, eta, *, rule, eps=1e-6, window=1, chunk=64,
     ``workspace`` is an optional contiguous CUDA tensor of at least
     ``falcon_workspace_size(args)`` bytes (nonzero only where the library splits the
     sequence of an inner-product problem with few heads); when it is needed and not
-    given, one is allocated here with torch for the call."""
+    given, one is allocated here with torch for the call (on the current stream, recorded
+    on ``stream`` when that is another torch stream; pass your own when ``stream`` is a raw
+    handle of a different stream)."""
     o, S_out, k_last = _outputs(k, v, o, S_out, k_last, want_state)
     args = make_args(q, k, v, alpha, eta, rule=rule, eps=eps, window=window, chunk=chunk, S0=S0,
                      k_prev=k_prev, o=o, S_out=S_out, k_last=k_last)
@@ -176,6 +178,10 @@ def falcon_fwd_chunk(q, k, v, alpha, eta, *, rule, eps=1e-6, window=1, chunk=64,
     elif need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=k.device)
         ws_ptr, ws_bytes = workspace.data_ptr(), need
+        if isinstance(stream, torch.cuda.Stream):
+            # the caching allocator may hand the block out again once this call returns; tie its
+            # reuse to the kernels queued on the caller's stream
+            workspace.record_stream(stream)
     st = lib().falcon_fwd_chunk(ctypes.byref(args), ws_ptr, ws_bytes, _stream(stream))
     if st != FALCON_OK:
         raise FalconError(st, "falcon_fwd_chunk")
