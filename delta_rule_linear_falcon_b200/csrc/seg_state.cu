@@ -299,23 +299,41 @@ seg_piece_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
 }
 
 // grid (16, heads) x 256 threads: each thread carries 4 consecutive entries of one head's
-// 128 x 128 state through the pieces in order.
+// 128 x 128 state through the pieces in order; the increments of four pieces are loaded
+// before they are applied, so their loads overlap.
 __global__ void __launch_bounds__(256) seg_scan_kernel(ScanParams p) {
     constexpr int E = 128 * 128;
     const int head = blockIdx.y;
     const int e = (blockIdx.x * 256 + threadIdx.x) * 4;
     float4 S = p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + (size_t)head * E + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sg = 0; sg < p.nseg; ++sg) {
-        *reinterpret_cast<float4 *>(p.Sinit + ((size_t)head * p.nseg + sg) * E + e) = S;
-        if (sg + 1 == p.nseg && !p.S_out) break;
-        for (int j = 0; j < p.pps; ++j) {
-            const size_t pc = (size_t)head * p.ptot + (size_t)sg * p.pps + j;
-            const float f = exp2f(fminf(p.a[pc], 0.f));
-            const float4 d = *reinterpret_cast<const float4 *>(p.D + pc * E + e);
-            S = make_float4(fmaf(f, S.x, d.x), fmaf(f, S.y, d.y), fmaf(f, S.z, d.z), fmaf(f, S.w, d.w));
+    // pieces read: all of them when the final state is wanted, else all but the last segment's
+    const int np = (p.S_out ? p.nseg : p.nseg - 1) * p.pps;
+    const size_t pbase = (size_t)head * p.ptot;
+    for (int pc0 = 0; pc0 < np; pc0 += 4) {
+        float4 d[4];
+        float f[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (pc0 + u < np) {
+                d[u] = *reinterpret_cast<const float4 *>(p.D + (pbase + pc0 + u) * E + e);
+                f[u] = exp2f(fminf(p.a[pbase + pc0 + u], 0.f));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int pc = pc0 + u;
+            if (pc < np) {
+                if (pc % p.pps == 0)   // first piece of segment pc / pps: its starting state
+                    *reinterpret_cast<float4 *>(p.Sinit + ((size_t)head * p.nseg + pc / p.pps) * E + e) = S;
+                S = make_float4(fmaf(f[u], S.x, d[u].x), fmaf(f[u], S.y, d[u].y), fmaf(f[u], S.z, d[u].z),
+                                fmaf(f[u], S.w, d[u].w));
+            }
         }
     }
-    if (p.S_out) *reinterpret_cast<float4 *>(p.S_out + (size_t)head * E + e) = S;
+    if (p.S_out)
+        *reinterpret_cast<float4 *>(p.S_out + (size_t)head * E + e) = S;
+    else   // the last segment's pieces were not read: S is its starting state
+        *reinterpret_cast<float4 *>(p.Sinit + ((size_t)head * p.nseg + p.nseg - 1) * E + e) = S;
     if (blockIdx.x == 0) {
         // key rows are 128 bf16 = 16 x 16 bytes: thread (r, c) copies chunk c of rows r, r + 16, ..
         const int c = threadIdx.x & 15, r = threadIdx.x >> 4;
