@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from delta_rule_linear_falcon_b200 import inputs as I
-from test_gpu_parity import F, TOL_BF16, check, dev, run_gpu, run_oracle  # noqa: F401
+from test_gpu_parity import F, TOL_BF16, check, dev, host, run_gpu, run_oracle  # noqa: F401
 
 pytestmark = pytest.mark.gpu
 SS = 0x100
@@ -76,3 +76,26 @@ def test_split_rejects_small_workspace(F):
     o = torch.empty_like(v)
     args = F.make_args(q, k, v, a, e, rule=2, eps=s.eps, o=o)
     assert F.lib().falcon_fwd_chunk(ctypes.byref(args), None, 0, None) == F.FALCON_ERR_WORKSPACE
+
+
+def test_split_on_a_side_stream_with_binding_workspace(F):
+    """The caller's current stream is the default one and the work goes to a side stream: the
+    binding allocates the workspace on the current stream and records the side stream on it,
+    so blocks of the same size allocated and filled on the current stream right after the call
+    cannot take the workspace while the split still runs."""
+    s = I.make_seq(2, 1, 2, 1024, 128, 128, seed=750, io_dtype="bf16", normalise_qk=False,
+                   alpha_mu=6.0, with_state=True, with_kprev=True)
+    need = _ws_bytes(F, 2, 1, 2, 1024)
+    assert need > 0
+    q, k, v = (dev(x, torch.bfloat16) for x in (s.q, s.k, s.v))
+    a, e = dev(s.alpha, torch.float32), dev(s.eta, torch.float32)
+    S0, kp = dev(s.S0, torch.float32), dev(s.k_prev, torch.bfloat16)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    o, S, kl = F.falcon_fwd_chunk(q, k, v, a, e, rule=2, eps=s.eps, S0=S0, k_prev=kp, stream=side)
+    junk = [torch.empty(need, dtype=torch.uint8, device="cuda").fill_(0xFF) for _ in range(8)]
+    side.synchronize()
+    torch.cuda.synchronize()
+    del junk
+    assert F.falcon_check_device_errors() == F.FALCON_OK
+    check(s, (host(o), host(S), host(kl)), run_oracle(s), TOL_BF16)
