@@ -139,7 +139,9 @@ FALCON_API size_t falcon_workspace_size(const falcon_args_t *args);
  * state, whatever io_dtype is; use falcon_fwd_recurrent for fp32-accurate work.
  *
  * Sequence split (inner-product write, window 1, dk = dv = 128, bf16, chunk 64,
- * T a multiple of 64, fewer heads than SMs): the additive write has a scalar
+ * T a multiple of 64, and room for nseg >= 2 segments of at least 8 blocks each
+ * with B*H*nseg <= the SM count; the largest such nseg dividing T/64 is taken):
+ * the additive write has a scalar
  * state transition, so each head is cut into nseg segments of whole blocks;
  * one parallel pass forms every piece's state increment
  * sum_t 2^(G_end - G_t) beta_t y_t x_t^T and its decay, a scan gives the state
