@@ -475,18 +475,53 @@ def cpu_oracle_sample(heads: int, T: int = 4096, threads=None):
     return heads * T / 16.0 / dt, dt, min(cores, heads)
 
 
-def cpu_baseline(min_seconds: float = 10.0, heads: int = 64):
-    """The oracle as it stands on the host cores: repeated passes over `heads` of the 128
-    heads of the B8 H16 T4096 d128 workload until at least `min_seconds` of work."""
-    total_t, total_tok, passes = 0.0, 0.0, 0
+def host_cpu():
+    """(logical cores, CPU model name) of this host."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count() or 1, model
+
+
+def oracle_heads(cores: int) -> int:
+    """Heads per oracle pass: at least one per core (OpenMP spreads heads over threads), a
+    multiple of the core count, at most the 128 heads of the workload."""
+    return max(1, min(128, cores * max(1, 16 // cores)))
+
+
+def _oracle_rate(heads: int, threads: int, min_seconds: float):
+    total_t, total_tok, passes, used = 0.0, 0.0, 0, 1
     while total_t < min_seconds:
-        tps, dt, used = cpu_oracle_sample(heads)
+        tps, dt, used = cpu_oracle_sample(heads, threads=threads)
         total_t += dt
         total_tok += tps * dt
         passes += 1
-    return {"value": round(total_tok / total_t, 1), "unit": "tokens/s", "cores": used, "kind": "oracle",
-            "sample": f"{passes} passes x {heads} of 128 heads x 4096 tokens of the B8 H16 T4096 d128 "
-                      f"workload, fp64 recurrent oracle, OpenMP over heads ({total_t:.1f} s)"}
+    return total_tok / total_t, total_t, passes, used
+
+
+def cpu_baseline(min_seconds: float = 10.0):
+    """The oracle as it stands on the host cores, on 1 core and on all cores: repeated passes
+    over a subset of the 128 heads of the B8 H16 T4096 d128 workload (at least one head per
+    thread) until at least `min_seconds` of work each."""
+    nproc, model = host_cpu()
+    heads = oracle_heads(nproc)
+    v_all, t_all, p_all, used = _oracle_rate(heads, nproc, min_seconds)
+    v_one, t_one, p_one, _ = _oracle_rate(1, 1, min_seconds / 2)
+    return {"value": round(v_all, 1), "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "nproc": nproc, "cpu_model": model,
+            "one_core": {"value": round(v_one, 1), "unit": "tokens/s", "cores": 1,
+                         "sample": f"{p_one} passes x 1 head x 4096 tokens ({t_one:.1f} s)"},
+            "all_cores": {"value": round(v_all, 1), "unit": "tokens/s", "cores": used,
+                          "sample": f"{p_all} passes x {heads} heads x 4096 tokens ({t_all:.1f} s)"},
+            "sample": f"{p_all} passes x {heads} of 128 heads x 4096 tokens of the B8 H16 T4096 d128 "
+                      f"workload, fp64 recurrent oracle, OpenMP over heads on {used} threads "
+                      f"({t_all:.1f} s); tokens are (b, t) positions of 16 heads each"}
 
 
 # ----------------------------------------------------------------------------- main
@@ -494,8 +529,8 @@ def cpu_baseline(min_seconds: float = 10.0, heads: int = 64):
 def run_reference(args):
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
-    heads = 4
-    cores = os.cpu_count() or 1
+    cores, model = host_cpu()
+    heads = oracle_heads(cores)
     vals = []
     for _ in range(args.warmup):
         cpu_oracle_sample(heads, threads=cores)
@@ -506,13 +541,13 @@ def run_reference(args):
     ms = statistics.median(v[1] for v in vals) * 1e3
     used = vals[0][2]
     sample = (f"{heads} of 128 heads x 4096 tokens of the B8 H16 T4096 d128 workload per step, "
-              f"fp64 recurrent oracle, OpenMP over heads")
+              f"fp64 recurrent oracle, OpenMP over heads on {used} of {cores} cores ({model})")
     line = {"impl": "reference", "metric": METRIC, "value": round(tps, 1), "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": base_config(args),
             "cpu_baseline": {"value": round(tps, 1), "unit": "tokens/s", "cores": used, "kind": "oracle",
-                             "sample": sample},
+                             "nproc": cores, "cpu_model": model, "sample": sample},
             "e2e": {"value": round(tps, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

@@ -81,6 +81,101 @@ def test_falcon1_hand_expanded_first_three_steps():
     np.testing.assert_allclose(o[0, 0], np.stack([o1, o2, o3]), rtol=1e-13, atol=1e-15)
 
 
+@pytest.mark.parametrize("name", ["falcon3", "falcon3a"])
+@pytest.mark.parametrize("form", ["recurrent", "masked", "chunk2", "chunk4", "chunk6"])
+def test_falcon3_window_slides_worked_by_hand(name, form):
+    """Falcon-3 / 3A with w = 2 over four tokens, every step worked by hand in exact rationals
+    (derivation in the fixture): the window fills, then slides and drops a pair. Each prefix of
+    the sequence gives the state after that step, so every step's output and state are pinned.
+    The chunk forms hold floor(chunk / w) tokens per block (1, 2 and 3)."""
+    from fractions import Fraction as Fr
+    g = json.load(open(os.path.join(HERE, "golden", "hand_worked_falcon3_w2_T4.json")))
+    inp, exp = g["inputs"], g["expected"][name]
+    val = lambda a: np.vectorize(lambda x: float(Fr(x)))(np.asarray(a, dtype=object)).astype(np.float64)
+    o_exp, S_exp = val(exp["o"]), val(exp["S_after"])
+    arr = lambda key: np.asarray(inp[key], dtype=np.float64)[None, None]
+    for T in range(1, 5):
+        q, k, v = arr("q")[:, :, :T], arr("k")[:, :, :T], arr("v")[:, :, :T]
+        a, e = arr("alpha")[:, :, :T], arr("eta")[:, :, :T]
+        if form == "recurrent":
+            o, S, kl = oracle.recurrent(exp["rule"], q, k, v, a, e, inp["eps"], inp["window"])
+        elif form == "masked":
+            o, S, kl = oracle.masked(exp["rule"], q, k, v, a, e, inp["eps"], inp["window"])
+        else:
+            o, S, kl = oracle.chunk(exp["rule"], q, k, v, a, e, inp["eps"], inp["window"],
+                                    chunk=int(form[5:]))
+        np.testing.assert_allclose(o[0, 0], o_exp[:T], rtol=0, atol=1e-14)
+        np.testing.assert_allclose(S[0, 0], S_exp[T - 1], rtol=0, atol=1e-14)
+    np.testing.assert_array_equal(kl[0, 0], g["expected"]["k_last"])
+
+
+def _unrolled_falcon1(k, v, q, alpha, eta, eps, S0, k_prev):
+    """Falcon-1 written out without its recurrence, in exact rationals: with
+    M_s = alpha_s (I - beta_s x_s x_s^T) (the state transition of step s, acting on the right),
+        S_t = S_0 M_1 ... M_t + sum_{j<=t} beta_j y_j x_j^T M_{j+1} ... M_t,   o_t = S_t q_t,
+    x_1 = k_prev (or 0), x_j = k_{j-1}, y_j = v_j, beta_j = eta_j / (||x_j||^2 + eps) (0 when that
+    denominator is 0). Returns the list of o_t and the final S as Fraction matrices."""
+    from fractions import Fraction as Fr
+    T, dk, dv = len(k), len(k[0]), len(v[0])
+    eye = [[Fr(int(i == j)) for j in range(dk)] for i in range(dk)]
+    mul = lambda A, B: [[sum(A[i][m] * B[m][j] for m in range(len(B))) for j in range(len(B[0]))]
+                        for i in range(len(A))]
+    x = [k_prev if k_prev is not None else [Fr(0)] * dk] + [k[j - 1] for j in range(1, T)]
+    beta = []
+    for j in range(T):
+        den = sum(c * c for c in x[j]) + eps
+        beta.append(eta[j] / den if den != 0 else Fr(0))
+    M = [[[alpha[s] * (eye[i][c] - beta[s] * x[s][i] * x[s][c]) for c in range(dk)] for i in range(dk)]
+         for s in range(T)]
+    outs, S = [], None
+    for t in range(T):
+        prod = eye
+        for s in range(t, -1, -1):          # prod = M_s ... M_t, built from the right
+            prod = mul(M[s], prod)
+        S = mul(S0, prod)                    # S_0 M_1 ... M_t
+        for j in range(t + 1):
+            tail = eye
+            for s in range(t, j, -1):
+                tail = mul(M[s], tail)       # M_{j+1} ... M_t
+            write = [[beta[j] * v[j][i] * x[j][c] for c in range(dk)] for i in range(dv)]
+            W = mul(write, tail)
+            S = [[S[i][c] + W[i][c] for c in range(dk)] for i in range(dv)]
+        outs.append([sum(S[i][c] * q[t][c] for c in range(dk)) for i in range(dv)])
+    return outs, S
+
+
+@pytest.mark.parametrize("with_cache", [False, True])
+def test_falcon1_unrolled_closed_form_T8(with_cache):
+    """Falcon-1 over eight tokens against the recurrence unrolled by hand into a sum of products
+    of step transitions, evaluated in exact rational arithmetic (d_k = 3, d_v = 2, small integer
+    keys, rational gates, an initial state and optionally a cached key). Every o_1..o_8 and the
+    final state are pinned."""
+    from fractions import Fraction as Fr
+    k = [[1, 0, 2], [0, 1, -1], [2, 1, 0], [1, -1, 1], [0, 2, 1], [1, 1, 1], [-1, 0, 2], [3, 1, -2]]
+    v = [[1, 2], [0, -1], [2, 1], [-1, 3], [1, 0], [2, -2], [0, 1], [1, 1]]
+    q = [[1, 1, 0], [0, 1, 2], [1, 0, -1], [2, 1, 1], [0, 0, 1], [1, -1, 0], [1, 2, 1], [0, 1, 1]]
+    alpha = [Fr(9, 10), Fr(4, 5), Fr(1), Fr(1, 2), Fr(7, 8), Fr(3, 4), Fr(1), Fr(5, 8)]
+    eta = [Fr(1), Fr(1, 2), Fr(3, 4), Fr(1), Fr(1, 4), Fr(2, 3), Fr(1), Fr(1, 2)]
+    eps = Fr(1, 10)
+    S0 = [[Fr(1, 2), Fr(0), Fr(-1, 4)], [Fr(0), Fr(1, 3), Fr(1)]]
+    k_prev = [Fr(1), Fr(-2), Fr(0)] if with_cache else None
+    F = lambda rows: [[Fr(c) for c in r] for r in rows]
+    outs, S = _unrolled_falcon1(F(k), F(v), F(q), alpha, eta, eps, S0, k_prev)
+    f64 = lambda a: np.asarray([[float(c) for c in r] for r in a], dtype=np.float64)[None, None]
+    o, So, kl = oracle.recurrent(R1, f64(q), f64(k), f64(v), np.asarray([[list(map(float, alpha))]]),
+                                 np.asarray([[list(map(float, eta))]]), float(eps), 1, S0=f64(S0),
+                                 k_prev=(np.asarray([[[float(c) for c in k_prev]]]) if with_cache else None))
+    np.testing.assert_allclose(o[0, 0], f64(outs)[0, 0], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(So[0, 0], f64(S)[0, 0], rtol=1e-13, atol=1e-14)
+    for form, kw in (("chunk", {"chunk": 3}), ("masked", {})):
+        fn = oracle.chunk if form == "chunk" else oracle.masked
+        o2, S2, _ = fn(R1, f64(q), f64(k), f64(v), np.asarray([[list(map(float, alpha))]]),
+                       np.asarray([[list(map(float, eta))]]), float(eps), 1, S0=f64(S0),
+                       k_prev=(np.asarray([[[float(c) for c in k_prev]]]) if with_cache else None), **kw)
+        np.testing.assert_allclose(o2[0, 0], f64(outs)[0, 0], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(S2[0, 0], f64(S)[0, 0], rtol=1e-12, atol=1e-13)
+
+
 def test_falcon1a_is_gated_linear_attention():
     """Falcon-1A closed form (S_0 = 0): S_T = sum_t (prod_{s>t} alpha_s) beta_t y_t x_t^T and
     o_t = sum_{j<=t} (prod_{j<s<=t} alpha_s) beta_j (x_j.q_t) y_j."""
