@@ -399,7 +399,7 @@ def bench_more_chunk(args, D: Dist):
 
     dev = torch.device("cuda", D.local)
     stream = torch.cuda.current_stream(dev)
-    hbm, _, _ = peaks()
+    hbm, tf, _ = peaks()
     out = {}
 
     def timed(s, rule, label):
@@ -427,10 +427,16 @@ def bench_more_chunk(args, D: Dist):
         assert F.falcon_check_device_errors(stream) == F.FALCON_OK
         ms = t0.elapsed_time(t1) / n
         nbytes = chunk_algorithmic_bytes(B, H, T, dk, dv)
+        flops = chunk_algorithmic_flops(B, H, T, dk, dv, window=s.window)
         gbs = nbytes / (ms * 1e-3) / 1e9
+        # roofline time = max(bytes / HBM peak, recurrent-form FLOPs / bf16 peak)
+        t_roof = max(nbytes / (hbm * 1e9), flops / (tf * 1e12))
         out[label] = {"workload": label, "ms_per_launch": round(ms, 4),
                       "tokens_per_s": round(B * T / (ms * 1e-3), 1), "gbs_algorithmic": round(gbs, 1),
-                      "roofline_frac": round(gbs / hbm, 4), "launches": n,
+                      "tflops_algorithmic": round(flops / (ms * 1e-3) / 1e12, 2),
+                      "t_roofline_us": round(t_roof * 1e6, 2),
+                      "roofline_bound": "hbm" if nbytes / (hbm * 1e9) >= flops / (tf * 1e12) else "tensor",
+                      "roofline_frac": round(t_roof / (ms * 1e-3), 4), "launches": n,
                       # the sequence split of the inner-product rule: state pass, scan, chunk kernel
                       "kernels_per_call": 3 if need else 1, "workspace_bytes": need}
         del q, k, v, a, e, o, S, kl, ws

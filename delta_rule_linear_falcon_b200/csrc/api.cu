@@ -19,6 +19,14 @@ __device__ int g_dev_error = 0;
 
 namespace {
 
+// One-shot stall armed by falcon_debug_stall_next_call for the next chunk call of this thread.
+struct DebugStall {
+    bool armed = false;
+    int block = -1;
+    long long budget = kDefaultWaitBudget;
+};
+thread_local DebugStall g_stall;
+
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 int *g_err_ptr[kMaxDevices] = {};
@@ -106,6 +114,8 @@ ChunkParams chunk_params(const falcon_args_t *a) {
     p.q = a->q; p.k = a->k; p.v = a->v; p.k_prev = a->k_prev;
     p.alpha = a->alpha; p.eta = a->eta; p.S0 = a->S0; p.eps = a->eps;
     p.o = a->o; p.k_last = a->k_last; p.S_out = a->S_out;
+    p.wait_budget = kDefaultWaitBudget;
+    p.dbg_stall_block = -1;
     return p;
 }
 
@@ -134,6 +144,7 @@ extern "C" {
 
 size_t falcon_workspace_size(const falcon_args_t *a) {
     if (!a || check_seq_args(a) != FALCON_OK) return 0;
+    if (a->io_dtype != FALCON_BF16) return 0;
     if (!dim_supported_chunk(a->dk) || !dim_supported_chunk(a->dv)) return 0;
     if (a->chunk != 16 && a->chunk != 32 && a->chunk != 64) return 0;
     if ((long long)a->B * a->H == 0) return 0;
@@ -147,6 +158,9 @@ falcon_status_t falcon_fwd_chunk(const falcon_args_t *a, void *workspace, size_t
                                  falcon_stream_t stream) {
     falcon_status_t st = check_seq_args(a);
     if (st != FALCON_OK) return st;
+    // The chunk form's products take bf16 tensor-core operands; fp32 inputs would be held to a
+    // bf16 error bound, so fp32-accurate work goes through falcon_fwd_recurrent instead.
+    if (a->io_dtype != FALCON_BF16) return FALCON_ERR_UNSUPPORTED;
     if (!dim_supported_chunk(a->dk) || !dim_supported_chunk(a->dv)) return FALCON_ERR_UNSUPPORTED;
     if (a->chunk != 16 && a->chunk != 32 && a->chunk != 64) return FALCON_ERR_UNSUPPORTED;
     const int w = is_windowed(a->rule) ? a->window : 1;
@@ -154,6 +168,11 @@ falcon_status_t falcon_fwd_chunk(const falcon_args_t *a, void *workspace, size_t
     if ((long long)a->B * a->H == 0) return FALCON_OK;
 
     ChunkParams p = chunk_params(a);
+    if (g_stall.armed) {
+        p.dbg_stall_block = g_stall.block;
+        p.wait_budget = g_stall.budget;
+        g_stall = DebugStall{};
+    }
     int sms = 0;
     if (!device_info(&p.err, &sms)) return FALCON_ERR_CUDA;
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -245,6 +264,15 @@ falcon_status_t falcon_check_device_errors(falcon_stream_t stream) {
     }
     if (h == kDevErrTimeout) return FALCON_ERR_TIMEOUT;
     if (h != 0) return FALCON_ERR_INVALID_ARG;
+    return FALCON_OK;
+}
+
+falcon_status_t falcon_debug_stall_next_call(int block, long long wait_budget_cycles) {
+    if (block < 0 || wait_budget_cycles < 10000 || wait_budget_cycles > kDefaultWaitBudget)
+        return FALCON_ERR_INVALID_ARG;
+    g_stall.armed = true;
+    g_stall.block = block;
+    g_stall.budget = wait_budget_cycles;
     return FALCON_OK;
 }
 

@@ -496,11 +496,9 @@ cudaError_t launch_chunk_t(const ChunkParams &p, cudaStream_t s) {
 
 template <int DK, int DVS>
 cudaError_t launch_chunk_dk_dvs(const ChunkParams &p, cudaStream_t s) {
-    if (p.io_bf16)
-        return p.regression ? launch_chunk_t<DK, DVS, true, __nv_bfloat16>(p, s)
-                            : launch_chunk_t<DK, DVS, false, __nv_bfloat16>(p, s);
-    return p.regression ? launch_chunk_t<DK, DVS, true, float>(p, s)
-                        : launch_chunk_t<DK, DVS, false, float>(p, s);
+    if (!p.io_bf16) return cudaErrorInvalidValue;  // the entry point admits bf16 I/O only
+    return p.regression ? launch_chunk_t<DK, DVS, true, __nv_bfloat16>(p, s)
+                        : launch_chunk_t<DK, DVS, false, __nv_bfloat16>(p, s);
 }
 
 // Per-DK dispatchers, one translation unit each (compile in parallel).

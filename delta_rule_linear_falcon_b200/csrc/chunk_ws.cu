@@ -1,6 +1,8 @@
 // chunk_ws.cu -- warp-specialised chunk-parallel forward pass on tcgen05 for
-// d_k = d_v = 128, bf16 I/O, one pair per step (Falcon-1, Falcon-1A), 64-token
-// blocks. The block algebra is the chunk-parallel form with positive-decay
+// d_k = d_v = 128, bf16 I/O, blocks of 64 pseudo-value rows: 64 tokens of one pair
+// each (Falcon-1, Falcon-1A), or 64 / w tokens of w pairs each (Falcon-3, Falcon-3A
+// with a window of w = 2 or 4; see "Windowed rules" below). The block algebra is the
+// chunk-parallel form with positive-decay
 // renormalisation of "Fast Weight Attention for Continual Learning" (authors'
 // abstract), written out in chunk_kernel.cuh, regrouped so that the state
 // recurrence crosses only two tensor-core steps per block. With g the block-local
@@ -33,11 +35,24 @@
 // Every decay factor is 2^(g_i - g_j) with i >= j (never a quotient of
 // cumulative products). Every wait is bounded; a timeout is recorded in the
 // device error word and all roles unwind.
+//
+// Windowed rules (W = w pairs per step, TB = 64 / W tokens per block). Row r of a block
+// holds pair j = t0 + s - m of token s = r % TB, m = r / TB (m-major order), so X and Y
+// arrive as W boxes of TB consecutive key / value rows (key rows t0 - m - 1, value rows
+// t0 - m; rows before the sequence read as zero, and zero rows are no-ops). A row takes the
+// decay and the step size of its token: beta_s = eta_s / (sum_m ||x_(m,s)||^2 + eps), the sum
+// over the W diagonal entries of G of that token. L couples a row only to rows of strictly
+// earlier tokens (all residuals of one step are taken at the same decayed state), so it is
+// strictly lower triangular in token-major order u = s * W + m: the local warps permute G
+// into that order for the solve and permute T back to m-major order for the MMAs. P~ masks
+// by token (a query reads the pairs of its own and earlier tokens); only the TB query rows
+// are loaded and only TB outputs are written per block.
 #include <cuda.h>
 
 #include "common.cuh"
 #include "launch.h"
 #include "tc_common.cuh"
+#include "tmap.h"
 
 namespace falcon {
 
@@ -45,7 +60,7 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kBlk = 64;
-constexpr long long kWaitBudget = 1ll << 31;  // SM clocks, about 1 s
+constexpr long long kDrainBudget = kDefaultWaitBudget;  // waits for own loads / MMAs in flight at exit
 constexpr int LDF = 68;                       // fp32 solve buffers: 16-byte rows, conflict-free A fragments
 constexpr int kChainWarps = 8;
 
@@ -60,8 +75,8 @@ constexpr uint32_t oPB = oTP + 8192;               // rows 0-63 P~ (A of (B')), 
 constexpr uint32_t oA = oPB + 16384;               // A^T bf16, 128 rows (d) x 64 (i) (B of (f'))
 constexpr uint32_t oL = oA + 16384;                // L / W fp32 64 x LDF
 constexpr uint32_t oTf = oL + 64 * LDF * 4;        // T fp32 64 x LDF
-constexpr uint32_t oScal = oTf + 64 * LDF * 4;     // 4 slots x {beta, 2^g, 2^(g_last-g), g}[64], 4 x cf[64], g_last[4], misc
-constexpr uint32_t oBar = oScal + 4096 + 1024 + 256;
+constexpr uint32_t oScal = oTf + 64 * LDF * 4;     // 4 slots x {beta, 2^g, 2^(g_last-g), g}[64], 4 x cf[64], g_last[4], misc, norms[64]
+constexpr uint32_t oBar = oScal + 4096 + 1024 + 512;
 constexpr uint32_t kSmem = oBar + 512 + 1024;
 static_assert(kSmem <= 232448, "shared memory");
 
@@ -76,11 +91,13 @@ constexpr uint32_t kIdN64 = tc::idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t kIdN128 = tc::idesc_bf16(128, 128, 0, 0);
 constexpr uint32_t kIdAT = tc::idesc_bf16(128, 64, 1, 1);   // X^T (MN-major A) x T_f (MN-major B)
 constexpr uint32_t kIdBP = tc::idesc_bf16(128, 64, 0, 1);   // P~ (K-major A) x T' (MN-major B)
+constexpr uint32_t kIdVP = tc::idesc_bf16(128, 64, 1, 0);   // (diag(beta) Y)^T (MN-major A) x P~ (K-major B)
+constexpr uint32_t kIdVX = tc::idesc_bf16(128, 128, 1, 1);  // (diag(w) Y)^T (MN-major A) x X (MN-major B)
 
 // barrier indices (arrival count 1 unless noted)
 enum {
     B_FULLXQ = 0,      // [3] TMA [X;Q] landed -> helpers
-    B_XQFREE = 3,      // [3] (b) done -> producer
+    B_XQFREE = 3,      // [3] (a), (A) done (feed warp) and (b) done (chain MMA warp): 2 arrivals -> producer
     B_FULLV = 6,       // [2] TMA V landed -> chain
     B_VFREE = 8,       // [2] chain read V (8 warps) -> producer
     B_XQRDY = 10,      // [3] helpers prepared the block -> MMA (a)
@@ -88,17 +105,17 @@ enum {
     B_GPFREE = 14,     // G read (local warps 4, 5) and P read (helpers): 3 arrivals -> MMA (a) of the next block
     B_SCAL = 15,       // [4] decay scalars of slot c % 4 ready -> local, chain
     B_SCALFREE = 19,   // [4] chain done with scalar slot, outputs stored (8 warps) -> helpers
-    B_UNUSED23 = 23,   // [3]
+    B_EDONE = 23,      // (e') done (it still reads R'^T from TMEM) -> chain (before S overwrites it), outputs
     B_PRDY = 26,       // P~ ready -> MMA (B')
     B_TRDY = 27,       // T_f, T' (and the step sizes) ready -> MMA (A), (B')
     B_ABDONE = 28,     // (A), (B') done -> chain, local (T tiles free), helpers (P~ tile free)
     B_EARDY = 29,      // A^T, B' in shared memory (8 warps) -> MMA (e'), (f')
     B_BDONE = 30,      // (b) done -> chain
     B_RT = 31,         // R'^T in TMEM (8 warps) -> MMA (e'), (f')
-    B_EFDONE = 32,     // (e'), (f') done -> chain
-    B_UNUSED = 33,
+    B_EFDONE = 32,     // (f') done: dS in TMEM -> chain
+    B_FINAL0 = 33,     // drain of the feed warp's MMAs at exit
     B_SRDY = 34,       // S bf16 in TMEM, dS read, O of the previous block read (8 warps) -> MMA (b)
-    B_FINAL = 35,      // MMA drain at exit
+    B_FINAL = 35,      // drain of the chain MMA warp's MMAs at exit
     B_COUNT = 36
 };
 
@@ -268,7 +285,7 @@ __device__ __forceinline__ void solve_local(float *sL, float *sTf, int lt, int l
 
 }  // namespace
 
-template <bool REG>
+template <bool REG, int W>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                 const __grid_constant__ CUtensorMap tmV, ChunkParams p) {
@@ -282,7 +299,8 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     float *sScal = reinterpret_cast<float *>(sm + oScal);
     float *sCF = sScal + 1024;                             // 4 x cf[64]
     float *sGL = sScal + 1280;                             // g_last per slot
-    float *sMisc = sScal + 1284;                           // helper scan carry
+    float *sMisc = sScal + 1284;                           // helper scan carry; token decays (windowed rules)
+    float *sNrm = sScal + 1344;                            // squared key norms of the rows (windowed rules)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + oBar);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + B_COUNT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
@@ -290,14 +308,20 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x;
     const int T = p.T;
-    const int nblk = (T + kBlk - 1) / kBlk;
+    constexpr int TB = kBlk / W;          // tokens per block
+    static_assert(W == 1 || W == 2 || W == 4, "window");
+    const int nblk = (T + TB - 1) / TB;
     constexpr int D = 128;
 
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i) {
-            const bool chain_arrivals = (i >= B_VFREE && i < B_VFREE + 2) || (i >= B_SCALFREE && i < B_SCALFREE + 4) ||
-                                        i == B_EARDY || i == B_RT || i == B_SRDY;
-            tc::mbar_init(&bars[i], chain_arrivals ? kChainWarps : (i == B_GPFREE ? 3 : 1));
+            // V slots: freed by the chain warps' reads (regression), or by the MMAs that read the scaled
+            // values (inner product)
+            const bool chain_arrivals = (REG && i >= B_VFREE && i < B_VFREE + 2) ||
+                                        (i >= B_SCALFREE && i < B_SCALFREE + 4) || i == B_EARDY || i == B_RT ||
+                                        i == B_SRDY;
+            const bool two = i >= B_XQFREE && i < B_XQFREE + 3;
+            tc::mbar_init(&bars[i], chain_arrivals ? kChainWarps : (i == B_GPFREE ? 3 : (two ? 2 : 1)));
         }
         *abort_flag = 0;
         tc::mbar_fence_init();
@@ -307,6 +331,14 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         tc::tmem_relinquish();
     }
     for (int idx = tid; idx < 64 * LDF; idx += kThreads) sTf[idx] = 0.f;
+    if constexpr (W > 1) {  // query rows TB..63 of every [X;Q] slot: never loaded, kept zero
+        for (int idx = tid; idx < 3 * 2 * (64 - TB) * 8; idx += kThreads) {
+            const int ch = idx & 7, row = TB + (idx >> 3) % (64 - TB), at = (idx >> 3) / (64 - TB);
+            *reinterpret_cast<uint4 *>(sm + oXQ + (at >> 1) * kXQ + (at & 1) * 16384 + 8192 + row * 128 + ch * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
+        tc::fence_proxy_async();
+    }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -315,7 +347,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     // Leader-polled bounded wait; the outcome is made uniform across the role by its named barrier.
     auto role_wait = [&](uint64_t *bar, uint32_t parity, bool leader, int bar_id, int nthr) -> bool {
         bool failed = false;
-        if (leader && !tc::mbar_wait(bar, parity, abort_flag, kWaitBudget)) {
+        if (leader && !tc::mbar_wait(bar, parity, abort_flag, p.wait_budget)) {
             *abort_flag = 1;
             failed = true;
         }
@@ -324,7 +356,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     // Lane-0-polled bounded wait, uniform across the warp.
     auto warp_wait = [&](uint64_t *bar, uint32_t parity) -> bool {
         int ok = 1;
-        if (lane == 0 && !tc::mbar_wait(bar, parity, abort_flag, kWaitBudget)) {
+        if (lane == 0 && !tc::mbar_wait(bar, parity, abort_flag, p.wait_budget)) {
             *abort_flag = 1;
             ok = 0;
         }
@@ -337,112 +369,89 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         if (lane == 0) mbar_arrive(bar);
     };
 
+    // Shared-memory descriptors (built once; a K step only moves the 14-bit start-address field,
+    // address >> 4, which stays below 2^14 for every operand here, so a plain add is exact). Slot u
+    // of the [X;Q] ring is kXQ bytes further: its descriptors are the slot-0 ones plus u * kXQ / 16,
+    // kept arithmetic so that they stay warp-uniform.
+    const uint64_t dXQ0 = tc::sdesc(tc::smem_u32(sm + oXQ), 16, 1024);      // [X;Q] K-major: (a), (b)
+    auto slot_off = [](int u) -> uint64_t { return (uint64_t)(u * (kXQ >> 4)); };
+    auto kmaj = [](int ks) -> uint64_t { return (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4); };
+    // Whole-warp bounded wait of an issuing warp: every lane polls, the outcome is warp-uniform.
+    auto wait_all = [&](int b, uint32_t parity) -> bool {
+        const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars[b], parity, abort_flag, p.wait_budget));
+        if (!ok) *abort_flag = 1;
+        return ok;
+    };
+
     if (warp == 0) {
-        // ================================================================ TMA producer
-        if (lane == 0) {
-            // [X;Q] of block j, then V of block j-1: the slot of XQ_j frees at (b) of block j-3, which
-            // precedes the chain's read of V_{j-3} that frees the slot of V_{j-1}, so the blocking waits
-            // below never hold back a load that could already start.
-            int kx = 0, kv = 0;
-            const int kshift = p.same_step ? 0 : 1;   // prefix-aligned key rows of block j start at t0 - 1
-            for (int j = 0; j <= nblk && !*abort_flag; ++j) {
-                if (j < nblk) {
-                    if (j >= 3 && !tc::mbar_wait(&bars[B_XQFREE + j % 3], ((j / 3) - 1) & 1, abort_flag, kWaitBudget)) {
-                        *abort_flag = 1;
-                        break;
-                    }
+        // ================================================================ feed: TMA loads and the
+        // state-independent MMAs (a), (A), (B'), issued by the whole warp (one elected lane issues).
+        // Iteration j loads [X;Q] of block j and V of block j-1, then issues (a) of block j-1 and
+        // (A), (B') of block j-2, each as soon as its inputs are ready. None of these waits on a later
+        // iteration's work, and the chain only needs what earlier iterations issued, so the order
+        // cannot deadlock; it keeps the Gram products and the solve of later blocks off the chain.
+        const uint64_t dXmn0 = tc::sdesc(tc::smem_u32(sm + oXQ), 16384, 1024);  // X as an MN-major A
+        const uint64_t dTF = tc::sdesc(tc::smem_u32(sTF), 8192, 1024);          // MN-major B, one N atom
+        const uint64_t dTP = tc::sdesc(tc::smem_u32(sTP), 8192, 1024);
+        const uint64_t dPB = tc::sdesc(tc::smem_u32(sPB), 16, 1024);            // [P~; B'] K-major
+        const int kshift = p.same_step ? 0 : 1;   // prefix-aligned key rows of block j start at t0 - 1
+        int kx = 0, kv = 0;
+        bool ok = true;
+        for (int j = 0; j <= nblk + 1 && ok; ++j) {
+            if (j < nblk) {
+                if (j == p.dbg_stall_block) break;  // test hook: this block is never loaded
+                if (j >= 3 && !(ok = wait_all(B_XQFREE + j % 3, ((j / 3) - 1) & 1))) break;
+                if (lane == 0) {
                     uint8_t *dst = sm + oXQ + (j % 3) * kXQ;
                     uint64_t *fb = &bars[B_FULLXQ + j % 3];
-                    const int t0 = j * kBlk;
-                    tc::mbar_arrive_expect_tx(fb, kXQ);
-                    tc::tma_load_3d(dst + 0, &tmK, 0, t0 - kshift, bh, fb);
-                    tc::tma_load_3d(dst + 16384, &tmK, 64, t0 - kshift, bh, fb);
+                    const int t0 = j * TB;
+                    tc::mbar_arrive_expect_tx(fb, 16384 + TB * 256);
+#pragma unroll
+                    for (int m = 0; m < W; ++m) {  // rows m*TB.. hold the pairs t0 - m ..: key rows t0 - m - kshift
+                        tc::tma_load_3d(dst + m * TB * 128, &tmK, 0, t0 - m - kshift, bh, fb);
+                        tc::tma_load_3d(dst + 16384 + m * TB * 128, &tmK, 64, t0 - m - kshift, bh, fb);
+                    }
                     tc::tma_load_3d(dst + 8192, &tmQ, 0, t0, bh, fb);
                     tc::tma_load_3d(dst + 16384 + 8192, &tmQ, 64, t0, bh, fb);
-                    kx = j + 1;
                 }
-                const int jv = j - 1;
-                if (jv >= 0) {
-                    if (jv >= 2 &&
-                        !tc::mbar_wait(&bars[B_VFREE + (jv & 1)], ((jv >> 1) - 1) & 1, abort_flag, kWaitBudget)) {
-                        *abort_flag = 1;
-                        break;
-                    }
+                __syncwarp();
+                kx = j + 1;
+            }
+            const int jv = j - 1;
+            if (jv >= 0 && jv < nblk) {
+                if (jv >= 2 && !(ok = wait_all(B_VFREE + (jv & 1), ((jv >> 1) - 1) & 1))) break;
+                if (lane == 0) {
                     uint8_t *dst = sm + oV + (jv & 1) * kVst;
                     uint64_t *fb = &bars[B_FULLV + (jv & 1)];
-                    const int t0 = jv * kBlk;
+                    const int t0 = jv * TB;
                     tc::mbar_arrive_expect_tx(fb, kVst);
-                    tc::tma_load_3d(dst + 0, &tmV, 0, t0, bh, fb);
-                    tc::tma_load_3d(dst + 8192, &tmV, 64, t0, bh, fb);
-                    kv = jv + 1;
+#pragma unroll
+                    for (int m = 0; m < W; ++m) {  // value rows t0 - m ..
+                        tc::tma_load_3d(dst + m * TB * 128, &tmV, 0, t0 - m, bh, fb);
+                        tc::tma_load_3d(dst + 8192 + m * TB * 128, &tmV, 64, t0 - m, bh, fb);
+                    }
                 }
+                __syncwarp();
+                kv = jv + 1;
             }
-            // drain: every armed load must have landed before the CTA can exit
-            const volatile int no_abort = 0;
-            for (int c = kx - 3 < 0 ? 0 : kx - 3; c < kx; ++c)
-                tc::mbar_wait(&bars[B_FULLXQ + c % 3], (c / 3) & 1, &no_abort, kWaitBudget);
-            for (int c = kv - 2 < 0 ? 0 : kv - 2; c < kv; ++c)
-                tc::mbar_wait(&bars[B_FULLV + (c & 1)], (c >> 1) & 1, &no_abort, kWaitBudget);
-        }
-    } else if (warp == 1) {
-        // ================================================================ MMA issuer (whole warp, elected lane issues)
-        {
-            // Descriptors are built once; a K step only moves the 14-bit start-address field
-            // (address >> 4), which stays below 2^14 for every operand here, so a plain add is exact.
-            // Slot u of the [X;Q] ring is kXQ bytes further: its descriptors are the slot-0 ones plus
-            // u * kXQ / 16 (kept arithmetic so that they stay warp-uniform, in uniform registers).
-            const uint64_t dXQ0 = tc::sdesc(tc::smem_u32(sm + oXQ), 16, 1024);      // [X;Q] K-major: (a), (b)
-            const uint64_t dXmn0 = tc::sdesc(tc::smem_u32(sm + oXQ), 16384, 1024);  // X as an MN-major A
-            auto slot_off = [](int u) -> uint64_t { return (uint64_t)(u * (kXQ >> 4)); };
-            const uint64_t dTF = tc::sdesc(tc::smem_u32(sTF), 8192, 1024);   // MN-major B, one N atom
-            const uint64_t dTP = tc::sdesc(tc::smem_u32(sTP), 8192, 1024);
-            const uint64_t dPB = tc::sdesc(tc::smem_u32(sPB), 16, 1024);     // [P~; B'] K-major
-            const uint64_t dBp = tc::sdesc(tc::smem_u32(sPB + 8192), 16, 1024);
-            const uint64_t dAt = tc::sdesc(tc::smem_u32(sA), 16, 1024);
-            auto kmaj = [](int ks) -> uint64_t { return (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4); };
-            // every lane waits; the outcome is made uniform across the warp
-            auto wait = [&](int b, uint32_t parity) -> bool {
-                const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars[b], parity, abort_flag, kWaitBudget));
-                if (!ok) *abort_flag = 1;
-                return ok;
-            };
-            auto test = [&](int b, uint32_t parity) -> bool {
-                return __all_sync(0xffffffffu, tc::mbar_test(&bars[b], parity));
-            };
-            // (a) of block na as soon as its slot is prepared and the GP columns are free;
-            // returns -1 on abort, else whether it issued.
-            int na = 0;
-            auto try_a = [&](bool block) -> int {
-                if (na >= nblk) return 0;
-                const uint32_t pr = (na / 3) & 1, pg = (na - 1) & 1;
-                if (block) {
-                    if (!wait(B_XQRDY + na % 3, pr) || (na > 0 && !wait(B_GPFREE, pg))) return -1;
-                } else if (!test(B_XQRDY + na % 3, pr) || (na > 0 && !test(B_GPFREE, pg))) {
-                    return 0;
-                }
+            const int ja = j - 1;   // (a) [X;Q] X^T -> G, P once the helpers prepared the block and the
+            if (ja >= 0 && ja < nblk) {  // G/P columns were read for the block before
+                if (!(ok = wait_all(B_XQRDY + ja % 3, (ja / 3) & 1) && (ja == 0 || wait_all(B_GPFREE, (ja - 1) & 1))))
+                    break;
                 tc::fence_after_sync();
-                const uint64_t d = dXQ0 + slot_off(na % 3);
+                const uint64_t d = dXQ0 + slot_off(ja % 3);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) tc::mma_bf16_elect(tbase + cGP, d + kmaj(ks), d + kmaj(ks), kIdN64, ks > 0);
                 tc::mma_commit_elect(&bars[B_ADONE]);
-                ++na;
-                return 1;
-            };
-            // (A) A^T = X^T T_f and (B') B' = P~ T' of block j into the AB columns (free once the chain
-            // copied A^T, B' of block j-1 to shared memory). Returns -1 on abort, else whether it issued.
-            auto issue_AB = [&](int j, bool block) -> int {
-                if (block) {
-                    while (na <= j)
-                        if (try_a(true) < 0) return -1;
-                    if (!(wait(B_TRDY, j & 1) && wait(B_PRDY, j & 1) && (j < 1 || wait(B_EARDY, (j - 1) & 1))))
-                        return -1;
-                } else {
-                    if (na <= j && try_a(false) < 0) return -1;
-                    if (na <= j || !test(B_TRDY, j & 1) || !test(B_PRDY, j & 1) || (j >= 1 && !test(B_EARDY, (j - 1) & 1)))
-                        return 0;
-                }
+                if (!REG) tc::mma_commit_elect(&bars[B_XQFREE + ja % 3]);   // one of the slot's two arrivals
+            }
+            const int jb = j - 2;   // (A) A^T = X^T T_f and (B') B' = P~ T' into the AB columns, free once
+            if (REG && jb >= 0 && jb < nblk) {  // the chain copied A^T, B' of the block before
+                if (!(ok = wait_all(B_TRDY, jb & 1) && wait_all(B_PRDY, jb & 1) &&
+                           (jb == 0 || wait_all(B_EARDY, (jb - 1) & 1))))
+                    break;
                 tc::fence_after_sync();
-                const int u = j % 3;
+                const int u = jb % 3;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     tc::mma_bf16_elect(tbase + cAB, dXmn0 + slot_off(u) + (uint64_t)(ks * 128), dTF + (uint64_t)(ks * 128), kIdAT, ks > 0);
@@ -450,43 +459,99 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 for (int ks = 0; ks < 4; ++ks)
                     tc::mma_bf16_elect(tbase + cAB + 64, dPB + (uint64_t)(ks * 2), dTP + (uint64_t)(ks * 128), kIdBP, ks > 0);
                 tc::mma_commit_elect(&bars[B_ABDONE]);
-                return 1;
-            };
-            bool ok = nblk == 0 || issue_AB(0, true) > 0;
+                tc::mma_commit_elect(&bars[B_XQFREE + u]);   // (a), (A) of the slot are done (one of two arrivals)
+            }
+        }
+        if (!ok) *abort_flag = 1;
+        // drain: every MMA this warp issued has completed, every armed load has landed
+        tc::mma_commit_elect(&bars[B_FINAL0]);
+        const volatile int no_abort = 0;
+        tc::mbar_wait(&bars[B_FINAL0], 0, &no_abort, kDrainBudget);
+        if (lane == 0) {
+            for (int c = kx - 3 < 0 ? 0 : kx - 3; c < kx; ++c)
+                tc::mbar_wait(&bars[B_FULLXQ + c % 3], (c / 3) & 1, &no_abort, kDrainBudget);
+            for (int c = kv - 2 < 0 ? 0 : kv - 2; c < kv; ++c)
+                tc::mbar_wait(&bars[B_FULLV + (c & 1)], (c >> 1) & 1, &no_abort, kDrainBudget);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ================================================================ chain MMAs (whole warp, elected lane issues)
+        const uint64_t dBp = tc::sdesc(tc::smem_u32(sPB + 8192), 16, 1024);
+        const uint64_t dAt = tc::sdesc(tc::smem_u32(sA), 16, 1024);
+        bool ok = true;
+        if (!REG) {
+            // Inner-product rules: no solve, so the block's writes do not depend on the state.
+            //   O   = diag(2^g) Q S^T + P~ diag(beta) Y     (E = (diag(beta) Y)^T P~^T, transposed)
+            //   dS  = (diag(w) Y)^T X,   w = beta 2^(g_last - g),   S <- 2^g_last S + dS
+            // The scaled value tiles (diag(beta) Y in place in the V slot, diag(w) Y in the T tile region)
+            // are the MN-major A operands, read straight from shared memory; X is the MN-major B of dS and
+            // P~ the K-major B of E. Slots alternate: dS of block c lands in the slot that held the outputs
+            // of block c-1, [E | S Q^T] of block c in the one dS of block c-1 was read from.
+            const uint64_t dPB = tc::sdesc(tc::smem_u32(sPB), 16, 1024);              // P~ rows 0-63, K-major B
+            const uint64_t dVw = tc::sdesc(tc::smem_u32(sTF), 8192, 1024);            // diag(w) Y, MN-major A
+            const uint64_t dXmnB = tc::sdesc(tc::smem_u32(sm + oXQ), 16384, 1024);   // X as an MN-major B
             for (int c = 0; c < nblk && ok; ++c) {
                 const int s = c & 1, u = c % 3;
-                // (b) [S X^T | S Q^T] -> slot s, S from TMEM
-                if (!(ok = wait(B_SRDY, c & 1))) break;
+                const uint64_t dVb = tc::sdesc(tc::smem_u32(sm + oV + s * kVst), 8192, 1024);  // diag(beta) Y
+                if (!(ok = wait_all(B_SRDY, c & 1) && wait_all(B_TRDY, c & 1) && wait_all(B_PRDY, c & 1))) break;
                 tc::fence_after_sync();
+                const uint64_t dQ = dXQ0 + slot_off(u) + (8192 >> 4);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)   // S Q^T -> columns 64-127 of slot s
+                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s + 64, tbase + cSR + 8 * ks, dQ + kmaj(ks), kIdN64, ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)   // E -> columns 0-63 of slot s
+                    tc::mma_bf16_elect(tbase + cSXO + 128 * s, dVb + (uint64_t)(ks * 128), dPB + (uint64_t)(ks * 2), kIdVP, ks > 0);
+                tc::mma_commit_elect(&bars[B_BDONE]);              // outputs of block c ready
+                // dS into slot s^1 once the outputs of block c-1 have been read out of it
+                if (c >= 1 && !(ok = wait_all(B_EARDY, (c - 1) & 1))) break;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16_elect(tbase + cSXO + 128 * (s ^ 1), dVw + (uint64_t)(ks * 128),
+                                       dXmnB + slot_off(u) + (uint64_t)(ks * 128), kIdVX, ks > 0);
+                tc::mma_commit_elect(&bars[B_EFDONE]);
+                tc::mma_commit_elect(&bars[B_XQFREE + u]);   // the other arrival of the slot
+                tc::mma_commit_elect(&bars[B_VFREE + s]);    // diag(beta) Y read: the V slot may refill
+                tc::mma_commit_elect(&bars[B_ABDONE]);       // diag(w) Y read: the tile may be rewritten
+            }
+        }
+        for (int c = 0; c < nblk && ok && REG; ++c) {
+            const int s = c & 1, u = c % 3;
+            // (b) S X^T (regression only) then S Q^T -> slot s, S (bf16) from TMEM; the chain starts
+            // forming R'^T as soon as the first half is done
+            if (!(ok = wait_all(B_SRDY, c & 1))) break;
+            tc::fence_after_sync();
+            const uint64_t dX = dXQ0 + slot_off(u), dQ = dX + (8192 >> 4);   // X rows 0-63, Q rows 64-127
+            if (REG) {
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dXQ0 + slot_off(u) + kmaj(ks), kIdN128, ks > 0);
+                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dX + kmaj(ks), kIdN64, ks > 0);
                 tc::mma_commit_elect(&bars[B_BDONE]);
-                tc::mma_commit_elect(&bars[B_XQFREE + u]);
-                // state-independent work of the next block runs while the chain forms R'^T, if it is ready
-                int ab = 0;
-                if (c + 1 < nblk && (ab = issue_AB(c + 1, false)) < 0) { ok = false; break; }
-                if ((ok = try_a(false) >= 0) == false) break;
-                // (e') R'^T B'^T over S X^T in slot s and (f') dS = R'^T A into slot s^1, R'^T from TMEM
-                if (!(ok = wait(B_RT, c & 1) && wait(B_EARDY, c & 1))) break;
-                tc::fence_after_sync();
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dBp + (uint64_t)(ks * 2), kIdN64, ks > 0);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * (s ^ 1), tbase + cSR + 8 * ks, dAt + (uint64_t)(ks * 2), kIdN128, ks > 0);
-                tc::mma_commit_elect(&bars[B_EFDONE]);
-                if (c + 1 < nblk && ab == 0 && issue_AB(c + 1, true) < 0) { ok = false; break; }
-                if ((ok = try_a(false) >= 0) == false) break;
             }
-            if (!ok) *abort_flag = 1;
-            // drain every MMA issued so far
-            tc::mma_commit_elect(&bars[B_FINAL]);
-            const volatile int no_abort = 0;
-            tc::mbar_wait(&bars[B_FINAL], 0, &no_abort, kWaitBudget);
-            __syncwarp();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s + 64, tbase + cSR + 8 * ks, dQ + kmaj(ks), kIdN64, ks > 0);
+            tc::mma_commit_elect(&bars[B_XQFREE + u]);   // (b) of the slot is done (the other arrival)
+            // (f') dS = R'^T A into slot s^1 first (the state update waits for it), then (e') R'^T B'^T
+            // over S X^T in slot s (the outputs wait for it); R'^T from TMEM
+            if (!(ok = wait_all(B_RT, c & 1) && wait_all(B_EARDY, c & 1))) break;
+            tc::fence_after_sync();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                tc::mma_bf16_ts_elect(tbase + cSXO + 128 * (s ^ 1), tbase + cSR + 8 * ks, dAt + (uint64_t)(ks * 2), kIdN128, ks > 0);
+            tc::mma_commit_elect(&bars[B_EFDONE]);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dBp + (uint64_t)(ks * 2), kIdN64, ks > 0);
+            tc::mma_commit_elect(&bars[B_EDONE]);
         }
+        if (!ok) *abort_flag = 1;
+        // drain every MMA issued by this warp
+        tc::mma_commit_elect(&bars[B_FINAL]);
+        const volatile int no_abort = 0;
+        tc::mbar_wait(&bars[B_FINAL], 0, &no_abort, kDrainBudget);
+        __syncwarp();
     } else if (warp < 4) {
         // ================================================================ helpers (64 threads)
         const int ht = tid - 64;           // row / token index 0..63
@@ -494,19 +559,21 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         const float *alpha_h = p.alpha + (size_t)bh * T;
         float ga = 1.f;                    // decay gate of the block prep() handles next
         auto load_gates = [&](int c) {
-            const int t = c * kBlk + ht;
-            ga = t < T ? alpha_h[t] : 1.f;
+            const int t = c * TB + ht;
+            ga = (ht < TB && t < T) ? alpha_h[t] : 1.f;
         };
         auto prep = [&](int c) -> bool {   // block c: x_1 patch, decay tables
             const int u3 = c % 3, u4 = c % 4;
             uint8_t *xq = sm + oXQ + u3 * kXQ;
             if (c >= 4 && !role_wait(&bars[B_SCALFREE + u4], ((c >> 2) - 1) & 1, leader, 1, 64)) return false;
             if (!role_wait(&bars[B_FULLXQ + u3], (c / 3) & 1, leader, 1, 64)) return false;
-            const int t0 = c * kBlk, nval = min(kBlk, T - t0);
-            if (c == 0 && p.k_prev && !p.same_step && ht < 16) {
+            const int t0 = c * TB, nval = min(TB, T - t0);
+            if (c == 0 && p.k_prev && !p.same_step && ht < 16 * W) {
+                // pair 0 = (k_prev, v_0) sits in row m * TB + m of block 0 for every m < W
+                const int m = ht >> 4, chunk = ht & 15;
                 const uint4 v = *reinterpret_cast<const uint4 *>(
-                    reinterpret_cast<const __nv_bfloat16 *>(p.k_prev) + (size_t)bh * D + ht * 8);
-                *reinterpret_cast<uint4 *>(xq + (ht >> 3) * 16384 + (ht & 7) * 16) = v;
+                    reinterpret_cast<const __nv_bfloat16 *>(p.k_prev) + (size_t)bh * D + chunk * 8);
+                *reinterpret_cast<uint4 *>(xq + (chunk >> 3) * 16384 + tc::sw128_chunk(m * TB + m, chunk & 7)) = v;
                 tc::fence_proxy_async();
             }
             const bool valid = ht < nval;
@@ -516,16 +583,28 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 const float y = __shfl_up_sync(0xffffffffu, la, off);
                 if (lane >= off) la += y;
             }
-            if (ht == 31) sMisc[0] = la;
-            named_bar(1, 64);
-            if (ht >= 32) la += sMisc[0];
             float *sc = sScal + u4 * 256;
-            sc[64 + ht] = exp2f(la);
-            sc[192 + ht] = la;
-            named_bar(1, 64);
-            const float gl = sc[192 + nval - 1];
-            sc[128 + ht] = exp2f(gl - la);
-            sCF[64 * u4 + ht] = exp2f(sc[192 + (ht | 15)] - la);
+            float gl;
+            if (W == 1) {
+                if (ht == 31) sMisc[0] = la;
+                named_bar(1, 64);
+                if (ht >= 32) la += sMisc[0];
+                sc[64 + ht] = exp2f(la);
+                sc[192 + ht] = la;
+                named_bar(1, 64);
+                gl = sc[192 + nval - 1];
+                sc[128 + ht] = exp2f(gl - la);
+                sCF[64 * u4 + ht] = exp2f(sc[192 + (ht | 15)] - la);
+            } else {
+                // TB <= 32 tokens: one warp's scan gives the token decays; every row takes its token's
+                if (ht < TB) sMisc[1 + ht] = la;
+                named_bar(1, 64);
+                const float g = sMisc[1 + ht % TB];
+                gl = sMisc[nval];
+                sc[64 + ht] = exp2f(g);
+                sc[192 + ht] = g;
+                sc[128 + ht] = exp2f(gl - g);
+            }
             if (leader) sGL[u4] = gl;
             named_bar(1, 64);
             if (leader) {
@@ -564,7 +643,18 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             if (leader) mbar_arrive(&bars[B_GPFREE]);
             // P~ = Gamma o P (inclusive), packed to bf16 while (B') of the previous block still reads the tile
             uint32_t pk[32];
-            {
+            if (W > 1) {
+                // query token i = ht < TB reads the rows of tokens s' <= i (inclusive); rows of one token
+                // share its decay 2^(g_i - g_s'); rows i >= TB of P are zero (their query rows are)
+                const float *g2 = sc + 192;
+                const int i = ht;
+                const float gri = g2[i];
+                float fac[TB];
+#pragma unroll
+                for (int sp = 0; sp < TB; ++sp) fac[sp] = sp <= i ? exp2f(fminf(gri - g2[sp], 0.f)) : 0.f;
+#pragma unroll
+                for (int j = 0; j < 64; j += 2) pk[j >> 1] = pack_bf16x2(fac[j % TB] * v[j], fac[(j + 1) % TB] * v[j + 1]);
+            } else {
                 const float *g2 = sc + 192, *cf = sCF + 64 * (c % 4);
                 const int i = ht, rb = i >> 4;
                 const float gri = g2[i];
@@ -593,7 +683,9 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                     }
                 }
             }
-            if (c >= 1 && !(ok = role_wait(&bars[B_ABDONE], (c - 1) & 1, leader, 1, 64))) break;
+            // the tile is free once the products of block c-1 that read P~ are done: (B') for the
+            // regression rules, E for the inner-product rules
+            if (c >= 1 && !(ok = role_wait(&bars[REG ? B_ABDONE : B_BDONE], (c - 1) & 1, leader, 1, 64))) break;
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch)
                 *reinterpret_cast<uint4 *>(sPB + tc::sw128_chunk(ht, ch)) =
@@ -611,7 +703,8 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         const bool leader = lt == 0;
         const uint32_t tl = tbase + ((uint32_t)(32 * lw) << 16);
         const float *eta_h = p.eta + (size_t)bh * T;
-        float ge = (lw < 2 && r < T) ? eta_h[r] : 0.f;   // step-size gate of row r, one block ahead
+        const int rs = r % TB;             // token of row r (rows of one token share its step size)
+        float ge = (lw < 2 && rs < T) ? eta_h[rs] : 0.f;  // step-size gate of row r's token, one block ahead
         for (int c = 0; c < nblk; ++c) {
             const int u4 = c % 4;
             if (!role_wait(&bars[B_ADONE], c & 1, leader, 2, 128)) break;
@@ -637,12 +730,39 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 float nrm = 0.f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) nrm += (j == lane) ? (lw == 0 ? v[j] : v[32 + j]) : 0.f;
-                const bool valid = c * kBlk + r < T;
+                if (W > 1) {   // the token's window: rows m * TB + rs, m < W
+                    sNrm[r] = nrm;
+                    named_bar(3, 64);
+                    nrm = 0.f;
+#pragma unroll
+                    for (int m = 0; m < W; ++m) nrm += sNrm[m * TB + rs];
+                }
+                const bool valid = c * TB + rs < T;
                 const float be = valid ? step_size(ge, nrm, p.eps) : 0.f;
                 sc[r] = be;
-                const int tn = (c + 1) * kBlk + r;
+                const int tn = (c + 1) * TB + rs;
                 ge = tn < T ? eta_h[tn] : 0.f;
-              if (REG) {
+              if (REG && W > 1) {
+                // row u = rs * W + m of L in token-major order couples to the rows of earlier tokens
+                // s' < rs only: L[u][s' W + m'] = beta 2^(g_rs - g_s') G[r][m' TB + s'], zero otherwise
+                // (the rows of one token form the identity block of I + L)
+                const float *g2 = sc + 192;
+                const float gri = g2[r];
+                float gd[TB];
+#pragma unroll
+                for (int sp = 0; sp < TB; ++sp) gd[sp] = sp < rs ? be * exp2f(fminf(gri - g2[sp], 0.f)) : 0.f;
+                float *Lr = sL + (rs * W + r / TB) * LDF;
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    float w4[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int up = 4 * q + k, sp = up / W, mp = up % W;
+                        w4[k] = gd[sp] * v[mp * TB + sp];
+                    }
+                    *reinterpret_cast<float4 *>(Lr + 4 * q) = make_float4(w4[0], w4[1], w4[2], w4[3]);
+                }
+              } else if (REG) {
                 // Decay factors 2^(g_r - g_j), j < r: below the 16x16 diagonal blocks they factor
                 // through the last index of column block jb, 2^(g_r - g_{16jb+15}) * cf[j] with
                 // cf[j] = 2^(g_{16jb+15} - g_j) (a helper table), both in (0, 1]; inside the
@@ -678,7 +798,39 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
               }
             }
             named_bar(2, 128);
-            if (REG) solve_local(sL, sTf, lt, lw, lane);
+            if (!REG) {
+                // The scaled value tiles of block c (inner-product rules): diag(beta) Y in place in its V
+                // slot and diag(w) Y, w = beta 2^(g_last - g), into the T tile region, once V has landed and
+                // the products of block c-1 no longer read the region. Thread (row rr, atom at) scales the
+                // 64 values of its row in that atom; scaling does not care where the swizzle put them.
+                if (!role_wait(&bars[B_FULLV + (c & 1)], (c >> 1) & 1, leader, 2, 128)) break;
+                if (c >= 1 && !role_wait(&bars[B_ABDONE], (c - 1) & 1, leader, 2, 128)) break;
+                const int rr = lt >> 1, at = lt & 1;
+                const float bb = sc[rr], ww = bb * sc[128 + rr];
+                const uint32_t line = at * 8192 + (rr >> 3) * 1024 + (rr & 7) * 128;
+                uint8_t *vrow = sm + oV + (c & 1) * kVst + line;
+                uint8_t *wrow = sTF + line;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const int cc = ch ^ (rr & 7);      // rows of a group start on different banks
+                    const uint4 x = *reinterpret_cast<const uint4 *>(vrow + 16 * cc);
+                    const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+                    uint32_t bs[4], ws[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xs[k]));
+                        bs[k] = pack_bf16x2(bb * f.x, bb * f.y);
+                        ws[k] = pack_bf16x2(ww * f.x, ww * f.y);
+                    }
+                    *reinterpret_cast<uint4 *>(vrow + 16 * cc) = make_uint4(bs[0], bs[1], bs[2], bs[3]);
+                    *reinterpret_cast<uint4 *>(wrow + 16 * cc) = make_uint4(ws[0], ws[1], ws[2], ws[3]);
+                }
+                tc::fence_proxy_async();
+                named_bar(2, 128);
+                if (leader) mbar_arrive(&bars[B_TRDY]);
+                continue;
+            }
+            solve_local(sL, sTf, lt, lw, lane);
             // T_f = diag(2^(g_last - g)) T diag(beta), T' = T diag(beta) once (A), (B') of c-1 are done
             if (c >= 1 && !role_wait(&bars[B_ABDONE], (c - 1) & 1, leader, 2, 128)) break;
             {
@@ -688,7 +840,13 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 for (int cc = 0; cc < 4; ++cc) {
                     const int j0 = 8 * (ch0 + cc);
                     float t8[8], f8[8];
-                    if (REG) {
+                    if (REG && W > 1) {
+                        // T is in token-major order: row (rr % TB) W + rr / TB; the eight m-major columns
+                        // j0.. share m' = j0 / TB and take tokens j0 % TB + k, i.e. a stride of W
+                        const float *Trow = sTf + ((rr % TB) * W + rr / TB) * LDF + (j0 % TB) * W + j0 / TB;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) t8[k] = Trow[k * W];
+                    } else if (REG) {
                         const float4 x0 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + j0);
                         const float4 x1 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + j0 + 4);
                         t8[0] = x0.x; t8[1] = x0.y; t8[2] = x0.z; t8[3] = x0.w;
@@ -735,22 +893,25 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         // memory: lane pairs (2k, 2k+1) hold neighbouring value rows; the even lane stores the pair for
         // even tokens, the odd lane for odd tokens.
         auto store_out = [&](int c) {
-            const int t0 = c * kBlk, nval = min(kBlk, T - t0);
+            const int t0 = c * TB, nval = min(TB, T - t0);
             const bool odd = lane & 1;
             __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.o) + ((size_t)bh * T + t0) * D + (row & ~1);
 #pragma unroll 1
-            for (int h = 0; h < 4; ++h) {          // 8 tokens at a time
-                const int i0 = 32 * hf + 8 * h;
+            for (int h = 0; h < 2; ++h) {          // 16 tokens at a time
+                const int i0 = 32 * hf + 16 * h;
+                if (i0 >= TB) break;               // a block has TB query tokens
                 const float *d2 = sScal + (c % 4) * 256 + 64 + i0;   // 2^g of the tokens
                 // the scales first, so that their shared-memory latency overlaps the TMEM loads
-                const float4 da = *reinterpret_cast<const float4 *>(d2);
-                const float4 db = *reinterpret_cast<const float4 *>(d2 + 4);
-                float v[8], w[8];
-                tc::tmem_ld8(tl + cSXO + 128 * (c & 1) + 64 + i0, v);
-                tc::tmem_ld8(tl + cSXO + 128 * (c & 1) + i0, w);
-                const float dg[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+                float dg[16];
 #pragma unroll
-                for (int j = 0; j < 8; j += 2) {
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 d4 = *reinterpret_cast<const float4 *>(d2 + 4 * q4);
+                    dg[4 * q4] = d4.x; dg[4 * q4 + 1] = d4.y; dg[4 * q4 + 2] = d4.z; dg[4 * q4 + 3] = d4.w;
+                }
+                float v[16], w[16];
+                tc::tmem_ld16x2(tl + cSXO + 128 * (c & 1) + 64 + i0, tl + cSXO + 128 * (c & 1) + i0, v, w);
+#pragma unroll
+                for (int j = 0; j < 16; j += 2) {
                     const float v0 = dg[j] * v[j] + w[j], v1 = dg[j + 1] * v[j + 1] + w[j + 1];
                     const float mine = odd ? v1 : v0;
                     const float give = odd ? v0 : v1;
@@ -772,7 +933,34 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             warp_arrive(&bars[B_SRDY]);
         }
         bool ok = true;
-        for (int c = 0; c < nblk; ++c) {
+        for (int c = 0; c < nblk && !REG; ++c) {
+            // Inner-product rules: the state update is the whole chain; the outputs of the block are
+            // read out of the other slot afterwards, which frees it for dS of the next block.
+            const int s = c & 1, u4 = c % 4;
+            if (!(ok = warp_wait(&bars[B_EFDONE], c & 1))) break;
+            tc::fence_after_sync();
+            {
+                const float dl = exp2f(sGL[u4]);
+                const uint32_t cds = cSXO + 128 * (s ^ 1) + 64 * hf;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float v[32];
+                    tc::tmem_ld32(tl + cds + 32 * hh, v);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) S[32 * hh + j] = dl * S[32 * hh + j] + v[j];
+                }
+            }
+            store_S();
+            warp_arrive(&bars[B_SRDY]);
+            store_out(c);
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars[B_EARDY]);            // slot s read: dS of block c+1 may take it
+                mbar_arrive(&bars[B_SCALFREE + u4]);
+            }
+        }
+        for (int c = 0; c < nblk && REG; ++c) {
             const int s = c & 1, u4 = c % 4;
             // A^T (rows d, columns i) and B' (rows i < 64) from TMEM to their shared-memory tiles
             if (!(ok = warp_wait(&bars[B_ABDONE], c & 1))) break;
@@ -799,7 +987,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 if (lane == 0) mbar_arrive(&bars[B_SCALFREE + (c - 1) % 4]);
             }
             // R'^T = Y^T - SX diag(2^g) (regression) or Y^T (inner product), bf16 into TMEM
-            if (!(ok = warp_wait(&bars[B_BDONE], c & 1) && warp_wait(&bars[B_SCAL + u4], (c >> 2) & 1) &&
+            if (!(ok = (!REG || warp_wait(&bars[B_BDONE], c & 1)) && warp_wait(&bars[B_SCAL + u4], (c >> 2) & 1) &&
                        warp_wait(&bars[B_FULLV + s], (c >> 1) & 1)))
                 break;
             tc::fence_after_sync();
@@ -808,24 +996,25 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 const uint8_t *sV = sm + oV + s * kVst + vcol;
                 uint32_t pk[16];
 #pragma unroll
-                for (int hh = 0; hh < 4; ++hh) {           // 8 tokens at a time
-                    const int i0 = 32 * hf + 8 * hh;
-                    float x[8], dg[8];
+                for (int hh = 0; hh < 2; ++hh) {           // 16 rows at a time
+                    const int i0 = 32 * hf + 16 * hh;
+                    float x[16], dg[16];
                     if (REG) {                             // scales first: their latency overlaps the TMEM load
-                        const float4 da = *reinterpret_cast<const float4 *>(sc + 64 + i0);
-                        const float4 db = *reinterpret_cast<const float4 *>(sc + 64 + i0 + 4);
-                        dg[0] = da.x; dg[1] = da.y; dg[2] = da.z; dg[3] = da.w;
-                        dg[4] = db.x; dg[5] = db.y; dg[6] = db.z; dg[7] = db.w;
-                        tc::tmem_ld8(tl + cSXO + 128 * s + i0, x);
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const float4 d4 = *reinterpret_cast<const float4 *>(sc + 64 + i0 + 4 * q4);
+                            dg[4 * q4] = d4.x; dg[4 * q4 + 1] = d4.y; dg[4 * q4 + 2] = d4.z; dg[4 * q4 + 3] = d4.w;
+                        }
+                        tc::tmem_ld16(tl + cSXO + 128 * s + i0, x);
                     }
 #pragma unroll
-                    for (int j = 0; j < 8; j += 2) {
+                    for (int j = 0; j < 16; j += 2) {
                         const int i = i0 + j;              // token row of V: swizzle depends on i & 7 only
                         const float y0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sV + voff[i & 7] + (i >> 3) * 1024));
                         const float y1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sV + voff[(i + 1) & 7] + ((i + 1) >> 3) * 1024));
                         const float r0 = REG ? y0 - dg[j] * x[j] : y0;
                         const float r1 = REG ? y1 - dg[j + 1] * x[j + 1] : y1;
-                        pk[4 * hh + (j >> 1)] = pack_bf16x2(r0, r1);
+                        pk[8 * hh + (j >> 1)] = pack_bf16x2(r0, r1);
                     }
                 }
                 tc::tmem_st16(tl + cSR + 16 * hf, pk);
@@ -846,10 +1035,12 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                     for (int j = 0; j < 32; ++j) S[32 * hh + j] = dl * S[32 * hh + j] + v[j];
                 }
             }
+            // (e') still reads R'^T from the columns the bf16 state takes
+            if (!(ok = warp_wait(&bars[B_EDONE], c & 1))) break;
             store_S();
             warp_arrive(&bars[B_SRDY]);
         }
-        if (ok && nblk > 0 && !*abort_flag) {
+        if (REG && ok && nblk > 0 && !*abort_flag) {
             store_out(nblk - 1);
             tc::fence_before_sync();
         }
@@ -878,53 +1069,38 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 
 // ------------------------------------------------------------------ host side
 
+bool chunk_ws_supported(const ChunkParams &p) {
+    const bool w_ok = p.window == 1 || p.window == 2 || p.window == 4;
+    return p.dk == 128 && p.dv == 128 && p.io_bf16 && w_ok && p.tok_per_blk * p.window == kBlk && p.T >= 1 &&
+           encode_tiled_fn() != nullptr;
+}
+
 namespace {
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
-                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                  CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn_ws() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-// (128 columns, T rows, B*H heads) bf16 view with 64 x 64 boxes, 128-byte swizzle.
-bool map_tile(CUtensorMap *m, const void *base, int T, long long BH) {
-    cuuint64_t dims[3] = {128, (cuuint64_t)T, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {128 * 2, (cuuint64_t)T * 128 * 2};
-    cuuint32_t box[3] = {64, 64, 1};
-    cuuint32_t es[3] = {1, 1, 1};
-    return encode_fn_ws()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-}  // namespace
-
-bool chunk_ws_supported(const ChunkParams &p) {
-    return p.dk == 128 && p.dv == 128 && p.io_bf16 && p.window == 1 && p.tok_per_blk == kBlk && p.T >= 1 &&
-           encode_fn_ws() != nullptr;
-}
-
-cudaError_t launch_chunk_ws(const ChunkParams &p, cudaStream_t s) {
+template <int W>
+cudaError_t launch_chunk_ws_w(const ChunkParams &p, cudaStream_t s) {
     const long long BH = (long long)p.B * p.H;
+    constexpr int TB = kBlk / W;  // boxes of TB rows: the W shifted copies of a block's keys and values
     CUtensorMap mK, mQ, mV;
-    if (!map_tile(&mK, p.k, p.T, BH) || !map_tile(&mQ, p.q, p.T, BH) || !map_tile(&mV, p.v, p.T, BH))
+    if (!map_head_rows(&mK, p.k, p.T, BH, TB) || !map_head_rows(&mQ, p.q, p.T, BH, TB) ||
+        !map_head_rows(&mV, p.v, p.T, BH, TB))
         return cudaErrorInvalidValue;
-    auto kern = p.regression ? chunk_ws_kernel<true> : chunk_ws_kernel<false>;
+    auto kern = p.regression ? chunk_ws_kernel<true, W> : chunk_ws_kernel<false, W>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)BH, kThreads, kSmem, s>>>(mK, mQ, mV, p);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_ws(const ChunkParams &p, cudaStream_t s) {
+    switch (p.window) {
+        case 1: return launch_chunk_ws_w<1>(p, s);
+        case 2: return launch_chunk_ws_w<2>(p, s);
+        case 4: return launch_chunk_ws_w<4>(p, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace falcon

@@ -44,7 +44,15 @@ struct ChunkParams {
     void *o, *k_last;
     float *S_out;
     int *err;
+    // Bounded waits of the tensor-core kernels give up after wait_budget SM clocks. A test hook
+    // (falcon_debug_stall_next_call) shortens it and makes the TMA producers stop loading at
+    // block dbg_stall_block, so that the timeout path runs without faulting or hanging the GPU;
+    // -1 = no stall.
+    long long wait_budget;
+    int dbg_stall_block;
 };
+
+constexpr long long kDefaultWaitBudget = 1ll << 31;  // SM clocks, about 1 s
 
 size_t recurrent_smem_bytes(int dk, int dv, int window);
 cudaError_t launch_recurrent(const RecParams &p, cudaStream_t s);

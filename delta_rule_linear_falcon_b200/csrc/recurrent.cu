@@ -3,9 +3,12 @@
 // Learning": authors' abstract; ai.info overview, Methodology in Plain English).
 //
 // One CTA per (b, h). Thread i owns row i of S in registers (d_k padded to
-// DKMAX); keys and values of the last w pairs live in a ring in shared memory.
-// The inputs of step t+1 are loaded into registers while step t computes, so
-// the per-step latency is two barriers and the row arithmetic.
+// DKMAX); keys and values of the last w pairs live in a ring of w + 1 slots in
+// shared memory, so a single barrier per step separates writing a slot from its
+// last read. The inputs of step t + A are loaded into registers while step t
+// computes (a register queue A = 3..8 steps deep), which keeps global-load latency off
+// the per-step path. The squared norm of each pair is reduced once, when the pair
+// is staged (one partial per warp), and the window sum reads those partials.
 // Per step t (0-based, pair j = t - m for window slot m):
 //   Sbar = alpha_t S
 //   beta = eta_t / (sum_m ||x_{t-m}||^2 + eps)
@@ -18,18 +21,40 @@
 namespace falcon {
 
 constexpr int kRecThreads = 128;
+constexpr int kRecWarps = kRecThreads / 32;
 constexpr int kRecMaxWindow = 64;
+// Steps of inputs in flight ahead of the one being computed: fewer for wide rows, whose
+// longer steps cover the load latency sooner and whose state row takes more registers.
+template <int DKMAX> __host__ __device__ constexpr int ahead() { return DKMAX >= 128 ? 3 : (DKMAX >= 64 ? 6 : 8); }
+
+// Dot product of a register row with a shared-memory vector, four independent partial sums.
+template <int DKMAX>
+__device__ __forceinline__ float row_dot(const float (&S)[DKMAX], const float *x) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+    for (int c = 0; c < DKMAX; c += 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(x + c);
+        a0 = fmaf(S[c], v.x, a0);
+        a1 = fmaf(S[c + 1], v.y, a1);
+        a2 = fmaf(S[c + 2], v.z, a2);
+        a3 = fmaf(S[c + 3], v.w, a3);
+    }
+    return (a0 + a1) + (a2 + a3);
+}
 
 template <typename IO, bool REGRESSION, int DKMAX>
 __global__ void __launch_bounds__(kRecThreads)
 recurrent_kernel(RecParams p) {
-    extern __shared__ float smem[];
-    const int dk = p.dk, dv = p.dv, W = p.window;
-    float *sX = smem;                   // W x DKMAX key ring (zero padded)
-    float *sY = sX + (size_t)W * DKMAX; // W x dv   value ring
-    float *sQ = sY + (size_t)W * dv;    // 2 x DKMAX queries (double buffered)
+    extern __shared__ __align__(16) float smem[];
+    const int dk = p.dk, dv = p.dv, W = p.window, RS = W + 1;
+    float *sX = smem;                        // RS x DKMAX key ring (zero padded)
+    float *sY = sX + (size_t)RS * DKMAX;     // RS x DVP value ring
+    const int DVP = (dv + 3) & ~3;
+    float *sQ = sY + (size_t)RS * DVP;       // 2 x DKMAX queries (double buffered)
+    float *sN = sQ + 2 * DKMAX;              // RS x kRecWarps partial squared norms of the pairs
+    constexpr int kAhead = ahead<DKMAX>();
 
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long bh = blockIdx.x;
     const int T = p.T;
     const IO *q = reinterpret_cast<const IO *>(p.q) + bh * (size_t)T * dk;
@@ -40,7 +65,7 @@ recurrent_kernel(RecParams p) {
     const float *eta = p.eta + bh * (size_t)T;
     IO *o = reinterpret_cast<IO *>(p.o) + bh * (size_t)T * dv;
 
-    for (int idx = tid; idx < W * (DKMAX + dv) + 2 * DKMAX; idx += kRecThreads) smem[idx] = 0.f;
+    for (int idx = tid; idx < RS * (DKMAX + DVP + kRecWarps) + 2 * DKMAX; idx += kRecThreads) smem[idx] = 0.f;
 
     const bool has_row = tid < dv;
     float S[DKMAX];
@@ -48,99 +73,102 @@ recurrent_kernel(RecParams p) {
     for (int c = 0; c < DKMAX; ++c)
         S[c] = (has_row && p.S0 && c < dk) ? p.S0[(bh * (size_t)dv + tid) * dk + c] : 0.f;
 
-    // registers holding the inputs of the step about to be staged
     auto load_x = [&](int t) -> float {   // key half of pair t, coordinate tid
         if (tid >= dk) return 0.f;
         if (p.same_step) return Io<IO>::ld(k, (size_t)t * dk + tid);
         if (t >= 1) return Io<IO>::ld(k, (size_t)(t - 1) * dk + tid);
         return kp ? Io<IO>::ld(kp, tid) : 0.f;
     };
-    float xr = 0.f, qr = 0.f, yr = 0.f, ar = 1.f, er = 0.f;
-    if (T > 0) {
-        xr = load_x(0);
-        qr = tid < dk ? Io<IO>::ld(q, tid) : 0.f;
-        yr = has_row ? Io<IO>::ld(v, tid) : 0.f;
-        ar = alpha[0];
-        er = eta[0];
+    // register queue: inputs of steps t .. t + kAhead - 1, slot t % kAhead
+    float xr[kAhead], qr[kAhead], yr[kAhead], ar[kAhead], er[kAhead];
+    auto fetch = [&](int t, float &x, float &qq, float &y, float &a, float &e) {
+        if (t < T) {
+            x = load_x(t);
+            qq = tid < dk ? Io<IO>::ld(q, (size_t)t * dk + tid) : 0.f;
+            y = has_row ? Io<IO>::ld(v, (size_t)t * dv + tid) : 0.f;
+            a = alpha[t];
+            e = eta[t];
+        }
+    };
+#pragma unroll
+    for (int i = 0; i < kAhead; ++i) {
+        xr[i] = 0.f; qr[i] = 0.f; yr[i] = 0.f; ar[i] = 1.f; er[i] = 0.f;
+        fetch(i, xr[i], qr[i], yr[i], ar[i], er[i]);
     }
     __syncthreads();
 
     int slot = 0;
-    for (int t = 0; t < T; ++t) {
-        // (A) stage pair t and q_t, then start loading step t+1
-        if (tid < dk) {
-            sX[slot * DKMAX + tid] = xr;
-            sQ[(t & 1) * DKMAX + tid] = qr;
-        }
-        if (has_row) sY[slot * dv + tid] = yr;
-        const float a = ar, e = er;
-        if (t + 1 < T) {
-            xr = load_x(t + 1);
-            qr = tid < dk ? Io<IO>::ld(q, (size_t)(t + 1) * dk + tid) : 0.f;
-            yr = has_row ? Io<IO>::ld(v, (size_t)(t + 1) * dv + tid) : 0.f;
-            ar = alpha[t + 1];
-            er = eta[t + 1];
-        }
-        __syncthreads();
-
-        // (B) window step size (every thread computes it from the ring)
-        const int nw = t + 1 < W ? t + 1 : W;
-        float ns = 0.f;
-        {
-            int sl = slot;
-            for (int m = 0; m < nw; ++m) {
-                const float *x = sX + sl * DKMAX;
-#pragma unroll 8
-                for (int c = 0; c < DKMAX; ++c) ns += x[c] * x[c];
-                sl = sl == 0 ? W - 1 : sl - 1;
+    for (int t0 = 0; t0 < T; t0 += kAhead) {
+#pragma unroll
+        for (int i = 0; i < kAhead; ++i) {
+            const int t = t0 + i;
+            if (t >= T) break;
+            // (A) stage pair t and q_t with the pair's squared-norm partial, refill the queue slot
+            {
+                float x2 = xr[i] * xr[i];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) x2 += __shfl_xor_sync(0xffffffffu, x2, off);
+                if (lane == 0) sN[slot * kRecWarps + warp] = x2;
             }
-        }
-        const float beta = step_size(e, ns, p.eps);
+            if (tid < dk) {
+                sX[slot * DKMAX + tid] = xr[i];
+                sQ[(t & 1) * DKMAX + tid] = qr[i];
+            }
+            if (has_row) sY[slot * DVP + tid] = yr[i];
+            const float a = ar[i], e = er[i];
+            fetch(t + kAhead, xr[i], qr[i], yr[i], ar[i], er[i]);
+            __syncthreads();
 
-        // (C) row update and the read after the write
-        if (has_row) {
-#pragma unroll
-            for (int c = 0; c < DKMAX; ++c) S[c] *= a;  // Sbar
-            if (W == 1) {
-                const float *x = sX;  // slot 0
-                float r = 0.f;
-#pragma unroll
-                for (int c = 0; c < DKMAX; ++c) r += S[c] * x[c];
-                const float coef = REGRESSION ? beta * (r - sY[tid]) : -beta * sY[tid];
-#pragma unroll
-                for (int c = 0; c < DKMAX; ++c) S[c] -= coef * x[c];
-            } else {
-                float coef[kRecMaxWindow];
+            // (B) window step size from the staged partial norms
+            const int nw = t + 1 < W ? t + 1 : W;
+            float ns = 0.f;
+            {
                 int sl = slot;
                 for (int m = 0; m < nw; ++m) {
-                    const float *x = sX + sl * DKMAX;
-                    if (REGRESSION) {
-                        float r = 0.f;
 #pragma unroll
-                        for (int c = 0; c < DKMAX; ++c) r += S[c] * x[c];
-                        coef[m] = beta * (r - sY[sl * dv + tid]);
-                    } else {
-                        coef[m] = -beta * sY[sl * dv + tid];
-                    }
-                    sl = sl == 0 ? W - 1 : sl - 1;
-                }
-                sl = slot;
-                for (int m = 0; m < nw; ++m) {
-                    const float *x = sX + sl * DKMAX;
-                    const float cm = coef[m];
-#pragma unroll
-                    for (int c = 0; c < DKMAX; ++c) S[c] -= cm * x[c];
-                    sl = sl == 0 ? W - 1 : sl - 1;
+                    for (int w = 0; w < kRecWarps; ++w) ns += sN[sl * kRecWarps + w];
+                    sl = sl == 0 ? RS - 1 : sl - 1;
                 }
             }
-            const float *qq = sQ + (t & 1) * DKMAX;
-            float out = 0.f;
+            const float beta = step_size(e, ns, p.eps);
+
+            // (C) row update and the read after the write
+            if (has_row) {
 #pragma unroll
-            for (int c = 0; c < DKMAX; ++c) out += S[c] * qq[c];
-            Io<IO>::st(o, (size_t)t * dv + tid, out);
+                for (int c = 0; c < DKMAX; ++c) S[c] *= a;  // Sbar
+                if (W == 1) {
+                    const float *x = sX + slot * DKMAX;
+                    const float y = sY[slot * DVP + tid];
+                    const float coef = REGRESSION ? beta * (row_dot<DKMAX>(S, x) - y) : -beta * y;
+#pragma unroll
+                    for (int c = 0; c < DKMAX; c += 4) {
+                        const float4 xv = *reinterpret_cast<const float4 *>(x + c);
+                        S[c] -= coef * xv.x;
+                        S[c + 1] -= coef * xv.y;
+                        S[c + 2] -= coef * xv.z;
+                        S[c + 3] -= coef * xv.w;
+                    }
+                } else {
+                    float coef[kRecMaxWindow];
+                    int sl = slot;
+                    for (int m = 0; m < nw; ++m) {
+                        const float y = sY[sl * DVP + tid];
+                        coef[m] = REGRESSION ? beta * (row_dot<DKMAX>(S, sX + sl * DKMAX) - y) : -beta * y;
+                        sl = sl == 0 ? RS - 1 : sl - 1;
+                    }
+                    sl = slot;
+                    for (int m = 0; m < nw; ++m) {
+                        const float *x = sX + sl * DKMAX;
+                        const float cm = coef[m];
+#pragma unroll
+                        for (int c = 0; c < DKMAX; ++c) S[c] -= cm * x[c];
+                        sl = sl == 0 ? RS - 1 : sl - 1;
+                    }
+                }
+                Io<IO>::st(o, (size_t)t * dv + tid, row_dot<DKMAX>(S, sQ + (t & 1) * DKMAX));
+            }
+            slot = slot + 1 == RS ? 0 : slot + 1;
         }
-        slot = slot + 1 == W ? 0 : slot + 1;
-        __syncthreads();
     }
 
     if (p.S_out && has_row) {
@@ -164,7 +192,8 @@ static int dk_max(int dk) { return dk <= 32 ? 32 : (dk <= 64 ? 64 : 128); }
 
 size_t recurrent_smem_bytes(int dk, int dv, int window) {
     const int D = dk_max(dk);
-    return sizeof(float) * ((size_t)window * (D + dv) + 2 * D);
+    const size_t rs = (size_t)window + 1, dvp = (size_t)((dv + 3) & ~3);
+    return sizeof(float) * (rs * (D + dvp + kRecWarps) + 2 * D);
 }
 
 template <typename IO, bool REG, int DKMAX>

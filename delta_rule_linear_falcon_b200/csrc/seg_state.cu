@@ -23,6 +23,7 @@
 #include "common.cuh"
 #include "launch.h"
 #include "tc_common.cuh"
+#include "tmap.h"
 
 namespace falcon {
 
@@ -40,7 +41,7 @@ constexpr uint32_t oPBar = oRed + 64;
 enum : int { P_FULL = 0, P_SCALED = kStages, P_EMPTY = 2 * kStages, P_DONE = 3 * kStages, P_COUNT };
 constexpr uint32_t kPSmem = oPBar + P_COUNT * 8 + 16 + 1024;   // + TMEM slot and abort flag, alignment slack
 constexpr uint32_t kPCols = 128;
-constexpr long long kPWaitBudget = 1ll << 31;                  // SM clocks, about 1 s
+constexpr long long kPDrainBudget = kDefaultWaitBudget;       // waits for own loads / MMAs in flight at exit
 constexpr uint32_t kIdD = tc::idesc_bf16(128, 128, 1, 1);     // (diag(w) Y)^T (MN-major A) x X (MN-major B)
 constexpr size_t kStateBytes = 128 * 128 * sizeof(float);
 
@@ -55,6 +56,8 @@ struct PieceParams {
     float eps;
     float *D, *a;  // per piece: the state increment (d_v x d_k) and the log2 decay of the piece
     int *err;
+    long long wait_budget;  // bounded waits give up after this many SM clocks
+    int dbg_stall_block;    // test hook: the producer stops loading at this block (-1: never)
 };
 
 struct ScanParams {
@@ -134,9 +137,10 @@ seg_piece_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             const int kshift = p.same_step ? 0 : 1;
             int armed = 0;
             for (int i = 0; i < nst && !*abort_flag; ++i) {
+                if (i == p.dbg_stall_block) break;  // test hook: this block is never loaded
                 const int s = i % kStages;
                 if (i >= kStages &&
-                    !tc::mbar_wait(&bars[P_EMPTY + s], ((i / kStages) - 1) & 1, abort_flag, kPWaitBudget)) {
+                    !tc::mbar_wait(&bars[P_EMPTY + s], ((i / kStages) - 1) & 1, abort_flag, p.wait_budget)) {
                     *abort_flag = 1;
                     break;
                 }
@@ -153,7 +157,7 @@ seg_piece_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             // every armed load must have landed before the CTA can exit
             const volatile int no_abort = 0;
             for (int i = armed - kStages < 0 ? 0 : armed - kStages; i < armed; ++i)
-                tc::mbar_wait(&bars[P_FULL + i % kStages], (i / kStages) & 1, &no_abort, kPWaitBudget);
+                tc::mbar_wait(&bars[P_FULL + i % kStages], (i / kStages) & 1, &no_abort, kPDrainBudget);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (whole warp, elected lane issues)
@@ -163,7 +167,7 @@ seg_piece_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         for (int i = 0; i < nst; ++i) {
             const int s = i % kStages;
             ok = __all_sync(0xffffffffu,
-                            tc::mbar_wait(&bars[P_SCALED + s], (i / kStages) & 1, abort_flag, kPWaitBudget));
+                            tc::mbar_wait(&bars[P_SCALED + s], (i / kStages) & 1, abort_flag, p.wait_budget));
             if (!ok) break;
             tc::fence_after_sync();
             const uint64_t so = (uint64_t)(s * (kStage >> 4));
@@ -176,7 +180,7 @@ seg_piece_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         if (!ok) *abort_flag = 1;
         tc::mma_commit_elect(&bars[P_DONE]);
         const volatile int no_abort = 0;
-        tc::mbar_wait(&bars[P_DONE], 0, &no_abort, kPWaitBudget);
+        tc::mbar_wait(&bars[P_DONE], 0, &no_abort, kPDrainBudget);
         __syncwarp();
     } else {
         // ------------------------------------------------ scaling warps (128 threads), then the drain
@@ -220,7 +224,7 @@ seg_piece_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         for (int i = 0; i < nst; ++i) {
             const int s = i % kStages;
             bool failed = false;
-            if (leader && !tc::mbar_wait(&bars[P_FULL + s], (i / kStages) & 1, abort_flag, kPWaitBudget)) {
+            if (leader && !tc::mbar_wait(&bars[P_FULL + s], (i / kStages) & 1, abort_flag, p.wait_budget)) {
                 *abort_flag = 1;
                 failed = true;
             }
@@ -269,7 +273,7 @@ seg_piece_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         }
         if (ok) {
             bool failed = false;
-            if (leader && !tc::mbar_wait(&bars[P_DONE], 0, abort_flag, kPWaitBudget)) {
+            if (leader && !tc::mbar_wait(&bars[P_DONE], 0, abort_flag, p.wait_budget)) {
                 *abort_flag = 1;
                 failed = true;
             }
@@ -353,39 +357,6 @@ __global__ void __launch_bounds__(256) seg_scan_kernel(ScanParams p) {
     }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
-                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                  CUtensorMapFloatOOBfill);
-
-// Resolved once (a function-local static is initialised once even when several host threads
-// make their first call together).
-EncodeTiledFn encode_fn_seg() {
-    static const EncodeTiledFn fn = []() -> EncodeTiledFn {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            return reinterpret_cast<EncodeTiledFn>(ptr);
-        return nullptr;
-    }();
-    return fn;
-}
-
-// (128 columns, T rows, heads) bf16 view, 64 x 64 boxes, 128-byte swizzle; rows outside
-// [0, T) of a head read as zero.
-bool seg_map(CUtensorMap *m, const void *base, int T, long long heads) {
-    EncodeTiledFn fn = encode_fn_seg();
-    if (!fn) return false;
-    cuuint64_t dims[3] = {128, (cuuint64_t)T, (cuuint64_t)heads};
-    cuuint64_t strides[2] = {128 * 2, (cuuint64_t)T * 128 * 2};
-    cuuint32_t box[3] = {64, 64, 1};
-    cuuint32_t es[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Workspace: D per piece | log2 decay per piece | state at each segment start | cached key per segment.
@@ -438,12 +409,14 @@ cudaError_t launch_chunk_seg(const ChunkParams &p, const SegPlan &pl, void *work
     void *kp = ws + l.oK;
 
     CUtensorMap mK, mV;
-    if (!seg_map(&mK, p.k, p.T, heads) || !seg_map(&mV, p.v, p.T, heads)) return cudaErrorInvalidValue;
+    if (!map_head_rows(&mK, p.k, p.T, heads, 64) || !map_head_rows(&mV, p.v, p.T, heads, 64))
+        return cudaErrorInvalidValue;
     PieceParams pp{};
     pp.T = p.T; pp.piece = pl.piece; pp.pneed = pneed; pp.ptot = ptot;
     pp.same_step = p.same_step; pp.k_prev = p.k_prev;
     pp.alpha = p.alpha; pp.eta = p.eta; pp.eps = p.eps;
     pp.D = D; pp.a = a; pp.err = p.err;
+    pp.wait_budget = p.wait_budget; pp.dbg_stall_block = p.dbg_stall_block;
     cudaError_t e = cudaFuncSetAttribute(seg_piece_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPSmem);
     if (e != cudaSuccess) return e;
     seg_piece_kernel<<<(unsigned)(heads * pneed), kPThreads, kPSmem, stream>>>(mK, mV, pp);

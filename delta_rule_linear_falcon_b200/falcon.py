@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
             L.falcon_check_device_errors.restype = i
             L.falcon_version.argtypes = []
             L.falcon_version.restype = i
+            L.falcon_debug_stall_next_call.argtypes = [i, ctypes.c_longlong]
+            L.falcon_debug_stall_next_call.restype = i
             _lib = L
     return _lib
 
@@ -219,6 +221,12 @@ def falcon_decode_step(S, k_prev, q, k, v, alpha, eta, *, rule="falcon1", eps=1e
     if st != FALCON_OK:
         raise FalconError(st, "falcon_decode_step")
     return o
+
+
+def falcon_debug_stall_next_call(block: int, wait_budget_cycles: int) -> int:
+    """Test hook: the next chunk call of this thread stalls its TMA producers at ``block`` and
+    gives up its waits after ``wait_budget_cycles`` SM clocks (see include/falcon.h)."""
+    return int(lib().falcon_debug_stall_next_call(int(block), int(wait_budget_cycles)))
 
 
 def falcon_check_device_errors(stream=None) -> int:

@@ -133,10 +133,12 @@ FALCON_API size_t falcon_workspace_size(const falcon_args_t *args);
  * Decay factors are only ever formed as exp(g_i - g_j) with i >= j on a
  * block-local cumulative log decay, so each lies in (0, 1].
  *
- * Supported: dk, dv in {32, 64, 128}; chunk in {16, 32, 64}; Falcon-3/3A need
- * 1 <= window <= chunk and process floor(chunk / window) tokens per block.
- * Tensor-core products take bf16 operands with fp32 accumulation and an fp32
- * state, whatever io_dtype is; use falcon_fwd_recurrent for fp32-accurate work.
+ * Supported: io_dtype FALCON_BF16 only; dk, dv in {32, 64, 128}; chunk in
+ * {16, 32, 64}; Falcon-3/3A need 1 <= window <= chunk and process
+ * floor(chunk / window) tokens per block. Tensor-core products take the bf16
+ * inputs as operands with fp32 accumulation and an fp32 state. FALCON_F32
+ * inputs return FALCON_ERR_UNSUPPORTED: bf16 operands could not hold them to an
+ * fp32 error bound, so fp32-accurate work goes through falcon_fwd_recurrent.
  *
  * Sequence split (inner-product write, window 1, dk = dv = 128, bf16, chunk 64,
  * T a multiple of 64, and room for nseg >= 2 segments of at least 8 blocks each
@@ -171,14 +173,18 @@ FALCON_API falcon_status_t falcon_fwd_chunk(const falcon_args_t *args, void *wor
  * Arguments, results and errors are those of falcon_fwd_chunk. Where that call
  * needs workspace (falcon_workspace_size() > 0), this one uses a fixed array of
  * FALCON_NOALLOC_SCRATCH_BYTES in the library's device image instead; every
- * GPU that loads the library holds that array until the process exits. Larger
+ * GPU that uses the library holds that array until the process exits. Larger
  * needs are rejected before anything runs with FALCON_ERR_WORKSPACE (use
  * falcon_fwd_chunk with your own workspace then). The call allocates and frees
  * nothing.
  *
- * The first call on each device resolves the array's device address (with that
- * device current) and keeps it; make that first call before any stream
- * capture. All calls share the one array per device: calls whose kernels can
+ * The array is reserved on a device no later than the first call there (with
+ * lazy module loading, the CUDA default, that first call loads it; with eager
+ * loading it is reserved when the library loads). The first call on each device
+ * resolves the array's device address (with that device current) and keeps it;
+ * make that first call before any stream capture. The kept address does not
+ * survive cudaDeviceReset: do not use this entry point on a device after
+ * resetting it in the same process. All calls share the one array per device: calls whose kernels can
  * overlap on the GPU (different streams without an ordering between them,
  * several host threads) race on it and give wrong results, so order them, for
  * example on one stream. Nothing in the array needs clearing between calls:
@@ -229,6 +235,25 @@ FALCON_API const char *falcon_status_string(falcon_status_t status);
  * (a kernel rejected its launch geometry).
  */
 FALCON_API falcon_status_t falcon_check_device_errors(falcon_stream_t stream);
+
+/*
+ * falcon_debug_stall_next_call -- test hook for the failure path; not for production use.
+ * Arms a one-shot stall for the next falcon_fwd_chunk (or falcon_fwd_chunk_noalloc) call
+ * made from this host thread: the TMA producer of every tensor-core kernel of that call
+ * stops loading at block `block` (0-based 64-row block of each head or segment), and every
+ * bounded device-side wait of the call gives up after `wait_budget_cycles` SM clocks
+ * instead of about 2^31. A consumer's wait then runs out: the kernel records
+ * FALCON_ERR_TIMEOUT in the device error word, waits for its own loads in flight (no load
+ * is left pending, none was started for the stalled block), frees its tensor memory and
+ * returns, so the context stays usable; falcon_check_device_errors() reports the timeout,
+ * the call's outputs are undefined, and the following call runs normally. Calls that run
+ * no tensor-core kernel, or that have fewer blocks than `block`, ignore the stall (it is
+ * consumed all the same). The kernels' waits are bounded whether or not the hook is used;
+ * the hook only lets a test reach that code without faulting or hanging a GPU (the pages
+ * have no counterpart).
+ * Errors: INVALID_ARG for block < 0 or a budget outside [10^4, 2^31].
+ */
+FALCON_API falcon_status_t falcon_debug_stall_next_call(int block, long long wait_budget_cycles);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 FALCON_API int falcon_version(void);

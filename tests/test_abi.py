@@ -81,6 +81,7 @@ def _args(**kw):
     (dict(rule=3, window=0), F.FALCON_ERR_INVALID_ARG),
     (dict(dk=96), F.FALCON_ERR_UNSUPPORTED),
     (dict(dv=48), F.FALCON_ERR_UNSUPPORTED),
+    (dict(io_dtype=0), F.FALCON_ERR_UNSUPPORTED),   # fp32 inputs: the recurrent form serves them
     (dict(chunk=128), F.FALCON_ERR_UNSUPPORTED),
     (dict(chunk=8), F.FALCON_ERR_UNSUPPORTED),
     (dict(rule=3, window=65), F.FALCON_ERR_UNSUPPORTED),
@@ -160,3 +161,19 @@ def test_product_package_never_imports_the_oracle():
                 txt = open(os.path.join(dirpath, fn)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, fn
                 assert "falcon_oracle" not in txt, fn
+
+
+@pytest.mark.parametrize("block,budget,expect", [
+    (-1, 10 ** 6, F.FALCON_ERR_INVALID_ARG),
+    (0, 100, F.FALCON_ERR_INVALID_ARG),
+    (0, 1 << 40, F.FALCON_ERR_INVALID_ARG),
+    (3, 10 ** 6, F.FALCON_OK),
+])
+def test_debug_stall_hook_checks_its_arguments(L, block, budget, expect):
+    """The failure-path test hook validates on the host; arming it launches nothing, and an
+    armed stall is consumed by the next chunk call of the thread (here one with no GPU, which
+    returns FALCON_ERR_CUDA after the host checks)."""
+    assert F.falcon_debug_stall_next_call(block, budget) == expect
+    if expect == F.FALCON_OK:
+        a = _args()
+        assert L.falcon_fwd_chunk(ctypes.byref(a), None, 0, None) in (F.FALCON_ERR_CUDA, F.FALCON_OK)

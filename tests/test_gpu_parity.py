@@ -1,10 +1,10 @@
 """GPU parity: the CUDA library (through its C ABI) against the fp64 CPU oracle,
 element by element on the same seeded inputs.
 
-Tolerance (max |gpu - oracle| / max |oracle|): 1e-4 for fp32 inputs with fp32
-arithmetic (recurrent and decode paths), 2e-2 for bf16 inputs or the
-chunk-parallel path, whose tensor-core products take bf16 operands with fp32
-accumulation and an fp32 state.
+Tolerance (max |gpu - oracle| / max |oracle|): 1e-4 for fp32 inputs (the recurrent
+and decode paths, fp32 arithmetic), 2e-2 for bf16 inputs with an fp32 state. The
+chunk-parallel path takes bf16 inputs only (its tensor-core operands are the bf16
+inputs themselves) and refuses fp32 ones, so no fp32 input is ever held to 2e-2.
 """
 import math
 
@@ -120,10 +120,16 @@ def test_chunk_mixed_widths(F, dk, dv):
     check(s, run_gpu(F, s, "chunk"), run_oracle(s), TOL_BF16)
 
 
-def test_chunk_fp32_io(F):
-    """fp32 I/O through the chunk path: bf16 tensor-core operands, bf16 tolerance."""
-    s = I.make_seq(1, 2, 4, 300, 128, 128, seed=8, io_dtype="f32", with_state=True, with_kprev=True)
-    check(s, run_gpu(F, s, "chunk"), run_oracle(s), TOL_BF16)
+@pytest.mark.parametrize("rule,d", [(1, 128), (2, 128), (3, 64)])
+def test_chunk_refuses_fp32_io(F, rule, d):
+    """fp32 I/O is refused by the chunk path (its bf16 tensor-core operands could not meet the
+    fp32 error bound) before anything is launched; the recurrent path serves fp32 at 1e-4."""
+    s = I.make_seq(rule, 2, 4, 300, d, d, seed=8, io_dtype="f32", window=2 if rule == 3 else 1,
+                   with_state=True, with_kprev=True)
+    with pytest.raises(F.FalconError) as ei:
+        run_gpu(F, s, "chunk")
+    assert ei.value.status == F.FALCON_ERR_UNSUPPORTED
+    check(s, run_gpu(F, s, "recurrent"), run_oracle(s), TOL_F32)
 
 
 @pytest.mark.parametrize("T", [0, 1, 2, 63, 64, 65])
@@ -195,36 +201,57 @@ def test_chunk_guard_bands_untouched(F):
 
 # ------------------------------------------------------------------ full-size workloads
 
-FULL_HEADS = [(0, 0), (3, 7)]
+def _spread_heads(B, H, n=16):
+    """n distinct (b, h) pairs spread over the batch and the heads (so over CTAs and SMs)."""
+    pairs, i = [], 0
+    while len(pairs) < min(n, B * H):
+        bh = (i * 37 + 5) % (B * H)
+        if (bh // H, bh % H) not in pairs:
+            pairs.append((bh // H, bh % H))
+        i += 1
+    return pairs
 
 
-def _sampled(s, b, h):
-    return (slice(b, b + 1), slice(h, h + 1))
+def _gather(s: I.SeqInputs, pairs):
+    """The sampled heads of a workload as one (1, n, ...) problem, so that the oracle runs them
+    in one call (OpenMP over heads)."""
+    b = np.array([p[0] for p in pairs])
+    h = np.array([p[1] for p in pairs])
+    take = lambda x: None if x is None else np.ascontiguousarray(x[b, h][None])
+    return I.SeqInputs(s.rule, s.io_dtype, take(s.q), take(s.k), take(s.v), take(s.alpha), take(s.eta),
+                       s.eps, window=s.window, chunk=s.chunk, S0=take(s.S0), k_prev=take(s.k_prev))
 
 
-@pytest.mark.parametrize("b,h", FULL_HEADS)
-def test_full_falcon1_chunk_workload(F, b, h):
-    """Falcon-1 chunk-parallel at full size (B8 H16 T4096 d128, chunk 64), sampled heads."""
-    s = _full("f1")
-    got = _full_gpu(F, "f1")
-    hs = _sampled(s, b, h)
-    check(s, got, run_oracle(s, hs), TOL_BF16, heads=hs)
+def _check_full(name):
+    s = _full(name)
+    o, S, kl = _full_gpu(name)
+    B, H = s.q.shape[:2]
+    pairs = _spread_heads(B, H)
+    b = np.array([p[0] for p in pairs])
+    h = np.array([p[1] for p in pairs])
+    g = _gather(s, pairs)
+    return check(g, (o[b, h][None], S[b, h][None], kl[b, h][None]), run_oracle(g), TOL_BF16)
+
+
+def test_full_falcon1_chunk_workload(F):
+    """Falcon-1 chunk-parallel at full size (B8 H16 T4096 d128, chunk 64), 16 heads spread over
+    the batch and the heads."""
+    _check_full("f1")
 
 
 def test_full_falcon1a_long_workload(F):
-    """Falcon-1A at full size (B1 H16 T32768 d128): long-range decay renormalisation."""
-    s = _full("f1a")
-    got = _full_gpu(F, "f1a")
-    hs = _sampled(s, 0, 5)
-    check(s, got, run_oracle(s, hs), TOL_BF16, heads=hs)
+    """Falcon-1A at full size (B1 H16 T32768 d128): long-range decay renormalisation, all 16 heads."""
+    _check_full("f1a")
 
 
 def test_full_falcon3_workload(F):
-    """Falcon-3 (w = 4) at full size (B4 H16 T8192 d128), one sampled head."""
-    s = _full("f3")
-    got = _full_gpu(F, "f3")
-    hs = _sampled(s, 2, 11)
-    check(s, got, run_oracle(s, hs), TOL_BF16, heads=hs)
+    """Falcon-3 (w = 4) at full size (B4 H16 T8192 d128), 16 sampled heads."""
+    _check_full("f3")
+
+
+def test_full_falcon3a_workload(F):
+    """Falcon-3A (w = 4) at full size (B4 H16 T8192 d128, the Falcon-3 inputs), 16 sampled heads."""
+    _check_full("f3a")
 
 
 _FULL = {}
@@ -232,16 +259,23 @@ _FULL = {}
 
 def _full(name):
     if name not in _FULL:
-        _FULL[name] = {"f1": I.workload_chunk_f1, "f1a": I.workload_chunk_f1a_long,
-                       "f3": I.workload_chunk_f3}[name]()
+        if name == "f3a":
+            s = I.workload_chunk_f3()
+            s.rule = I.RULE_3A
+            _FULL[name] = s
+        else:
+            _FULL[name] = {"f1": I.workload_chunk_f1, "f1a": I.workload_chunk_f1a_long,
+                           "f3": I.workload_chunk_f3}[name]()
     return _FULL[name]
 
 
 _FULL_OUT = {}
 
 
-def _full_gpu(F, name):
+def _full_gpu(name):
+    import delta_rule_linear_falcon_b200.falcon as F
     if name not in _FULL_OUT:
+        _FULL_OUT.clear()   # one full-size result on the device at a time
         _FULL_OUT[name] = run_gpu(F, _full(name), "chunk")
     return _FULL_OUT[name]
 

@@ -20,7 +20,7 @@ SS = 0x100
     (2, 1, 128, 64, "bf16"),   # tensor-core kernel, inner-product rule
     (1, 1, 64, 32, "bf16"),    # mma.sync kernel
     (3, 4, 64, 64, "bf16"),    # windowed
-    (4, 2, 32, 16, "f32"),
+    (4, 2, 32, 16, "bf16"),
 ])
 def test_same_step_chunk(F, rule, w, d, chunk, io):
     """Several blocks and a ragged tail, an initial state and a cached key (which must be ignored)."""

@@ -5,7 +5,8 @@ which a cudaMalloc could synchronise the device).
 
 Called through the C ABI and compared with falcon_fwd_chunk on a workspace of the
 caller's own, on two calls in a row with different inputs (the second call finds the
-first one's leftovers in the shared array), on a problem that needs no scratch, and on a
+first one's leftovers in the shared array), on a smaller problem without state outputs
+after a larger one, on a problem that needs no scratch, and on a
 problem whose scratch would not fit, which must be refused before anything runs. This
 file is collected last so that a run stopping at its first failure has run every other
 test; it passes alone in a fresh process as well.
@@ -31,7 +32,7 @@ def _noalloc(F):
     return fn
 
 
-def _tensors(F, s: I.SeqInputs):
+def _tensors(F, s: I.SeqInputs, want_state=True):
     q, k, v = (dev(x, torch.bfloat16) for x in (s.q, s.k, s.v))
     a, e = dev(s.alpha, torch.float32), dev(s.eta, torch.float32)
     S0 = dev(s.S0, torch.float32) if s.S0 is not None else None
@@ -39,15 +40,16 @@ def _tensors(F, s: I.SeqInputs):
     B, H, T, dk = k.shape
     dv = v.shape[-1]
     o = torch.empty_like(v)
-    S = torch.empty((B, H, dv, dk), dtype=torch.float32, device="cuda")
-    kl = torch.empty((B, H, dk), dtype=torch.bfloat16, device="cuda")
+    S = torch.empty((B, H, dv, dk), dtype=torch.float32, device="cuda") if want_state else None
+    kl = torch.empty((B, H, dk), dtype=torch.bfloat16, device="cuda") if want_state else None
     args = F.make_args(q, k, v, a, e, rule=s.rule, eps=s.eps, chunk=64, S0=S0, k_prev=kp, o=o, S_out=S,
                        k_last=kl)
-    return args, (o, S, kl), (q, k, v, a, e, S0, kp)
+    outs = (o, S, kl) if want_state else (o,)
+    return args, outs, (q, k, v, a, e, S0, kp)
 
 
-def _run(F, s, noalloc):
-    args, outs, keep = _tensors(F, s)
+def _run(F, s, noalloc, want_state=True):
+    args, outs, keep = _tensors(F, s, want_state)
     L = F.lib()
     need = L.falcon_workspace_size(ctypes.byref(args))
     if noalloc:
@@ -81,6 +83,26 @@ def test_noalloc_matches_the_workspace_entry_point_on_two_calls(F):
         need2, got = _run(F, s, noalloc=True)
         assert need2 == need
         _same(got, ref)
+
+
+def test_noalloc_smaller_problem_without_state_after_a_larger_one(F):
+    """A larger split problem fills more of the shared array; a smaller one with a different
+    head count and length, and no final state or key requested (the split then skips the last
+    segment's pieces and takes that segment's start state from the scan alone), follows it and
+    must not read the leftovers."""
+    big = I.make_seq(2, 1, 2, 8192, 128, 128, seed=780, io_dtype="bf16", normalise_qk=False,
+                     alpha_mu=6.0, with_state=True, with_kprev=True)
+    small = I.make_seq(2, 1, 3, 2048, 128, 128, seed=781, io_dtype="bf16", normalise_qk=False,
+                       alpha_mu=6.0, with_state=True, with_kprev=True)
+    need_b, ref_b = _run(F, big, noalloc=False)
+    need_s, ref_s = _run(F, small, noalloc=False, want_state=False)
+    assert 0 < need_s < need_b <= SCRATCH_BYTES
+    _same(_run(F, big, noalloc=True)[1], ref_b)
+    for _ in range(2):
+        need2, (o,) = _run(F, small, noalloc=True, want_state=False)
+        assert need2 == need_s
+        assert np.all(np.isfinite(o))
+        assert relerr(o, ref_s[0]) <= TOL_BF16
 
 
 def test_noalloc_without_scratch_runs_the_plain_pass(F):
