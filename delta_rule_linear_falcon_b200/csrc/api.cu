@@ -56,8 +56,11 @@ bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0
 
 int base_rule(int r) { return r & ~FALCON_SAME_STEP; }
 bool same_step(int r) { return (r & FALCON_SAME_STEP) != 0; }
-bool rule_valid(int r) { return base_rule(r) >= FALCON_RULE_1 && base_rule(r) <= FALCON_RULE_3A; }
-bool is_regression(int r) { return base_rule(r) == FALCON_RULE_1 || base_rule(r) == FALCON_RULE_3; }
+bool rule_valid(int r) { return base_rule(r) >= FALCON_RULE_1 && base_rule(r) <= FALCON_RULE_2A; }
+bool is_regression(int r) {
+    return base_rule(r) == FALCON_RULE_1 || base_rule(r) == FALCON_RULE_3 || base_rule(r) == FALCON_RULE_2;
+}
+bool is_per_column(int r) { return base_rule(r) == FALCON_RULE_2 || base_rule(r) == FALCON_RULE_2A; }
 bool is_windowed(int r) { return base_rule(r) == FALCON_RULE_3 || base_rule(r) == FALCON_RULE_3A; }
 
 // Checks shared by the two sequence entry points.
@@ -82,6 +85,8 @@ falcon_status_t check_seq_args(const falcon_args_t *a) {
     if (a->S_out && !aligned16(a->S_out)) return FALCON_ERR_INVALID_ARG;
     if (a->k_prev && !aligned16(a->k_prev)) return FALCON_ERR_INVALID_ARG;
     if (a->k_last && !aligned16(a->k_last)) return FALCON_ERR_INVALID_ARG;
+    if (is_per_column(a->rule) && ((a->n0 && !aligned4(a->n0)) || (a->n_out && !aligned4(a->n_out))))
+        return FALCON_ERR_INVALID_ARG;
     return FALCON_OK;
 }
 
@@ -144,6 +149,7 @@ extern "C" {
 
 size_t falcon_workspace_size(const falcon_args_t *a) {
     if (!a || check_seq_args(a) != FALCON_OK) return 0;
+    if (is_per_column(a->rule)) return 0;
     if (a->io_dtype != FALCON_BF16) return 0;
     if (!dim_supported_chunk(a->dk) || !dim_supported_chunk(a->dv)) return 0;
     if (a->chunk != 16 && a->chunk != 32 && a->chunk != 64) return 0;
@@ -161,6 +167,7 @@ falcon_status_t falcon_fwd_chunk(const falcon_args_t *a, void *workspace, size_t
     // The chunk form's products take bf16 tensor-core operands; fp32 inputs would be held to a
     // bf16 error bound, so fp32-accurate work goes through falcon_fwd_recurrent instead.
     if (a->io_dtype != FALCON_BF16) return FALCON_ERR_UNSUPPORTED;
+    if (is_per_column(a->rule)) return FALCON_ERR_UNSUPPORTED;   // Falcon-2/2A: falcon_fwd_recurrent
     if (!dim_supported_chunk(a->dk) || !dim_supported_chunk(a->dv)) return FALCON_ERR_UNSUPPORTED;
     if (a->chunk != 16 && a->chunk != 32 && a->chunk != 64) return FALCON_ERR_UNSUPPORTED;
     const int w = is_windowed(a->rule) ? a->window : 1;
@@ -197,10 +204,13 @@ falcon_status_t falcon_fwd_recurrent(const falcon_args_t *a, falcon_stream_t str
     p.B = a->B; p.H = a->H; p.T = a->T; p.dk = a->dk; p.dv = a->dv; p.window = w;
     p.regression = is_regression(a->rule);
     p.same_step = same_step(a->rule);
+    p.per_column = is_per_column(a->rule);
     p.io_bf16 = a->io_dtype == FALCON_BF16;
     p.q = a->q; p.k = a->k; p.v = a->v; p.k_prev = a->k_prev;
     p.alpha = a->alpha; p.eta = a->eta; p.S0 = a->S0; p.eps = a->eps;
     p.o = a->o; p.k_last = a->k_last; p.S_out = a->S_out;
+    p.n0 = p.per_column ? a->n0 : nullptr;
+    p.n_out = p.per_column ? a->n_out : nullptr;
     int sms = 0;
     if (!device_info(&p.err, &sms)) return FALCON_ERR_CUDA;
     return launch_recurrent(p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? FALCON_OK
@@ -215,7 +225,7 @@ falcon_status_t falcon_decode_step(int rule, int io_dtype, int N, int H, int dk,
     if (io_dtype != FALCON_F32 && io_dtype != FALCON_BF16) return FALCON_ERR_INVALID_ARG;
     if (N < 0 || H < 0 || dk <= 0 || dv <= 0) return FALCON_ERR_INVALID_ARG;
     if (!(eps >= 0.f) || !isfinite(eps)) return FALCON_ERR_INVALID_ARG;
-    if (is_windowed(rule)) return FALCON_ERR_UNSUPPORTED;
+    if (is_windowed(rule) || is_per_column(rule)) return FALCON_ERR_UNSUPPORTED;
     if (dk != 32 && dk != 64 && dk != 128) return FALCON_ERR_UNSUPPORTED;
     if (dv > 256) return FALCON_ERR_UNSUPPORTED;
     const long long nh = (long long)N * H;

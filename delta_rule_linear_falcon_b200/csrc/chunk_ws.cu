@@ -519,8 +519,9 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         for (int c = 0; c < nblk && ok && REG; ++c) {
             const int s = c & 1, u = c % 3;
             // (b) S X^T (regression only) then S Q^T -> slot s, S (bf16) from TMEM; the chain starts
-            // forming R'^T as soon as the first half is done
-            if (!(ok = wait_all(B_SRDY, c & 1))) break;
+            // forming R'^T as soon as the first half is done. The [X;Q] slot must have landed (and the
+            // cached key be patched into block 0): the helpers' readiness of the block says both.
+            if (!(ok = wait_all(B_SRDY, c & 1) && wait_all(B_XQRDY + u, (c / 3) & 1))) break;
             tc::fence_after_sync();
             const uint64_t dX = dXQ0 + slot_off(u), dQ = dX + (8192 >> 4);   // X rows 0-63, Q rows 64-127
             if (REG) {
@@ -890,36 +891,25 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             tc::tmem_st32(tl + cSR + 32 * hf, pk);
         };
         // O^T of block c (TMEM slot c & 1: S Q^T scaled by 2^g per token, plus R'^T B'^T) to global
-        // memory: lane pairs (2k, 2k+1) hold neighbouring value rows; the even lane stores the pair for
-        // even tokens, the odd lane for odd tokens.
+        // memory: for each token a warp stores the bf16 outputs of its 32 consecutive value rows, 64
+        // contiguous bytes per store instruction.
         auto store_out = [&](int c) {
             const int t0 = c * TB, nval = min(TB, T - t0);
-            const bool odd = lane & 1;
-            __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.o) + ((size_t)bh * T + t0) * D + (row & ~1);
+            __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.o) + ((size_t)bh * T + t0) * D + row;
 #pragma unroll 1
-            for (int h = 0; h < 2; ++h) {          // 16 tokens at a time
-                const int i0 = 32 * hf + 16 * h;
+            for (int h = 0; h < 4; ++h) {          // 8 tokens at a time
+                const int i0 = 32 * hf + 8 * h;
                 if (i0 >= TB) break;               // a block has TB query tokens
                 const float *d2 = sScal + (c % 4) * 256 + 64 + i0;   // 2^g of the tokens
                 // the scales first, so that their shared-memory latency overlaps the TMEM loads
-                float dg[16];
+                const float4 da = *reinterpret_cast<const float4 *>(d2);
+                const float4 db = *reinterpret_cast<const float4 *>(d2 + 4);
+                const float dg[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+                float v[8], w[8];
+                tc::tmem_ld8x2(tl + cSXO + 128 * (c & 1) + 64 + i0, tl + cSXO + 128 * (c & 1) + i0, v, w);
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const float4 d4 = *reinterpret_cast<const float4 *>(d2 + 4 * q4);
-                    dg[4 * q4] = d4.x; dg[4 * q4 + 1] = d4.y; dg[4 * q4 + 2] = d4.z; dg[4 * q4 + 3] = d4.w;
-                }
-                float v[16], w[16];
-                tc::tmem_ld16x2(tl + cSXO + 128 * (c & 1) + 64 + i0, tl + cSXO + 128 * (c & 1) + i0, v, w);
-#pragma unroll
-                for (int j = 0; j < 16; j += 2) {
-                    const float v0 = dg[j] * v[j] + w[j], v1 = dg[j + 1] * v[j + 1] + w[j + 1];
-                    const float mine = odd ? v1 : v0;
-                    const float give = odd ? v0 : v1;
-                    const float other = __shfl_xor_sync(0xffffffffu, give, 1);
-                    const int i = i0 + j + (odd ? 1 : 0);
-                    const float lo = odd ? other : mine, hi = odd ? mine : other;
-                    if (i < nval) *reinterpret_cast<uint32_t *>(o + (size_t)i * D) = pack_bf16x2(lo, hi);
-                }
+                for (int j = 0; j < 8; ++j)
+                    if (i0 + j < nval) o[(size_t)(i0 + j) * D] = __float2bfloat16_rn(dg[j] * v[j] + w[j]);
             }
         };
         {

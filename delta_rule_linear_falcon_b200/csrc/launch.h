@@ -11,6 +11,9 @@ struct RecParams {
     int B, H, T, dk, dv, window;  // window = 1 for Falcon-1/1A
     bool regression, io_bf16;
     bool same_step;               // pair (k_t, v_t) instead of (k_{t-1}, v_t)
+    bool per_column;              // Falcon-2/2A: write key z = eta D x / (x^T D x + eps)
+    const float *n0;              // (B,H,dk) running column energies, or NULL (Falcon-2/2A)
+    float *n_out;
     const void *q, *k, *v, *k_prev;
     const float *alpha, *eta, *S0;
     float eps;

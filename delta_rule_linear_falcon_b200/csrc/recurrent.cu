@@ -15,6 +15,10 @@
 //   regression:     S_i = Sbar_i - beta sum_m (Sbar_i . x_{t-m} - y_{t-m,i}) x_{t-m}
 //   inner product:  S_i = Sbar_i + beta sum_m y_{t-m,i} x_{t-m}
 //   o_{t,i} = S_i . q_t                       (read after write)
+// Falcon-2 / 2A (window 1): thread c also keeps the running energy n_c of key coordinate c,
+// n_c <- alpha_t n_c + x_c^2, and stages the write key direction z_c = x_c / (n_c + eps) beside
+// the key; the pair's norm partial is x . z, so beta = eta / (x^T D x + eps) and the row update is
+//   Falcon-2:  S_i = Sbar_i - beta (Sbar_i . x - y_i) z      Falcon-2A: S_i = Sbar_i + beta y_i z
 #include "common.cuh"
 #include "launch.h"
 
@@ -42,7 +46,7 @@ __device__ __forceinline__ float row_dot(const float (&S)[DKMAX], const float *x
     return (a0 + a1) + (a2 + a3);
 }
 
-template <typename IO, bool REGRESSION, int DKMAX>
+template <typename IO, bool REGRESSION, int DKMAX, bool PERCOL>
 __global__ void __launch_bounds__(kRecThreads)
 recurrent_kernel(RecParams p) {
     extern __shared__ __align__(16) float smem[];
@@ -52,6 +56,7 @@ recurrent_kernel(RecParams p) {
     const int DVP = (dv + 3) & ~3;
     float *sQ = sY + (size_t)RS * DVP;       // 2 x DKMAX queries (double buffered)
     float *sN = sQ + 2 * DKMAX;              // RS x kRecWarps partial squared norms of the pairs
+    float *sZ = sN + RS * kRecWarps;         // per-column rules: RS x DKMAX write-key directions
     constexpr int kAhead = ahead<DKMAX>();
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -65,7 +70,10 @@ recurrent_kernel(RecParams p) {
     const float *eta = p.eta + bh * (size_t)T;
     IO *o = reinterpret_cast<IO *>(p.o) + bh * (size_t)T * dv;
 
-    for (int idx = tid; idx < RS * (DKMAX + DVP + kRecWarps) + 2 * DKMAX; idx += kRecThreads) smem[idx] = 0.f;
+    for (int idx = tid; idx < RS * (DKMAX + DVP + kRecWarps) + 2 * DKMAX + (PERCOL ? RS * DKMAX : 0); idx += kRecThreads)
+        smem[idx] = 0.f;
+    // running energy of key coordinate tid (per-column rules)
+    float ncol = (PERCOL && p.n0 && tid < dk) ? p.n0[bh * (size_t)dk + tid] : 0.f;
 
     const bool has_row = tid < dv;
     float S[DKMAX];
@@ -106,6 +114,13 @@ recurrent_kernel(RecParams p) {
             // (A) stage pair t and q_t with the pair's squared-norm partial, refill the queue slot
             {
                 float x2 = xr[i] * xr[i];
+                if (PERCOL) {   // x . z with z = D x: the D-weighted squared norm
+                    ncol = ar[i] * ncol + x2;
+                    const float den = ncol + p.eps;
+                    const float z = (tid < dk && den > 0.f) ? xr[i] / den : 0.f;
+                    if (tid < dk) sZ[slot * DKMAX + tid] = z;   // entries dk.. stay zero
+                    x2 = z * xr[i];
+                }
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) x2 += __shfl_xor_sync(0xffffffffu, x2, off);
                 if (lane == 0) sN[slot * kRecWarps + warp] = x2;
@@ -138,11 +153,12 @@ recurrent_kernel(RecParams p) {
                 for (int c = 0; c < DKMAX; ++c) S[c] *= a;  // Sbar
                 if (W == 1) {
                     const float *x = sX + slot * DKMAX;
+                    const float *zw = PERCOL ? sZ + slot * DKMAX : x;   // write-key direction
                     const float y = sY[slot * DVP + tid];
                     const float coef = REGRESSION ? beta * (row_dot<DKMAX>(S, x) - y) : -beta * y;
 #pragma unroll
                     for (int c = 0; c < DKMAX; c += 4) {
-                        const float4 xv = *reinterpret_cast<const float4 *>(x + c);
+                        const float4 xv = *reinterpret_cast<const float4 *>(zw + c);
                         S[c] -= coef * xv.x;
                         S[c + 1] -= coef * xv.y;
                         S[c + 2] -= coef * xv.z;
@@ -171,6 +187,7 @@ recurrent_kernel(RecParams p) {
         }
     }
 
+    if (PERCOL && p.n_out && tid < dk) p.n_out[bh * (size_t)dk + tid] = ncol;
     if (p.S_out && has_row) {
         float *So = p.S_out + (bh * (size_t)dv + tid) * dk;
 #pragma unroll
@@ -193,13 +210,13 @@ static int dk_max(int dk) { return dk <= 32 ? 32 : (dk <= 64 ? 64 : 128); }
 size_t recurrent_smem_bytes(int dk, int dv, int window) {
     const int D = dk_max(dk);
     const size_t rs = (size_t)window + 1, dvp = (size_t)((dv + 3) & ~3);
-    return sizeof(float) * (rs * (D + dvp + kRecWarps) + 2 * D);
+    return sizeof(float) * (rs * (D + dvp + kRecWarps) + 2 * D + rs * D);   // + write-key ring
 }
 
 template <typename IO, bool REG, int DKMAX>
 static cudaError_t launch_rec(const RecParams &p, cudaStream_t s) {
     const size_t smem = recurrent_smem_bytes(p.dk, p.dv, p.window);
-    auto kern = recurrent_kernel<IO, REG, DKMAX>;
+    auto kern = p.per_column ? recurrent_kernel<IO, REG, DKMAX, true> : recurrent_kernel<IO, REG, DKMAX, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long grid = (long)p.B * p.H;
@@ -219,6 +236,7 @@ static cudaError_t launch_rec_dk(const RecParams &p, cudaStream_t s) {
 
 cudaError_t launch_recurrent(const RecParams &p, cudaStream_t s) {
     if (p.dk > 128 || p.dv > kRecThreads || p.window > kRecMaxWindow || p.window < 1) return cudaErrorInvalidValue;
+    if (p.per_column && p.window != 1) return cudaErrorInvalidValue;
     const bool reg = p.regression;
     if (p.io_bf16) return reg ? launch_rec_dk<__nv_bfloat16, true>(p, s) : launch_rec_dk<__nv_bfloat16, false>(p, s);
     return reg ? launch_rec_dk<float, true>(p, s) : launch_rec_dk<float, false>(p, s);

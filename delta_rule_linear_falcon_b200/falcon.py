@@ -19,10 +19,11 @@ LIB_PATH = os.path.join(PKG, "libfalcon.so")
 FALCON_OK, FALCON_ERR_INVALID_ARG, FALCON_ERR_UNSUPPORTED = 0, 1, 2
 FALCON_ERR_WORKSPACE, FALCON_ERR_CUDA, FALCON_ERR_TIMEOUT = 3, 4, 5
 FALCON_RULE_1, FALCON_RULE_1A, FALCON_RULE_3, FALCON_RULE_3A = 1, 2, 3, 4
+FALCON_RULE_2, FALCON_RULE_2A = 5, 6
 FALCON_F32, FALCON_BF16 = 0, 1
 FALCON_SAME_STEP = 0x100  # OR into a rule code: pair (k_t, v_t) at step t (same-step association)
 RULES = {"falcon1": FALCON_RULE_1, "falcon1a": FALCON_RULE_1A, "falcon3": FALCON_RULE_3,
-         "falcon3a": FALCON_RULE_3A}
+         "falcon3a": FALCON_RULE_3A, "falcon2": FALCON_RULE_2, "falcon2a": FALCON_RULE_2A}
 
 
 class FalconError(RuntimeError):
@@ -42,6 +43,7 @@ class FalconArgs(ctypes.Structure):
         ("eps", ctypes.c_float), ("window", ctypes.c_int), ("chunk", ctypes.c_int),
         ("S0", ctypes.c_void_p), ("k_prev", ctypes.c_void_p), ("o", ctypes.c_void_p),
         ("S_out", ctypes.c_void_p), ("k_last", ctypes.c_void_p),
+        ("n0", ctypes.c_void_p), ("n_out", ctypes.c_void_p),
     ]
 
 
@@ -127,19 +129,19 @@ def _rule_code(rule) -> int:
 
 
 def make_args(q, k, v, alpha, eta, *, rule, eps=1e-6, window=1, chunk=64, S0=None, k_prev=None,
-              o=None, S_out=None, k_last=None) -> FalconArgs:
+              o=None, S_out=None, k_last=None, n0=None, n_out=None) -> FalconArgs:
     """Fill falcon_args_t from tensors (shapes taken from k and v)."""
     B, H, T, dk = k.shape
     dv = v.shape[-1]
     io = _dtype_code(k)
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (k_prev, "k_prev"), (k_last, "k_last")):
         _need(t, n, k.dtype)
-    for t, n in ((alpha, "alpha"), (eta, "eta"), (S0, "S0"), (S_out, "S_out")):
+    for t, n in ((alpha, "alpha"), (eta, "eta"), (S0, "S0"), (S_out, "S_out"), (n0, "n0"), (n_out, "n_out")):
         _need(t, n, torch.float32)
     return FalconArgs(_rule_code(rule), io, B, H, T, dk, dv, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                       alpha.data_ptr(), eta.data_ptr(), float(eps), int(window), int(chunk),
                       _ptr(S0), _ptr(k_prev), o.data_ptr() if o is not None else None,
-                      _ptr(S_out), _ptr(k_last))
+                      _ptr(S_out), _ptr(k_last), _ptr(n0), _ptr(n_out))
 
 
 def _outputs(k, v, o, S_out, k_last, want_state: bool):
@@ -191,11 +193,13 @@ def falcon_fwd_chunk(q, k, v, alpha, eta, *, rule, eps=1e-6, window=1, chunk=64,
 
 
 def falcon_fwd_recurrent(q, k, v, alpha, eta, *, rule, eps=1e-6, window=1, S0=None, k_prev=None,
-                         o=None, S_out=None, k_last=None, want_state=True, stream=None):
-    """Recurrent forward pass (fp32 arithmetic). Returns (o, S_out, k_last)."""
+                         o=None, S_out=None, k_last=None, want_state=True, n0=None, n_out=None,
+                         stream=None):
+    """Recurrent forward pass (fp32 arithmetic). Returns (o, S_out, k_last); for Falcon-2/2A
+    pass n_out (B, H, dk) fp32 to receive the running column energies (n0 to start from them)."""
     o, S_out, k_last = _outputs(k, v, o, S_out, k_last, want_state)
     args = make_args(q, k, v, alpha, eta, rule=rule, eps=eps, window=window, chunk=64, S0=S0,
-                     k_prev=k_prev, o=o, S_out=S_out, k_last=k_last)
+                     k_prev=k_prev, o=o, S_out=S_out, k_last=k_last, n0=n0, n_out=n_out)
     st = lib().falcon_fwd_recurrent(ctypes.byref(args), _stream(stream))
     if st != FALCON_OK:
         raise FalconError(st, "falcon_fwd_recurrent")

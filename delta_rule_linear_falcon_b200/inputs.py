@@ -112,8 +112,9 @@ def l2_normalise_rows(x: np.ndarray) -> np.ndarray:
     return (x / n).astype(np.float32)
 
 
-RULE_1, RULE_1A, RULE_3, RULE_3A = 1, 2, 3, 4
-RULE_NAMES = {RULE_1: "falcon1", RULE_1A: "falcon1a", RULE_3: "falcon3", RULE_3A: "falcon3a"}
+RULE_1, RULE_1A, RULE_3, RULE_3A, RULE_2, RULE_2A = 1, 2, 3, 4, 5, 6
+RULE_NAMES = {RULE_1: "falcon1", RULE_1A: "falcon1a", RULE_3: "falcon3", RULE_3A: "falcon3a",
+              RULE_2: "falcon2", RULE_2A: "falcon2a"}
 
 
 @dataclass

@@ -16,6 +16,12 @@
  *       S_t  = Sbar - beta_t sum_{j in W_t} (Sbar x_j - y_j) x_j^T
  *   Falcon-1A / Falcon-3A (negative inner-product objective):
  *       S_t  = Sbar + beta_t sum_{j in W_t} y_j x_j^T
+ *   Falcon-2 / Falcon-2A (the per-column extension; a reading of the pages, which
+ *   name it without equations): column c of S keeps the running energy of its key
+ *   coordinate, n_{t,c} = alpha_t n_{t-1,c} + x_{t,c}^2, and the step is the NLMS
+ *   step in the metric D = diag(1 / (n_c + eps)):
+ *       z_t = eta_t D x_t / (x_t^T D x_t + eps)
+ *       Falcon-2:  S_t = Sbar - (Sbar x_t - y_t) z_t^T     Falcon-2A: S_t = Sbar + y_t z_t^T
  * The step size is the Kaczmarz/NLMS one (Kaczmarz Linear Attention abstract,
  * thelatestinai.com page "Fast Weight Attention for Continual Learning").
  * W_t = {max(1, t-w+1) .. t} (1-based). x_1 = k_prev when a cache is given,
@@ -71,7 +77,9 @@ typedef enum {
     FALCON_RULE_1 = 1,  /* Falcon-1: scalar NLMS                                  */
     FALCON_RULE_1A = 2, /* Falcon-1A: normalised additive (inner-product) write   */
     FALCON_RULE_3 = 3,  /* Falcon-3: sliding-window mini-batch (window w)         */
-    FALCON_RULE_3A = 4  /* Falcon-3A: windowed inner-product write (window w)     */
+    FALCON_RULE_3A = 4, /* Falcon-3A: windowed inner-product write (window w)     */
+    FALCON_RULE_2 = 5,  /* Falcon-2: per-column normalised NLMS (see below)       */
+    FALCON_RULE_2A = 6  /* Falcon-2A: its inner-product counterpart               */
 } falcon_rule_t;
 
 /*
@@ -107,6 +115,10 @@ typedef struct {
     void *o;            /* (B,H,T,dv) output, written                                  */
     float *S_out;       /* (B,H,dv,dk) final state, or NULL                            */
     void *k_last;       /* (B,H,dk) last key (the cache for a continuation), or NULL   */
+    const float *n0;    /* Falcon-2/2A: (B,H,dk) running column energies to start from,
+                           or NULL for zero; ignored by the other rules                */
+    float *n_out;       /* Falcon-2/2A: (B,H,dk) running column energies after the
+                           sequence (part of the continuation cache), or NULL          */
 } falcon_args_t;
 
 /*
@@ -133,7 +145,8 @@ FALCON_API size_t falcon_workspace_size(const falcon_args_t *args);
  * Decay factors are only ever formed as exp(g_i - g_j) with i >= j on a
  * block-local cumulative log decay, so each lies in (0, 1].
  *
- * Supported: io_dtype FALCON_BF16 only; dk, dv in {32, 64, 128}; chunk in
+ * Supported: Falcon-1/1A/3/3A (Falcon-2/2A return UNSUPPORTED here: they run on
+ * falcon_fwd_recurrent); io_dtype FALCON_BF16 only; dk, dv in {32, 64, 128}; chunk in
  * {16, 32, 64}; Falcon-3/3A need 1 <= window <= chunk and process
  * floor(chunk / window) tokens per block. Tensor-core products take the bf16
  * inputs as operands with fp32 accumulation and an fp32 state. FALCON_F32
@@ -197,7 +210,8 @@ FALCON_API falcon_status_t falcon_fwd_chunk_noalloc(const falcon_args_t *args, f
  * section Methodology in Plain English): the literal per-token recurrence
  * with an fp32 state and fp32 arithmetic. One CTA per (b, h) walks t = 1..T.
  * Supported: 1 <= dk, dv <= 128; window <= 64 for Falcon-3/3A; `chunk` is
- * ignored. Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ * ignored. This is the entry point for Falcon-2/2A (with n0 / n_out).
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
  */
 FALCON_API falcon_status_t falcon_fwd_recurrent(const falcon_args_t *args, falcon_stream_t stream);
 
@@ -216,7 +230,8 @@ FALCON_API falcon_status_t falcon_fwd_recurrent(const falcon_args_t *args, falco
  * place; q, k (N,H,dk), v (N,H,dv) io_dtype; alpha, eta (N,H) fp32;
  * o (N,H,dv) io_dtype is written. The buffers of one call must not overlap.
  * Supported: rule Falcon-1 or Falcon-1A (Falcon-3/3A need a window of past
- * pairs and return UNSUPPORTED); dk in {32, 64, 128}; 1 <= dv <= 256.
+ * pairs and Falcon-2/2A their column energies: both return UNSUPPORTED); dk in
+ * {32, 64, 128}; 1 <= dv <= 256.
  * Errors: INVALID_ARG, UNSUPPORTED, CUDA.
  */
 FALCON_API falcon_status_t falcon_decode_step(int rule, int io_dtype, int N, int H, int dk, int dv,

@@ -13,8 +13,10 @@ itself; see tests/test_oracle_pins.py):
                 orthonormal-key recall, Kaczmarz convergence, segment split.
   chunk      -- pinned: agrees with the recurrent form for every chunk size.
   masked     -- pinned: agrees with the recurrent form (one block of T steps).
+  backward   -- pinned: central finite differences of the recurrent form for every
+                input (tests/test_oracle_backward.py).
 """
 from .oracle import (  # noqa: F401
-    RULE_1, RULE_1A, RULE_3, RULE_3A,
-    build_oracle, oracle_lib_path, recurrent, chunk, masked, decode_step, max_threads,
+    RULE_1, RULE_1A, RULE_3, RULE_3A, RULE_2, RULE_2A, falcon2,
+    build_oracle, oracle_lib_path, recurrent, chunk, masked, decode_step, max_threads, backward,
 )

@@ -14,7 +14,7 @@ import threading
 
 import numpy as np
 
-RULE_1, RULE_1A, RULE_3, RULE_3A = 1, 2, 3, 4
+RULE_1, RULE_1A, RULE_3, RULE_3A, RULE_2, RULE_2A = 1, 2, 3, 4, 5, 6
 SAME_STEP = 0x100  # flag OR-ed into a rule: pair (k_t, v_t) at step t (same-step association)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -56,6 +56,11 @@ def _load():
             lib.falcon_oracle_chunk.restype = I
             lib.falcon_oracle_masked.argtypes = common + [D, D, D, D, D, I]
             lib.falcon_oracle_masked.restype = I
+            lib.falcon_oracle_backward.argtypes = common[:12] + [I, D, D, D, D, D, D, D, D, D, D, D, I]
+            lib.falcon_oracle_backward.restype = I
+            lib.falcon_oracle_f2.argtypes = [I, I, I, I, I, I, D, D, D, D, D, ctypes.c_double, I,
+                                             D, D, D, D, D, D, D, I]
+            lib.falcon_oracle_f2.restype = I
             lib.falcon_oracle_max_threads.argtypes = []
             lib.falcon_oracle_max_threads.restype = I
             _lib = lib
@@ -149,3 +154,44 @@ def decode_step(rule, S, k_prev, q, k, v, alpha, eta, eps, threads=None):
                              _d(v)[:, :, None, :], _d(alpha)[:, :, None], _d(eta)[:, :, None],
                              eps, 1, S0=S, k_prev=k_prev, threads=threads)
     return o[:, :, 0, :], S_new, kl
+
+
+def backward(rule, q, k, v, alpha, eta, eps, dO, dS_T=None, window=1, S0=None, k_prev=None, threads=None):
+    """Gradients of the recurrent form (reverse mode through the literal recurrence) for upstream
+    gradients dO (B,H,T,dv) of the outputs and dS_T (B,H,dv,dk) of the final state. Returns a dict
+    with dq, dk, dv, dalpha, deta, dS0 and dk_prev (None when k_prev is None)."""
+    lib = _load()
+    q, k, v, alpha, eta, S0, k_prev, (B, H, T, dk, dv) = _prep(q, k, v, alpha, eta, S0, k_prev)
+    dO = _d(dO)
+    dS_T = _d(dS_T)
+    assert dO.shape == (B, H, T, dv)
+    out = {"dq": np.zeros((B, H, T, dk)), "dk": np.zeros((B, H, T, dk)), "dv": np.zeros((B, H, T, dv)),
+           "dalpha": np.zeros((B, H, T)), "deta": np.zeros((B, H, T)), "dS0": np.zeros((B, H, dv, dk)),
+           "dk_prev": np.zeros((B, H, dk)) if k_prev is not None else None}
+    rc = lib.falcon_oracle_backward(int(rule), B, H, T, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                    _ptr(eta), float(eps), int(window), _ptr(S0), _ptr(k_prev), _ptr(dO),
+                                    _ptr(dS_T), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                                    _ptr(out["dalpha"]), _ptr(out["deta"]), _ptr(out["dS0"]),
+                                    _ptr(out["dk_prev"]), int(threads or max_threads()))
+    if rc != 0:
+        raise RuntimeError(f"oracle backward failed ({rc})")
+    return out
+
+
+def falcon2(rule, q, k, v, alpha, eta, eps, chunk=0, S0=None, k_prev=None, n0=None, threads=None):
+    """Falcon-2 / Falcon-2A (rule 5 / 6, optionally | SAME_STEP): chunk = 0 runs the literal
+    recurrence, chunk >= 1 the blocked form. Returns (o, S_out, k_last, n_out) as float64, n_out
+    being the running per-column key energies that a continuation starts from."""
+    lib = _load()
+    q, k, v, alpha, eta, S0, k_prev, (B, H, T, dk, dv) = _prep(q, k, v, alpha, eta, S0, k_prev)
+    n0 = _d(n0)
+    if n0 is not None:
+        assert n0.shape == (B, H, dk)
+    o, S, kl = _outs(B, H, T, dk, dv)
+    n_out = np.zeros((B, H, dk))
+    rc = lib.falcon_oracle_f2(int(rule), B, H, T, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(eta),
+                              float(eps), int(chunk), _ptr(S0), _ptr(k_prev), _ptr(n0), _ptr(o), _ptr(S),
+                              _ptr(kl), _ptr(n_out), int(threads or max_threads()))
+    if rc != 0:
+        raise RuntimeError(f"oracle falcon2 failed ({rc})")
+    return o, S, kl, n_out

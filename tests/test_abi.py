@@ -40,13 +40,23 @@ def test_library_exports_every_declared_symbol(L):
         assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
 
 
-def test_struct_layout_matches_header():
-    # ints: rule io_dtype B H T dk dv (28 B) -> pointers 8-aligned from offset 32
-    assert F.FalconArgs.q.offset == 32
-    assert F.FalconArgs.eps.offset == 72
-    assert F.FalconArgs.window.offset == 76 and F.FalconArgs.chunk.offset == 80
-    assert F.FalconArgs.S0.offset == 88
-    assert ctypes.sizeof(F.FalconArgs) == 128
+def test_struct_layout_matches_header(tmp_path):
+    """The binding's falcon_args_t mirror has the C compiler's offsets for every field of the
+    header's struct (a small C program compiled against include/falcon.h prints them)."""
+    import subprocess
+    fields = [name for name, _ in F.FalconArgs._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"falcon.h\"\nint main(void) {\n"
+                   + "".join(f'  printf("{f} %zu\\n", offsetof(falcon_args_t, {f}));\n' for f in fields)
+                   + '  printf("sizeof %zu\\n", sizeof(falcon_args_t));\n  return 0;\n}\n')
+    exe = tmp_path / "layout"
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    subprocess.run(["gcc", "-std=c99", "-I", inc, "-o", str(exe), str(src)], check=True)
+    got = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                        check=True).stdout.splitlines())
+    for f in fields:
+        assert getattr(F.FalconArgs, f).offset == int(got[f]), f
+    assert ctypes.sizeof(F.FalconArgs) == int(got["sizeof"])
 
 
 def test_status_strings(L):
@@ -82,6 +92,8 @@ def _args(**kw):
     (dict(dk=96), F.FALCON_ERR_UNSUPPORTED),
     (dict(dv=48), F.FALCON_ERR_UNSUPPORTED),
     (dict(io_dtype=0), F.FALCON_ERR_UNSUPPORTED),   # fp32 inputs: the recurrent form serves them
+    (dict(rule=5), F.FALCON_ERR_UNSUPPORTED),       # Falcon-2/2A run on the recurrent form
+    (dict(rule=6 | 0x100), F.FALCON_ERR_UNSUPPORTED),
     (dict(chunk=128), F.FALCON_ERR_UNSUPPORTED),
     (dict(chunk=8), F.FALCON_ERR_UNSUPPORTED),
     (dict(rule=3, window=65), F.FALCON_ERR_UNSUPPORTED),
