@@ -378,7 +378,9 @@ SegLayout seg_layout(long long heads, int nseg, int ptot) {
 
 SegPlan seg_plan(const ChunkParams &p, int num_sms) {
     SegPlan s;
-    if (p.regression || !chunk_ws_supported(p) || p.T % kPBlk != 0) return s;
+    // one pair per step only: the state pass writes each token's own pair (a window would need the
+    // pairs of the tokens before a piece as well)
+    if (p.regression || p.window != 1 || !chunk_ws_supported(p) || p.T % kPBlk != 0) return s;
     const long long heads = (long long)p.B * p.H;
     const int nblk = p.T / kPBlk;
     int best = 1;

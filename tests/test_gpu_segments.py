@@ -16,11 +16,12 @@ pytestmark = pytest.mark.gpu
 SS = 0x100
 
 
-def _ws_bytes(F, rule, B, H, T, d=128, chunk=64, io=torch.bfloat16):
+def _ws_bytes(F, rule, B, H, T, d=128, chunk=64, io=torch.bfloat16, window=1):
     z = lambda *s: torch.zeros(*s, dtype=io, device="cuda")
     zf = lambda *s: torch.zeros(*s, dtype=torch.float32, device="cuda")
     q, k, v = z(B, H, T, d), z(B, H, T, d), z(B, H, T, d)
-    args = F.make_args(q, k, v, zf(B, H, T), zf(B, H, T), rule=rule, chunk=chunk, o=z(B, H, T, d))
+    args = F.make_args(q, k, v, zf(B, H, T), zf(B, H, T), rule=rule, chunk=chunk, o=z(B, H, T, d),
+                       window=window)
     return F.falcon_workspace_size(args)
 
 
@@ -33,6 +34,17 @@ def test_split_is_chosen_only_where_it_applies(F):
     assert _ws_bytes(F, 2, 1, 2, 448) == 0                  # too short for two segments of 8 blocks
     assert _ws_bytes(F, 2, 1, 2, 4096, chunk=32) == 0       # not the 64-token tensor-core kernel
     assert _ws_bytes(F, 2, 1, sms, 4096) == 0               # one head per SM already
+    assert _ws_bytes(F, 4, 1, 2, 4096, window=4) == 0       # windowed inner-product rule: no split
+    assert _ws_bytes(F, 4, 1, 2, 4096, window=2) == 0
+
+
+@pytest.mark.parametrize("w", [2, 4])
+def test_windowed_inner_product_with_few_heads(F, w):
+    """Falcon-3A with few heads and a long sequence runs unsplit on the tensor-core kernel (the
+    state pass writes one pair per token, so the split does not apply to a window)."""
+    s = I.make_seq(4, 1, 2, 2048, 128, 128, seed=640 + w, io_dtype="bf16", window=w, with_state=True,
+                   with_kprev=True)
+    check(s, run_gpu(F, s, "chunk"), run_oracle(s), TOL_BF16)
 
 
 @pytest.mark.parametrize("T", [1024, 4096])
