@@ -106,8 +106,6 @@ enum {
     B_SCAL = 15,       // [4] decay scalars of slot c % 4 ready -> local, chain
     B_SCALFREE = 19,   // [4] chain done with scalar slot, outputs stored (8 warps) -> helpers
     B_EDONE = 23,      // (e') done (it still reads R'^T from TMEM) -> chain (before S overwrites it), outputs
-    B_SOLVED = 24,     // T of the block solved (fp32, local) -> helpers (T tiles)
-    B_TREAD = 25,      // helpers read T of the block -> local (the next solve may overwrite it)
     B_PRDY = 26,       // P~ ready -> MMA (B')
     B_TRDY = 27,       // T_f, T' (and the step sizes) ready -> MMA (A), (B')
     B_ABDONE = 28,     // (A), (B') done -> chain, local (T tiles free), helpers (P~ tile free)
@@ -385,6 +383,22 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         return ok;
     };
 
+    // V of block j (regression rules: loaded by the chain MMA warp, which sees the chain free a slot)
+    auto load_v = [&](int jv) {
+        if (lane == 0) {
+            uint8_t *dst = sm + oV + (jv & 1) * kVst;
+            uint64_t *fb = &bars[B_FULLV + (jv & 1)];
+            const int t0 = jv * TB;
+            tc::mbar_arrive_expect_tx(fb, kVst);
+#pragma unroll
+            for (int m = 0; m < W; ++m) {  // value rows t0 - m ..
+                tc::tma_load_3d(dst + m * TB * 128, &tmV, 0, t0 - m, bh, fb);
+                tc::tma_load_3d(dst + 8192 + m * TB * 128, &tmV, 64, t0 - m, bh, fb);
+            }
+        }
+        __syncwarp();
+    };
+
     if (warp == 0) {
         // ================================================================ feed: TMA loads and the
         // state-independent MMAs (a), (A), (B'), issued by the whole warp (one elected lane issues).
@@ -400,6 +414,19 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         int kx = 0, kv = 0;
         bool ok = true;
         for (int j = 0; j <= nblk + 1 && ok; ++j) {
+            // (a) first: it only needs its own slot (loaded in the previous iteration), so a slot that is
+            // still busy for a later load never holds back the Gram product of the block the solve wants next
+            const int ja = j - 1;   // (a) [X;Q] X^T -> G, P once the helpers prepared the block and the
+            if (ja >= 0 && ja < nblk) {  // G/P columns were read for the block before
+                if (!(ok = wait_all(B_XQRDY + ja % 3, (ja / 3) & 1) && (ja == 0 || wait_all(B_GPFREE, (ja - 1) & 1))))
+                    break;
+                tc::fence_after_sync();
+                const uint64_t d = dXQ0 + slot_off(ja % 3);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) tc::mma_bf16_elect(tbase + cGP, d + kmaj(ks), d + kmaj(ks), kIdN64, ks > 0);
+                tc::mma_commit_elect(&bars[B_ADONE]);
+                if (!REG) tc::mma_commit_elect(&bars[B_XQFREE + ja % 3]);   // one of the slot's two arrivals
+            }
             if (j < nblk) {
                 if (j == p.dbg_stall_block) break;  // test hook: this block is never loaded
                 if (j >= 3 && !(ok = wait_all(B_XQFREE + j % 3, ((j / 3) - 1) & 1))) break;
@@ -419,33 +446,11 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 __syncwarp();
                 kx = j + 1;
             }
-            const int jv = j - 1;
-            if (jv >= 0 && jv < nblk) {
+            const int jv = j - 1;   // inner-product rules: V of block j-1 (the local warps scale it in place)
+            if (!REG && jv >= 0 && jv < nblk) {
                 if (jv >= 2 && !(ok = wait_all(B_VFREE + (jv & 1), ((jv >> 1) - 1) & 1))) break;
-                if (lane == 0) {
-                    uint8_t *dst = sm + oV + (jv & 1) * kVst;
-                    uint64_t *fb = &bars[B_FULLV + (jv & 1)];
-                    const int t0 = jv * TB;
-                    tc::mbar_arrive_expect_tx(fb, kVst);
-#pragma unroll
-                    for (int m = 0; m < W; ++m) {  // value rows t0 - m ..
-                        tc::tma_load_3d(dst + m * TB * 128, &tmV, 0, t0 - m, bh, fb);
-                        tc::tma_load_3d(dst + 8192 + m * TB * 128, &tmV, 64, t0 - m, bh, fb);
-                    }
-                }
-                __syncwarp();
+                load_v(jv);
                 kv = jv + 1;
-            }
-            const int ja = j - 1;   // (a) [X;Q] X^T -> G, P once the helpers prepared the block and the
-            if (ja >= 0 && ja < nblk) {  // G/P columns were read for the block before
-                if (!(ok = wait_all(B_XQRDY + ja % 3, (ja / 3) & 1) && (ja == 0 || wait_all(B_GPFREE, (ja - 1) & 1))))
-                    break;
-                tc::fence_after_sync();
-                const uint64_t d = dXQ0 + slot_off(ja % 3);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) tc::mma_bf16_elect(tbase + cGP, d + kmaj(ks), d + kmaj(ks), kIdN64, ks > 0);
-                tc::mma_commit_elect(&bars[B_ADONE]);
-                if (!REG) tc::mma_commit_elect(&bars[B_XQFREE + ja % 3]);   // one of the slot's two arrivals
             }
             const int jb = j - 2;   // (A) A^T = X^T T_f and (B') B' = P~ T' into the AB columns, free once
             if (REG && jb >= 0 && jb < nblk) {  // the chain copied A^T, B' of the block before
@@ -518,6 +523,12 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 tc::mma_commit_elect(&bars[B_ABDONE]);       // diag(w) Y read: the tile may be rewritten
             }
         }
+        int kvr = 0;   // regression rules: V loads armed by this warp
+        if (REG) {
+            // (with the test hook, nothing at or after the stalled block is loaded, so that the armed loads
+            // are exactly blocks 0 .. kvr-1)
+            for (; kvr < 2 && kvr < nblk && (p.dbg_stall_block < 0 || kvr < p.dbg_stall_block); ++kvr) load_v(kvr);
+        }
         for (int c = 0; c < nblk && ok && REG; ++c) {
             const int s = c & 1, u = c % 3;
             // (b) S X^T (regression only) then S Q^T -> slot s, S (bf16) from TMEM; the chain starts
@@ -548,12 +559,21 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             for (int ks = 0; ks < 4; ++ks)
                 tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dBp + (uint64_t)(ks * 2), kIdN64, ks > 0);
             tc::mma_commit_elect(&bars[B_EDONE]);
+            // V of block c+2 into the slot the chain has just read (its arrivals follow R'^T)
+            if (c + 2 < nblk && (p.dbg_stall_block < 0 || c + 2 < p.dbg_stall_block)) {
+                if (!(ok = wait_all(B_VFREE + s, (c >> 1) & 1))) break;
+                load_v(c + 2);
+                kvr = c + 3;
+            }
         }
         if (!ok) *abort_flag = 1;
-        // drain every MMA issued by this warp
+        // drain every MMA issued by this warp and every V load it armed
         tc::mma_commit_elect(&bars[B_FINAL]);
         const volatile int no_abort = 0;
         tc::mbar_wait(&bars[B_FINAL], 0, &no_abort, kDrainBudget);
+        if (lane == 0)
+            for (int c = kvr - 2 < 0 ? 0 : kvr - 2; c < kvr; ++c)
+                tc::mbar_wait(&bars[B_FULLV + (c & 1)], (c >> 1) & 1, &no_abort, kDrainBudget);
         __syncwarp();
     } else if (warp < 4) {
         // ================================================================ helpers (64 threads)
@@ -696,46 +716,6 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             tc::fence_proxy_async();
             named_bar(1, 64);
             if (leader) mbar_arrive(&bars[B_PRDY]);
-            if (REG) {
-                // T_f = diag(2^(g_last - g)) T diag(beta) and T' = T diag(beta) (bf16, m-major order) from
-                // the solved T; the tiles are free since (A), (B') of block c-1 are done (waited above)
-                if (!(ok = role_wait(&bars[B_SOLVED], c & 1, leader, 1, 64))) break;
-                const int rr = ht;
-                const float fr = sc[128 + rr];
-#pragma unroll 2
-                for (int cc = 0; cc < 8; ++cc) {
-                    const int j0 = 8 * cc;
-                    float t8[8], f8[8];
-                    if (W > 1) {
-                        // T is in token-major order: row (rr % TB) W + rr / TB; the eight m-major columns
-                        // j0.. share m' = j0 / TB and take tokens j0 % TB + k, i.e. a stride of W
-                        const float *Trow = sTf + ((rr % TB) * W + rr / TB) * LDF + (j0 % TB) * W + j0 / TB;
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) t8[k] = Trow[k * W];
-                    } else {
-                        const float4 x0 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + j0);
-                        const float4 x1 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + j0 + 4);
-                        t8[0] = x0.x; t8[1] = x0.y; t8[2] = x0.z; t8[3] = x0.w;
-                        t8[4] = x1.x; t8[5] = x1.y; t8[6] = x1.z; t8[7] = x1.w;
-                    }
-                    const float4 b0 = *reinterpret_cast<const float4 *>(sc + j0);     // beta of the columns
-                    const float4 b1 = *reinterpret_cast<const float4 *>(sc + j0 + 4);
-                    const float bc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        t8[k] *= bc[k];
-                        f8[k] = fr * t8[k];
-                    }
-                    st_chunk8(sTP, tc::sw128_chunk(rr, cc), t8);
-                    st_chunk8(sTF, tc::sw128_chunk(rr, cc), f8);
-                }
-                tc::fence_proxy_async();
-                named_bar(1, 64);
-                if (leader) {
-                    mbar_arrive(&bars[B_TREAD]);
-                    mbar_arrive(&bars[B_TRDY]);
-                }
-            }
             // the block after next: its slot frees once (b) of block c-1 is done
             if (c + 2 < nblk && !(ok = prep(c + 2))) break;
         }
@@ -821,11 +801,9 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                     gd[4 * q + 2] = be * exp2f(fminf(gri - g4.z, 0.f));
                     gd[4 * q + 3] = be * exp2f(fminf(gri - g4.w, 0.f));
                 }
-                // Column blocks 0-1 here; rows 32-63 hand the raw G of column blocks 2-3 to the other
-                // two local warps through L itself (columns 32-63 of rows 0-31 lie above the diagonal).
                 float *Lr = sL + r * LDF;
 #pragma unroll
-                for (int jb = 0; jb < 2; ++jb) {
+                for (int jb = 0; jb < 4; ++jb) {
                     const float fac = be * exp2f(fminf(gri - g2[16 * jb + 15], 0.f));
                     const bool below = jb < rb;
 #pragma unroll
@@ -840,45 +818,9 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                             make_float4(w0 * v[j], w1 * v[j + 1], w2 * v[j + 2], w3 * v[j + 3]);
                     }
                 }
-                if (lw == 1) {
-#pragma unroll
-                    for (int j = 32; j < 64; j += 4)
-                        *reinterpret_cast<float4 *>(Lr + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-                }
               }
             }
             named_bar(2, 128);
-            if (REG && W == 1 && lw >= 2) {
-                // rows 32-63, column block jb = lw (16 columns): decay factors as above, in place on the
-                // raw G the warp of rows 32-63 left there; blocks above the diagonal are not needed
-                const int rr = 32 + lane, rbr = rr >> 4, jb = lw;
-                if (jb <= rbr) {
-                    const float *g2 = sc + 192, *cf = sCF + 64 * u4;
-                    const float gri = g2[rr], be = sc[rr];
-                    const float fac = be * exp2f(fminf(gri - g2[16 * jb + 15], 0.f));
-                    float *Lr = sL + rr * LDF + 16 * jb;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int j = 16 * jb + 4 * q;
-                        const float4 gg = *reinterpret_cast<const float4 *>(Lr + 4 * q);
-                        float w[4];
-                        if (jb < rbr) {
-                            const float4 c4 = *reinterpret_cast<const float4 *>(cf + j);
-                            w[0] = fac * c4.x; w[1] = fac * c4.y; w[2] = fac * c4.z; w[3] = fac * c4.w;
-                        } else {
-                            const float4 g4 = *reinterpret_cast<const float4 *>(g2 + j);
-                            w[0] = be * exp2f(fminf(gri - g4.x, 0.f));
-                            w[1] = be * exp2f(fminf(gri - g4.y, 0.f));
-                            w[2] = be * exp2f(fminf(gri - g4.z, 0.f));
-                            w[3] = be * exp2f(fminf(gri - g4.w, 0.f));
-                        }
-                        *reinterpret_cast<float4 *>(Lr + 4 * q) = make_float4(w[0] * gg.x, w[1] * gg.y, w[2] * gg.z, w[3] * gg.w);
-                    }
-                }
-                named_bar(2, 128);
-            } else if (REG && W == 1) {
-                named_bar(2, 128);
-            }
             if (!REG) {
                 // The scaled value tiles of block c (inner-product rules): diag(beta) Y in place in its V
                 // slot and diag(w) Y, w = beta 2^(g_last - g), into the T tile region, once V has landed and
@@ -911,10 +853,46 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 if (leader) mbar_arrive(&bars[B_TRDY]);
                 continue;
             }
-            // the previous block's T has been read into its bf16 tiles before this solve overwrites it
-            if (c >= 1 && !role_wait(&bars[B_TREAD], (c - 1) & 1, leader, 2, 128)) break;
-            solve_local(sL, sTf, lt, lw, lane);   // ends with the local warps' barrier
-            if (leader) mbar_arrive(&bars[B_SOLVED]);
+            solve_local(sL, sTf, lt, lw, lane);
+            // T_f = diag(2^(g_last - g)) T diag(beta), T' = T diag(beta) once (A), (B') of c-1 are done
+            if (c >= 1 && !role_wait(&bars[B_ABDONE], (c - 1) & 1, leader, 2, 128)) break;
+            {
+                const int rr = lt >> 1, ch0 = 4 * (lt & 1);
+                const float fr = sc[128 + rr];
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int j0 = 8 * (ch0 + cc);
+                    float t8[8], f8[8];
+                    if (REG && W > 1) {
+                        // T is in token-major order: row (rr % TB) W + rr / TB; the eight m-major columns
+                        // j0.. share m' = j0 / TB and take tokens j0 % TB + k, i.e. a stride of W
+                        const float *Trow = sTf + ((rr % TB) * W + rr / TB) * LDF + (j0 % TB) * W + j0 / TB;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) t8[k] = Trow[k * W];
+                    } else if (REG) {
+                        const float4 x0 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + j0);
+                        const float4 x1 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + j0 + 4);
+                        t8[0] = x0.x; t8[1] = x0.y; t8[2] = x0.z; t8[3] = x0.w;
+                        t8[4] = x1.x; t8[5] = x1.y; t8[6] = x1.z; t8[7] = x1.w;
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) t8[k] = (j0 + k == rr) ? 1.f : 0.f;
+                    }
+                    const float4 b0 = *reinterpret_cast<const float4 *>(sc + j0);     // beta of the columns
+                    const float4 b1 = *reinterpret_cast<const float4 *>(sc + j0 + 4);
+                    const float bc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        t8[k] *= bc[k];
+                        f8[k] = fr * t8[k];
+                    }
+                    st_chunk8(sTP, tc::sw128_chunk(rr, ch0 + cc), t8);
+                    st_chunk8(sTF, tc::sw128_chunk(rr, ch0 + cc), f8);
+                }
+            }
+            tc::fence_proxy_async();
+            named_bar(2, 128);
+            if (leader) mbar_arrive(&bars[B_TRDY]);
         }
     } else {
         // ================================================================ chain (256 threads)
