@@ -12,6 +12,10 @@
 //   R'^T = Y^T - (S X^T) diag(2^g)                          (regression; Y^T for inner product)
 //   O^T  = (S Q^T) diag(2^g) + R'^T B'^T,   S <- 2^g_last S + R'^T A.
 // For the inner-product rule T = I, so T_f and T' are diagonal and no solve runs.
+// The regression rules never form R'^T: with Z~ = (S X^T) diag(2^g) the products split into
+//   dS = Y^T A + (-Z~) A,   R'^T B'^T = Y^T B'^T + (-Z~) B'^T,
+// where the Y^T terms read the value tile straight from shared memory (an MN-major A operand)
+// and only -Z~ passes through the chain warps (fp32 -> bf16 in tensor memory).
 //
 // One CTA of 512 threads per (b, h); the state-independent work of later blocks
 // runs on other warps while the state chain of block c runs:
@@ -21,7 +25,8 @@
 //                 (a)  [X;Q] X^T -> G (lanes 0-63), P (lanes 64-127)
 //                 (A)  A^T = X^T T_f   and  (B')  B' = [P~; *] T'        (state independent)
 //                 (b)  [S X^T | S Q^T] with S (bf16) read from tensor memory
-//                 (e') R'^T B'^T   (f') dS = R'^T A   with R'^T (bf16) from tensor memory
+//                 Y^T A, then (f') dS += -Z~ A;  Y^T B'^T, then (e') += -Z~ B'^T
+//                 with -Z~ (bf16) from tensor memory
 //               The chain's groups go first; the state-independent ones of later blocks are issued
 //               right behind them, so they run while the chain warps work on the results.
 //   warps 2-3   helpers: x_1 patch, cumulative log2 decay and its tables; P~ = Gamma o P
@@ -29,7 +34,7 @@
 //   warps 4-7   local: step sizes from the key norms on the diagonal of G,
 //               L = diag(beta)(Gamma o G) (fp32) from TMEM lanes 0-63,
 //               T = (I + L)^-1 (fp32, tensor-core tf32 block products), T_f and T' in bf16
-//   warps 8-15  chain: A^T, B' from TMEM to shared memory; R'^T (bf16 into TMEM); the fp32
+//   warps 8-15  chain: A^T, B' from TMEM to shared memory; -Z~ (bf16 into TMEM); the fp32
 //               state S <- 2^g_last S + dS (in registers) and its bf16 copy in TMEM;
 //               O = 2^g o (Q S^T) + B' R' out
 // Every decay factor is 2^(g_i - g_j) with i >= j (never a quotient of
@@ -81,7 +86,7 @@ constexpr uint32_t kSmem = oBar + 512 + 1024;
 static_assert(kSmem <= 232448, "shared memory");
 
 // TMEM columns
-// GP | slot 0 | slot 1 | A^T, B' | S (bf16) then R'^T (bf16)
+// GP | slot 0 | slot 1 | A^T, B' | S (bf16) then -Z~ (bf16; R'^T for the inner-product rules' history)
 // Slot c & 1 holds [S X^T | S Q^T] of block c from (b); once the chain has read S X^T, (e') puts
 // R'^T B'^T in its place. dS of block c takes all of the other slot, free between the chain's read
 // of the outputs of block c-1 and (b) of block c+1.
@@ -93,30 +98,34 @@ constexpr uint32_t kIdAT = tc::idesc_bf16(128, 64, 1, 1);   // X^T (MN-major A) 
 constexpr uint32_t kIdBP = tc::idesc_bf16(128, 64, 0, 1);   // P~ (K-major A) x T' (MN-major B)
 constexpr uint32_t kIdVP = tc::idesc_bf16(128, 64, 1, 0);   // (diag(beta) Y)^T (MN-major A) x P~ (K-major B)
 constexpr uint32_t kIdVX = tc::idesc_bf16(128, 128, 1, 1);  // (diag(w) Y)^T (MN-major A) x X (MN-major B)
+constexpr uint32_t kIdVA = tc::idesc_bf16(128, 128, 1, 0);  // Y^T (MN-major A) x A (K-major B, the A^T tile)
 
 // barrier indices (arrival count 1 unless noted)
 enum {
     B_FULLXQ = 0,      // [3] TMA [X;Q] landed -> helpers
     B_XQFREE = 3,      // [3] (a), (A) done (feed warp) and (b) done (chain MMA warp): 2 arrivals -> producer
-    B_FULLV = 6,       // [2] TMA V landed -> chain
-    B_VFREE = 8,       // [2] chain read V (8 warps) -> producer
+    B_FULLV = 6,       // [2] TMA V landed -> MMAs (regression), local warps (inner product)
+    B_VFREE = 8,       // [2] the MMAs that read V are done -> producer
     B_XQRDY = 10,      // [3] helpers prepared the block -> MMA (a)
     B_ADONE = 13,      // (a) done -> helpers, local
     B_GPFREE = 14,     // G read (local warps 4, 5) and P read (helpers): 3 arrivals -> MMA (a) of the next block
     B_SCAL = 15,       // [4] decay scalars of slot c % 4 ready -> local, chain
     B_SCALFREE = 19,   // [4] chain done with scalar slot, outputs stored (8 warps) -> helpers
-    B_EDONE = 23,      // (e') done (it still reads R'^T from TMEM) -> chain (before S overwrites it), outputs
+    B_EDONE = 23,      // (e') done (it still reads -Z~ from TMEM) -> chain (before S overwrites it), outputs
+    B_SOLVED = 24,     // T of the block solved (fp32, local) -> helpers (T tiles)
+    B_TREAD = 25,      // helpers read T of the block -> local (the next solve may overwrite it)
     B_PRDY = 26,       // P~ ready -> MMA (B')
     B_TRDY = 27,       // T_f, T' (and the step sizes) ready -> MMA (A), (B')
     B_ABDONE = 28,     // (A), (B') done -> chain, local (T tiles free), helpers (P~ tile free)
     B_EARDY = 29,      // A^T, B' in shared memory (8 warps) -> MMA (e'), (f')
     B_BDONE = 30,      // (b) done -> chain
-    B_RT = 31,         // R'^T in TMEM (8 warps) -> MMA (e'), (f')
+    B_RT = 31,         // -Z~ in TMEM (8 warps) -> MMA (e'), (f')
     B_EFDONE = 32,     // (f') done: dS in TMEM -> chain
     B_FINAL0 = 33,     // drain of the feed warp's MMAs at exit
     B_SRDY = 34,       // S bf16 in TMEM, dS read, O of the previous block read (8 warps) -> MMA (b)
     B_FINAL = 35,      // drain of the chain MMA warp's MMAs at exit
-    B_COUNT = 36
+    B_OFREE = 36,      // outputs of the block read out of their slot (8 warps) -> MMA (Y^T A of the next block)
+    B_COUNT = 37
 };
 
 __device__ __forceinline__ void named_bar(int id, int n) {
@@ -146,6 +155,21 @@ __device__ __forceinline__ void st_chunk8(uint8_t *base, uint32_t off, const flo
     pk.z = pack_bf16x2(v8[4], v8[5]);
     pk.w = pack_bf16x2(v8[6], v8[7]);
     *reinterpret_cast<uint4 *>(base + off) = pk;
+}
+
+// v[OFF + lane] of a register array, by a five-level select tree on the lane's bits
+template <int OFF>
+__device__ __forceinline__ float pick_lane(const float (&v)[64], int lane) {
+    float t16[16], t8[8], t4[4], t2[2];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) t16[k] = (lane & 16) ? v[OFF + 16 + k] : v[OFF + k];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t8[k] = (lane & 8) ? t16[8 + k] : t16[k];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) t4[k] = (lane & 4) ? t8[4 + k] : t8[k];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) t2[k] = (lane & 2) ? t4[2 + k] : t4[k];
+    return (lane & 1) ? t2[1] : t2[0];
 }
 
 // ---- tf32 warp MMA for the 16 x 16 blocks of the triangular solve
@@ -315,11 +339,8 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i) {
-            // V slots: freed by the chain warps' reads (regression), or by the MMAs that read the scaled
-            // values (inner product)
-            const bool chain_arrivals = (REG && i >= B_VFREE && i < B_VFREE + 2) ||
-                                        (i >= B_SCALFREE && i < B_SCALFREE + 4) || i == B_EARDY || i == B_RT ||
-                                        i == B_SRDY;
+            const bool chain_arrivals = (i >= B_SCALFREE && i < B_SCALFREE + 4) || i == B_EARDY || i == B_RT ||
+                                        i == B_SRDY || i == B_OFREE;
             const bool two = i >= B_XQFREE && i < B_XQFREE + 3;
             tc::mbar_init(&bars[i], chain_arrivals ? kChainWarps : (i == B_GPFREE ? 3 : (two ? 2 : 1)));
         }
@@ -531,8 +552,8 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         }
         for (int c = 0; c < nblk && ok && REG; ++c) {
             const int s = c & 1, u = c % 3;
-            // (b) S X^T (regression only) then S Q^T -> slot s, S (bf16) from TMEM; the chain starts
-            // forming R'^T as soon as the first half is done. The [X;Q] slot must have landed (and the
+            // (b) S X^T then S Q^T -> slot s, S (bf16) from TMEM; the chain starts forming -Z~ as soon
+            // as the first half is done. The [X;Q] slot must have landed (and the
             // cached key be patched into block 0): the helpers' readiness of the block says both.
             if (!(ok = wait_all(B_SRDY, c & 1) && wait_all(B_XQRDY + u, (c / 3) & 1))) break;
             tc::fence_after_sync();
@@ -547,19 +568,33 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             for (int ks = 0; ks < 8; ++ks)
                 tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s + 64, tbase + cSR + 8 * ks, dQ + kmaj(ks), kIdN64, ks > 0);
             tc::mma_commit_elect(&bars[B_XQFREE + u]);   // (b) of the slot is done (the other arrival)
-            // (f') dS = R'^T A into slot s^1 first (the state update waits for it), then (e') R'^T B'^T
-            // over S X^T in slot s (the outputs wait for it); R'^T from TMEM
-            if (!(ok = wait_all(B_RT, c & 1) && wait_all(B_EARDY, c & 1))) break;
+            // The state-independent half of dS, Y^T A, into slot s^1 while the chain forms -Z~: A^T and B'
+            // in shared memory, V landed, and the outputs of block c-1 read out of that slot.
+            const uint64_t dY = tc::sdesc(tc::smem_u32(sm + oV + s * kVst), 8192, 1024);   // Y^T, MN-major A
+            if (!(ok = wait_all(B_EARDY, c & 1) && wait_all(B_FULLV + s, (c >> 1) & 1) &&
+                       (c == 0 || wait_all(B_OFREE, (c - 1) & 1))))
+                break;
             tc::fence_after_sync();
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                tc::mma_bf16_ts_elect(tbase + cSXO + 128 * (s ^ 1), tbase + cSR + 8 * ks, dAt + (uint64_t)(ks * 2), kIdN128, ks > 0);
+                tc::mma_bf16_elect(tbase + cSXO + 128 * (s ^ 1), dY + (uint64_t)(ks * 128), dAt + (uint64_t)(ks * 2), kIdVA, ks > 0);
+            // (f') dS += -Z~ A (the state update waits for it), then (e') Y^T B'^T - Z~ B'^T over S X^T in
+            // slot s (the outputs wait for it); -Z~ (bf16) from TMEM
+            if (!(ok = wait_all(B_RT, c & 1))) break;
+            tc::fence_after_sync();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                tc::mma_bf16_ts_elect(tbase + cSXO + 128 * (s ^ 1), tbase + cSR + 8 * ks, dAt + (uint64_t)(ks * 2), kIdN128, true);
             tc::mma_commit_elect(&bars[B_EFDONE]);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dBp + (uint64_t)(ks * 2), kIdN64, ks > 0);
+                tc::mma_bf16_elect(tbase + cSXO + 128 * s, dY + (uint64_t)(ks * 128), dBp + (uint64_t)(ks * 2), kIdVP, ks > 0);
+            tc::mma_commit_elect(&bars[B_VFREE + s]);    // Y read: the V slot may refill
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dBp + (uint64_t)(ks * 2), kIdN64, true);
             tc::mma_commit_elect(&bars[B_EDONE]);
-            // V of block c+2 into the slot the chain has just read (its arrivals follow R'^T)
+            // V of block c+2 into the slot block c has just been read from
             if (c + 2 < nblk && (p.dbg_stall_block < 0 || c + 2 < p.dbg_stall_block)) {
                 if (!(ok = wait_all(B_VFREE + s, (c >> 1) & 1))) break;
                 load_v(c + 2);
@@ -646,7 +681,6 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             ok = prep(1);
         }
         for (int c = 0; c < nblk && ok; ++c) {
-            const int u3 = c % 3;
             if (c + 2 < nblk) load_gates(c + 2);  // in flight while block c is handled
             const float *sc = sScal + (c % 4) * 256;
             if (!(ok = role_wait(&bars[B_ADONE], c & 1, leader, 1, 64))) break;
@@ -716,6 +750,46 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             tc::fence_proxy_async();
             named_bar(1, 64);
             if (leader) mbar_arrive(&bars[B_PRDY]);
+            if (REG) {
+                // T_f = diag(2^(g_last - g)) T diag(beta) and T' = T diag(beta) (bf16, m-major order) from
+                // the solved T; the tiles are free since (A), (B') of block c-1 are done (waited above)
+                if (!(ok = role_wait(&bars[B_SOLVED], c & 1, leader, 1, 64))) break;
+                const int rr = ht;
+                const float fr = sc[128 + rr];
+#pragma unroll 2
+                for (int cc = 0; cc < 8; ++cc) {
+                    const int j0 = 8 * cc;
+                    float t8[8], f8[8];
+                    if (W > 1) {
+                        // T is in token-major order: row (rr % TB) W + rr / TB; the eight m-major columns
+                        // j0.. share m' = j0 / TB and take tokens j0 % TB + k, i.e. a stride of W
+                        const float *Trow = sTf + ((rr % TB) * W + rr / TB) * LDF + (j0 % TB) * W + j0 / TB;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) t8[k] = Trow[k * W];
+                    } else {
+                        const float4 x0 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + j0);
+                        const float4 x1 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + j0 + 4);
+                        t8[0] = x0.x; t8[1] = x0.y; t8[2] = x0.z; t8[3] = x0.w;
+                        t8[4] = x1.x; t8[5] = x1.y; t8[6] = x1.z; t8[7] = x1.w;
+                    }
+                    const float4 b0 = *reinterpret_cast<const float4 *>(sc + j0);     // beta of the columns
+                    const float4 b1 = *reinterpret_cast<const float4 *>(sc + j0 + 4);
+                    const float bc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        t8[k] *= bc[k];
+                        f8[k] = fr * t8[k];
+                    }
+                    st_chunk8(sTP, tc::sw128_chunk(rr, cc), t8);
+                    st_chunk8(sTF, tc::sw128_chunk(rr, cc), f8);
+                }
+                tc::fence_proxy_async();
+                named_bar(1, 64);
+                if (leader) {
+                    mbar_arrive(&bars[B_TREAD]);
+                    mbar_arrive(&bars[B_TRDY]);
+                }
+            }
             // the block after next: its slot frees once (b) of block c-1 is done
             if (c + 2 < nblk && !(ok = prep(c + 2))) break;
         }
@@ -730,8 +804,9 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         float ge = (lw < 2 && rs < T) ? eta_h[rs] : 0.f;  // step-size gate of row r's token, one block ahead
         for (int c = 0; c < nblk; ++c) {
             const int u4 = c % 4;
+            // (a) of the block follows the helpers' readiness of it, which follows its decay scalars:
+            // ADONE alone says both
             if (!role_wait(&bars[B_ADONE], c & 1, leader, 2, 128)) break;
-            if (!role_wait(&bars[B_SCAL + u4], (c >> 2) & 1, leader, 2, 128)) break;
             tc::fence_after_sync();
             float *sc = sScal + u4 * 256;
             if (lw < 2) {                                   // G rows r = 0..63: step sizes, then L
@@ -749,10 +824,9 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_GPFREE]);
-                // ||x_r||^2 is the diagonal entry G[r][r]: column r = 32 lw + lane of this row
-                float nrm = 0.f;
-#pragma unroll
-                for (int j = 0; j < 32; ++j) nrm += (j == lane) ? (lw == 0 ? v[j] : v[32 + j]) : 0.f;
+                // ||x_r||^2 is the diagonal entry G[r][r] = v[32 lw + lane] (a warp-uniform branch on lw
+                // keeps v in registers)
+                float nrm = lw == 0 ? pick_lane<0>(v, lane) : pick_lane<32>(v, lane);
                 if (W > 1) {   // the token's window: rows m * TB + rs, m < W
                     sNrm[r] = nrm;
                     named_bar(3, 64);
@@ -853,46 +927,10 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 if (leader) mbar_arrive(&bars[B_TRDY]);
                 continue;
             }
-            solve_local(sL, sTf, lt, lw, lane);
-            // T_f = diag(2^(g_last - g)) T diag(beta), T' = T diag(beta) once (A), (B') of c-1 are done
-            if (c >= 1 && !role_wait(&bars[B_ABDONE], (c - 1) & 1, leader, 2, 128)) break;
-            {
-                const int rr = lt >> 1, ch0 = 4 * (lt & 1);
-                const float fr = sc[128 + rr];
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const int j0 = 8 * (ch0 + cc);
-                    float t8[8], f8[8];
-                    if (REG && W > 1) {
-                        // T is in token-major order: row (rr % TB) W + rr / TB; the eight m-major columns
-                        // j0.. share m' = j0 / TB and take tokens j0 % TB + k, i.e. a stride of W
-                        const float *Trow = sTf + ((rr % TB) * W + rr / TB) * LDF + (j0 % TB) * W + j0 / TB;
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) t8[k] = Trow[k * W];
-                    } else if (REG) {
-                        const float4 x0 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + j0);
-                        const float4 x1 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + j0 + 4);
-                        t8[0] = x0.x; t8[1] = x0.y; t8[2] = x0.z; t8[3] = x0.w;
-                        t8[4] = x1.x; t8[5] = x1.y; t8[6] = x1.z; t8[7] = x1.w;
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) t8[k] = (j0 + k == rr) ? 1.f : 0.f;
-                    }
-                    const float4 b0 = *reinterpret_cast<const float4 *>(sc + j0);     // beta of the columns
-                    const float4 b1 = *reinterpret_cast<const float4 *>(sc + j0 + 4);
-                    const float bc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        t8[k] *= bc[k];
-                        f8[k] = fr * t8[k];
-                    }
-                    st_chunk8(sTP, tc::sw128_chunk(rr, ch0 + cc), t8);
-                    st_chunk8(sTF, tc::sw128_chunk(rr, ch0 + cc), f8);
-                }
-            }
-            tc::fence_proxy_async();
-            named_bar(2, 128);
-            if (leader) mbar_arrive(&bars[B_TRDY]);
+            // the previous block's T has been read into its bf16 tiles before this solve overwrites it
+            if (c >= 1 && !role_wait(&bars[B_TREAD], (c - 1) & 1, leader, 2, 128)) break;
+            solve_local(sL, sTf, lt, lw, lane);   // ends with the local warps' barrier
+            if (leader) mbar_arrive(&bars[B_SOLVED]);
         }
     } else {
         // ================================================================ chain (256 threads)
@@ -900,11 +938,6 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         const int qd = warp & 3, hf = (warp - 8) >> 2;
         const int row = 32 * qd + lane;    // TMEM lane = value row (and key row d of A^T)
         const uint32_t tl = tbase + ((uint32_t)(32 * qd) << 16);
-        // V tile (token rows i, value columns): element (i, row) sits at vcol + voff[i & 7] + (i >> 3) * 1024
-        const uint32_t vcol = (row >> 6) * 8192 + (row & 7) * 2;
-        uint32_t voff[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) voff[k] = k * 128 + (((((row & 63) >> 3) ^ k)) << 4);
         float S[64];                       // fp32 state, row `row`, columns 64 hf ..
         auto store_S = [&]() {             // bf16 pairs of this thread's 64 columns -> TMEM A operand
             uint32_t pk[32];
@@ -996,43 +1029,32 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 store_out(c - 1);
                 tc::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[B_SCALFREE + (c - 1) % 4]);
+                if (lane == 0) {
+                    mbar_arrive(&bars[B_SCALFREE + (c - 1) % 4]);
+                    mbar_arrive(&bars[B_OFREE]);
+                }
             }
-            // R'^T = Y^T - SX diag(2^g) (regression) or Y^T (inner product), bf16 into TMEM
-            if (!(ok = (!REG || warp_wait(&bars[B_BDONE], c & 1)) && warp_wait(&bars[B_SCAL + u4], (c >> 2) & 1) &&
-                       warp_wait(&bars[B_FULLV + s], (c >> 1) & 1)))
-                break;
+            // -Z~ = -(S X^T) diag(2^g), bf16 into TMEM: with dS = Y^T A - Z~ A and E = Y^T B'^T - Z~ B'^T the
+            // values themselves only enter through the tensor cores
+            if (!(ok = warp_wait(&bars[B_BDONE], c & 1) && warp_wait(&bars[B_SCAL + u4], (c >> 2) & 1))) break;
             tc::fence_after_sync();
             {
-                const float *sc = sScal + u4 * 256;
-                const uint8_t *sV = sm + oV + s * kVst + vcol;
+                const float *dg = sScal + u4 * 256 + 64 + 32 * hf;   // 2^g of this thread's 32 rows
                 uint32_t pk[16];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {           // 16 rows at a time
-                    const int i0 = 32 * hf + 16 * hh;
-                    float x[16], dg[16];
-                    if (REG) {                             // scales first: their latency overlaps the TMEM load
+                for (int hh = 0; hh < 2; ++hh) {   // 16 rows at a time (the state stays in registers)
+                    float x[16];
+                    tc::tmem_ld16(tl + cSXO + 128 * s + 32 * hf + 16 * hh, x);
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            const float4 d4 = *reinterpret_cast<const float4 *>(sc + 64 + i0 + 4 * q4);
-                            dg[4 * q4] = d4.x; dg[4 * q4 + 1] = d4.y; dg[4 * q4 + 2] = d4.z; dg[4 * q4 + 3] = d4.w;
-                        }
-                        tc::tmem_ld16(tl + cSXO + 128 * s + i0, x);
-                    }
-#pragma unroll
-                    for (int j = 0; j < 16; j += 2) {
-                        const int i = i0 + j;              // token row of V: swizzle depends on i & 7 only
-                        const float y0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sV + voff[i & 7] + (i >> 3) * 1024));
-                        const float y1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sV + voff[(i + 1) & 7] + ((i + 1) >> 3) * 1024));
-                        const float r0 = REG ? y0 - dg[j] * x[j] : y0;
-                        const float r1 = REG ? y1 - dg[j + 1] * x[j + 1] : y1;
-                        pk[8 * hh + (j >> 1)] = pack_bf16x2(r0, r1);
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 d4 = *reinterpret_cast<const float4 *>(dg + 16 * hh + 4 * q4);
+                        pk[8 * hh + 2 * q4] = pack_bf16x2(-d4.x * x[4 * q4], -d4.y * x[4 * q4 + 1]);
+                        pk[8 * hh + 2 * q4 + 1] = pack_bf16x2(-d4.z * x[4 * q4 + 2], -d4.w * x[4 * q4 + 3]);
                     }
                 }
                 tc::tmem_st16(tl + cSR + 16 * hf, pk);
             }
             warp_arrive(&bars[B_RT]);
-            if (lane == 0) mbar_arrive(&bars[B_VFREE + s]);
             // state update: S <- 2^g_last S + dS, then its bf16 copy for (b) of the next block
             if (!(ok = warp_wait(&bars[B_EFDONE], c & 1))) break;
             tc::fence_after_sync();
@@ -1047,7 +1069,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                     for (int j = 0; j < 32; ++j) S[32 * hh + j] = dl * S[32 * hh + j] + v[j];
                 }
             }
-            // (e') still reads R'^T from the columns the bf16 state takes
+            // (e') still reads -Z~ from the columns the bf16 state takes
             if (!(ok = warp_wait(&bars[B_EDONE], c & 1))) break;
             store_S();
             warp_arrive(&bars[B_SRDY]);
