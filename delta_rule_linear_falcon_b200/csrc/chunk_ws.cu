@@ -21,19 +21,21 @@
 // runs on other warps while the state chain of block c runs:
 //   warp 0      TMA producer: [X;Q] of each block into a 3-slot ring (the solve runs two
 //               blocks ahead), V into a 2-slot ring
-//   warp 1      MMA issuer (one thread):
-//                 (a)  [X;Q] X^T -> G (lanes 0-63), P (lanes 64-127)
-//                 (A)  A^T = X^T T_f   and  (B')  B' = [P~; *] T'        (state independent)
+//   warp 1      inner-product rules: the MMA issuer of the chain ((b), E, dS below);
+//               regression rules: streams V into its ring as the chain frees the slots
+//   MMAs (one elected thread issues each group):
+//                 (a)  [X;Q] X^T -> G (lanes 0-63), P (lanes 64-127)                (warp 0)
+//                 (A)  A^T = X^T T_f   and  (B')  B' = [P~; *] T'        (state independent, warp 0)
 //                 (b)  [S X^T | S Q^T] with S (bf16) read from tensor memory
 //                 Y^T A, then (f') dS += -Z~ A;  Y^T B'^T, then (e') += -Z~ B'^T
-//                 with -Z~ (bf16) from tensor memory
-//               The chain's groups go first; the state-independent ones of later blocks are issued
-//               right behind them, so they run while the chain warps work on the results.
+//                 with -Z~ (bf16) from tensor memory          (regression rules: chain warp 8)
+//               The chain warps issue their own groups right after the named barrier that ends
+//               their tensor-memory writes, so only MMA completions cross an mbarrier.
 //   warps 2-3   helpers: x_1 patch, cumulative log2 decay and its tables; P~ = Gamma o P
-//               from TMEM lanes 64-127
+//               from TMEM lanes 64-127; T_f and T' in bf16 from the solved T
 //   warps 4-7   local: step sizes from the key norms on the diagonal of G,
 //               L = diag(beta)(Gamma o G) (fp32) from TMEM lanes 0-63,
-//               T = (I + L)^-1 (fp32, tensor-core tf32 block products), T_f and T' in bf16
+//               T = (I + L)^-1 (fp32, tensor-core tf32 block products)
 //   warps 8-15  chain: A^T, B' from TMEM to shared memory; -Z~ (bf16 into TMEM); the fp32
 //               state S <- 2^g_last S + dS (in registers) and its bf16 copy in TMEM;
 //               O = 2^g o (Q S^T) + B' R' out
@@ -124,7 +126,7 @@ enum {
     B_FINAL0 = 33,     // drain of the feed warp's MMAs at exit
     B_SRDY = 34,       // S bf16 in TMEM, dS read, O of the previous block read (8 warps) -> MMA (b)
     B_FINAL = 35,      // drain of the chain MMA warp's MMAs at exit
-    B_OFREE = 36,      // outputs of the block read out of their slot (8 warps) -> MMA (Y^T A of the next block)
+    B_SQDONE = 36,     // S Q^T done (it reads the bf16 state that -Z~ replaces) -> chain
     B_COUNT = 37
 };
 
@@ -340,7 +342,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i) {
             const bool chain_arrivals = (i >= B_SCALFREE && i < B_SCALFREE + 4) || i == B_EARDY || i == B_RT ||
-                                        i == B_SRDY || i == B_OFREE;
+                                        i == B_SRDY;
             const bool two = i >= B_XQFREE && i < B_XQFREE + 3;
             tc::mbar_init(&bars[i], chain_arrivals ? kChainWarps : (i == B_GPFREE ? 3 : (two ? 2 : 1)));
         }
@@ -550,62 +552,21 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             // are exactly blocks 0 .. kvr-1)
             for (; kvr < 2 && kvr < nblk && (p.dbg_stall_block < 0 || kvr < p.dbg_stall_block); ++kvr) load_v(kvr);
         }
-        for (int c = 0; c < nblk && ok && REG; ++c) {
-            const int s = c & 1, u = c % 3;
-            // (b) S X^T then S Q^T -> slot s, S (bf16) from TMEM; the chain starts forming -Z~ as soon
-            // as the first half is done. The [X;Q] slot must have landed (and the
-            // cached key be patched into block 0): the helpers' readiness of the block says both.
-            if (!(ok = wait_all(B_SRDY, c & 1) && wait_all(B_XQRDY + u, (c / 3) & 1))) break;
-            tc::fence_after_sync();
-            const uint64_t dX = dXQ0 + slot_off(u), dQ = dX + (8192 >> 4);   // X rows 0-63, Q rows 64-127
-            if (REG) {
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dX + kmaj(ks), kIdN64, ks > 0);
-                tc::mma_commit_elect(&bars[B_BDONE]);
-            }
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s + 64, tbase + cSR + 8 * ks, dQ + kmaj(ks), kIdN64, ks > 0);
-            tc::mma_commit_elect(&bars[B_XQFREE + u]);   // (b) of the slot is done (the other arrival)
-            // The state-independent half of dS, Y^T A, into slot s^1 while the chain forms -Z~: A^T and B'
-            // in shared memory, V landed, and the outputs of block c-1 read out of that slot.
-            const uint64_t dY = tc::sdesc(tc::smem_u32(sm + oV + s * kVst), 8192, 1024);   // Y^T, MN-major A
-            if (!(ok = wait_all(B_EARDY, c & 1) && wait_all(B_FULLV + s, (c >> 1) & 1) &&
-                       (c == 0 || wait_all(B_OFREE, (c - 1) & 1))))
-                break;
-            tc::fence_after_sync();
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                tc::mma_bf16_elect(tbase + cSXO + 128 * (s ^ 1), dY + (uint64_t)(ks * 128), dAt + (uint64_t)(ks * 2), kIdVA, ks > 0);
-            // (f') dS += -Z~ A (the state update waits for it), then (e') Y^T B'^T - Z~ B'^T over S X^T in
-            // slot s (the outputs wait for it); -Z~ (bf16) from TMEM
-            if (!(ok = wait_all(B_RT, c & 1))) break;
-            tc::fence_after_sync();
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                tc::mma_bf16_ts_elect(tbase + cSXO + 128 * (s ^ 1), tbase + cSR + 8 * ks, dAt + (uint64_t)(ks * 2), kIdN128, true);
-            tc::mma_commit_elect(&bars[B_EFDONE]);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                tc::mma_bf16_elect(tbase + cSXO + 128 * s, dY + (uint64_t)(ks * 128), dBp + (uint64_t)(ks * 2), kIdVP, ks > 0);
-            tc::mma_commit_elect(&bars[B_VFREE + s]);    // Y read: the V slot may refill
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dBp + (uint64_t)(ks * 2), kIdN64, true);
-            tc::mma_commit_elect(&bars[B_EDONE]);
-            // V of block c+2 into the slot block c has just been read from
-            if (c + 2 < nblk && (p.dbg_stall_block < 0 || c + 2 < p.dbg_stall_block)) {
-                if (!(ok = wait_all(B_VFREE + s, (c >> 1) & 1))) break;
-                load_v(c + 2);
-                kvr = c + 3;
-            }
+        // Regression rules: this warp only streams V; the chain warps issue their own MMAs and free a
+        // V slot once the products that read it are done.
+        for (int c = 0; c + 2 < nblk && ok && REG; ++c) {
+            if (p.dbg_stall_block >= 0 && c + 2 >= p.dbg_stall_block) break;
+            if (!(ok = wait_all(B_VFREE + (c & 1), (c >> 1) & 1))) break;
+            load_v(c + 2);
+            kvr = c + 3;
         }
         if (!ok) *abort_flag = 1;
         // drain every MMA issued by this warp and every V load it armed
-        tc::mma_commit_elect(&bars[B_FINAL]);
         const volatile int no_abort = 0;
-        tc::mbar_wait(&bars[B_FINAL], 0, &no_abort, kDrainBudget);
+        if (!REG) {
+            tc::mma_commit_elect(&bars[B_FINAL]);
+            tc::mbar_wait(&bars[B_FINAL], 0, &no_abort, kDrainBudget);
+        }
         if (lane == 0)
             for (int c = kvr - 2 < 0 ? 0 : kvr - 2; c < kvr; ++c)
                 tc::mbar_wait(&bars[B_FULLV + (c & 1)], (c >> 1) & 1, &no_abort, kDrainBudget);
@@ -756,17 +717,38 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 if (!(ok = role_wait(&bars[B_SOLVED], c & 1, leader, 1, 64))) break;
                 const int rr = ht;
                 const float fr = sc[128 + rr];
-#pragma unroll 2
+              if constexpr (W > 1) {
+                // T' row rr into registers (all reads before any store, so that their latencies overlap)
+                float tp[64];
+#pragma unroll
                 for (int cc = 0; cc < 8; ++cc) {
                     const int j0 = 8 * cc;
-                    float t8[8], f8[8];
-                    if (W > 1) {
+                    {
                         // T is in token-major order: row (rr % TB) W + rr / TB; the eight m-major columns
                         // j0.. share m' = j0 / TB and take tokens j0 % TB + k, i.e. a stride of W
                         const float *Trow = sTf + ((rr % TB) * W + rr / TB) * LDF + (j0 % TB) * W + j0 / TB;
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) t8[k] = Trow[k * W];
-                    } else {
+                        for (int k = 0; k < 8; ++k) tp[j0 + k] = Trow[k * W];
+                    }
+                    const float4 b0 = *reinterpret_cast<const float4 *>(sc + j0);     // beta of the columns
+                    const float4 b1 = *reinterpret_cast<const float4 *>(sc + j0 + 4);
+                    tp[j0] *= b0.x; tp[j0 + 1] *= b0.y; tp[j0 + 2] *= b0.z; tp[j0 + 3] *= b0.w;
+                    tp[j0 + 4] *= b1.x; tp[j0 + 5] *= b1.y; tp[j0 + 6] *= b1.z; tp[j0 + 7] *= b1.w;
+                }
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    float f8[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) f8[k] = fr * tp[8 * cc + k];
+                    st_chunk8(sTP, tc::sw128_chunk(rr, cc), tp + 8 * cc);
+                    st_chunk8(sTF, tc::sw128_chunk(rr, cc), f8);
+                }
+              } else {
+#pragma unroll 2
+                for (int cc = 0; cc < 8; ++cc) {
+                    const int j0 = 8 * cc;
+                    float t8[8], f8[8];
+                    {
                         const float4 x0 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + j0);
                         const float4 x1 = *reinterpret_cast<const float4 *>(sTf + rr * LDF + j0 + 4);
                         t8[0] = x0.x; t8[1] = x0.y; t8[2] = x0.z; t8[3] = x0.w;
@@ -783,6 +765,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                     st_chunk8(sTP, tc::sw128_chunk(rr, cc), t8);
                     st_chunk8(sTF, tc::sw128_chunk(rr, cc), f8);
                 }
+              }
                 tc::fence_proxy_async();
                 named_bar(1, 64);
                 if (leader) {
@@ -962,9 +945,15 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 const float dg[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
                 float v[8], w[8];
                 tc::tmem_ld8x2(tl + cSXO + 128 * (c & 1) + 64 + i0, tl + cSXO + 128 * (c & 1) + i0, v, w);
+                __nv_bfloat16 *oi = o + (size_t)i0 * D;
+                if (i0 + 8 <= nval) {              // whole group (every group but the sequence's last)
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    if (i0 + j < nval) o[(size_t)(i0 + j) * D] = __float2bfloat16_rn(dg[j] * v[j] + w[j]);
+                    for (int j = 0; j < 8; ++j) oi[j * D] = __float2bfloat16_rn(dg[j] * v[j] + w[j]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (i0 + j < nval) oi[j * D] = __float2bfloat16_rn(dg[j] * v[j] + w[j]);
+                }
             }
         };
         {
@@ -975,7 +964,8 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
             }
             store_S();
-            warp_arrive(&bars[B_SRDY]);
+            if (!REG) warp_arrive(&bars[B_SRDY]);
+            else tc::fence_before_sync();
         }
         bool ok = true;
         for (int c = 0; c < nblk && !REG; ++c) {
@@ -1005,11 +995,37 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 mbar_arrive(&bars[B_SCALFREE + u4]);
             }
         }
-        for (int c = 0; c < nblk && REG; ++c) {
-            const int s = c & 1, u4 = c % 4;
-            // A^T (rows d, columns i) and B' (rows i < 64) from TMEM to their shared-memory tiles
-            if (!(ok = warp_wait(&bars[B_ABDONE], c & 1))) break;
+        // Regression rules: the chain warps issue the state chain's MMAs themselves (warp 8, one elected
+        // lane), right after the named barrier that says their own TMEM writes are done; only the
+        // completions of MMAs are mbarrier handoffs. Every wait is taken by one thread for all 256 and
+        // its outcome shared through the barrier, so that a timeout unwinds all chain warps together.
+        const bool issuer = warp == 8;
+        auto chain_wait = [&](int b, uint32_t parity) -> bool {
+            const bool r = role_wait(&bars[b], parity, ct == 32, 4, 256);   // polled by a warp that does not issue
             tc::fence_after_sync();
+            return r;
+        };
+        const uint64_t dAtC = tc::sdesc(tc::smem_u32(sA), 16, 1024);          // A^T, K-major B of dS
+        const uint64_t dBpC = tc::sdesc(tc::smem_u32(sPB + 8192), 16, 1024);  // B', K-major B of E
+        for (int c = 0; c < nblk && REG; ++c) {
+            const int s = c & 1, u = c % 3, u4 = c % 4;
+            // (b) Z = S X^T then S Q^T -> slot s, S (bf16) from TMEM: the block's [X;Q] slot is ready (and
+            // so are its decay scalars), and every chain thread's bf16 state is in TMEM (barrier).
+            if (!(ok = chain_wait(B_XQRDY + u, (c / 3) & 1))) break;
+            if (issuer) {
+                const uint64_t dX = dXQ0 + slot_off(u), dQ = dX + (8192 >> 4);   // X rows 0-63, Q rows 64-127
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dX + kmaj(ks), kIdN64, ks > 0);
+                tc::mma_commit_elect(&bars[B_BDONE]);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s + 64, tbase + cSR + 8 * ks, dQ + kmaj(ks), kIdN64, ks > 0);
+                tc::mma_commit_elect(&bars[B_SQDONE]);
+                tc::mma_commit_elect(&bars[B_XQFREE + u]);   // (b) of the slot is done (the other arrival)
+            }
+            // A^T (rows d, columns i) and B' (rows i < 64) from TMEM to their shared-memory tiles
+            if (!(ok = chain_wait(B_ABDONE, c & 1))) break;
             {
                 float v[32];
                 tc::tmem_ld32(tl + cAB + 32 * hf, v);
@@ -1023,21 +1039,27 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 }
             }
             tc::fence_proxy_async();
-            warp_arrive(&bars[B_EARDY]);
-            // outputs of the previous block (off the chain; their columns take dS of this block)
+            warp_arrive(&bars[B_EARDY]);    // the AB columns may take (A), (B') of the next block
+            // outputs of the previous block (their columns take dS of this block)
             if (c >= 1) {
                 store_out(c - 1);
                 tc::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&bars[B_SCALFREE + (c - 1) % 4]);
-                    mbar_arrive(&bars[B_OFREE]);
-                }
+                if (lane == 0) mbar_arrive(&bars[B_SCALFREE + (c - 1) % 4]);
+            }
+            // Y^T A, the state-independent half of dS, into slot s^1 once V has landed (the barrier also
+            // says that A^T is in shared memory and the outputs of block c-1 are read out of the slot)
+            if (!(ok = chain_wait(B_FULLV + s, (c >> 1) & 1))) break;
+            const uint64_t dY = tc::sdesc(tc::smem_u32(sm + oV + s * kVst), 8192, 1024);   // Y^T, MN-major A
+            if (issuer) {
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16_elect(tbase + cSXO + 128 * (s ^ 1), dY + (uint64_t)(ks * 128), dAtC + (uint64_t)(ks * 2), kIdVA, ks > 0);
             }
             // -Z~ = -(S X^T) diag(2^g), bf16 into TMEM: with dS = Y^T A - Z~ A and E = Y^T B'^T - Z~ B'^T the
-            // values themselves only enter through the tensor cores
-            if (!(ok = warp_wait(&bars[B_BDONE], c & 1) && warp_wait(&bars[B_SCAL + u4], (c >> 2) & 1))) break;
-            tc::fence_after_sync();
+            // values themselves only enter through the tensor cores. It replaces the bf16 state, which
+            // S Q^T may still be reading.
+            if (!(ok = chain_wait(B_BDONE, c & 1))) break;
             {
                 const float *dg = sScal + u4 * 256 + 64 + 32 * hf;   // 2^g of this thread's 32 rows
                 uint32_t pk[16];
@@ -1052,12 +1074,29 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                         pk[8 * hh + 2 * q4 + 1] = pack_bf16x2(-d4.z * x[4 * q4 + 2], -d4.w * x[4 * q4 + 3]);
                     }
                 }
+                if (!(ok = chain_wait(B_SQDONE, c & 1))) break;
                 tc::tmem_st16(tl + cSR + 16 * hf, pk);
             }
-            warp_arrive(&bars[B_RT]);
+            tc::fence_before_sync();
+            // (f') dS += -Z~ A (the state update waits for it), then (e') Y^T B'^T - Z~ B'^T over S X^T in
+            // slot s (the outputs wait for it); -Z~ (bf16) from TMEM
+            if ((ok = !named_bar_or(4, 256, false)) && issuer) {
+                tc::fence_after_sync();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * (s ^ 1), tbase + cSR + 8 * ks, dAtC + (uint64_t)(ks * 2), kIdN128, true);
+                tc::mma_commit_elect(&bars[B_EFDONE]);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16_elect(tbase + cSXO + 128 * s, dY + (uint64_t)(ks * 128), dBpC + (uint64_t)(ks * 2), kIdVP, ks > 0);
+                tc::mma_commit_elect(&bars[B_VFREE + s]);    // Y read: the V slot may refill
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dBpC + (uint64_t)(ks * 2), kIdN64, true);
+                tc::mma_commit_elect(&bars[B_EDONE]);
+            }
             // state update: S <- 2^g_last S + dS, then its bf16 copy for (b) of the next block
-            if (!(ok = warp_wait(&bars[B_EFDONE], c & 1))) break;
-            tc::fence_after_sync();
+            if (!(ok = chain_wait(B_EFDONE, c & 1))) break;
             {
                 const float dl = exp2f(sGL[u4]);
                 const uint32_t cds = cSXO + 128 * (s ^ 1) + 64 * hf;
@@ -1070,9 +1109,16 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 }
             }
             // (e') still reads -Z~ from the columns the bf16 state takes
-            if (!(ok = warp_wait(&bars[B_EDONE], c & 1))) break;
+            if (!(ok = chain_wait(B_EDONE, c & 1))) break;
             store_S();
-            warp_arrive(&bars[B_SRDY]);
+            tc::fence_before_sync();
+        }
+        if (REG && issuer) {
+            // drain every MMA this warp issued (after a timeout some may still be in flight)
+            tc::mma_commit_elect(&bars[B_FINAL]);
+            const volatile int no_abort = 0;
+            tc::mbar_wait(&bars[B_FINAL], 0, &no_abort, kDrainBudget);
+            __syncwarp();
         }
         if (REG && ok && nblk > 0 && !*abort_flag) {
             store_out(nblk - 1);
