@@ -217,6 +217,68 @@ falcon_status_t falcon_fwd_recurrent(const falcon_args_t *a, falcon_stream_t str
                                                                                      : FALCON_ERR_CUDA;
 }
 
+namespace {
+
+// The forward arguments of a backward call (its outputs may be absent) and the backward limits.
+falcon_status_t check_bwd_args(const falcon_args_t *a) {
+    if (!a) return FALCON_ERR_INVALID_ARG;
+    falcon_args_t b = *a;
+    if (!b.o) b.o = const_cast<void *>(b.q);   // o is not read by the backward pass (only checked)
+    b.S_out = nullptr;
+    b.k_last = nullptr;
+    falcon_status_t st = check_seq_args(&b);
+    if (st != FALCON_OK) return st;
+    if (is_per_column(a->rule)) return FALCON_ERR_UNSUPPORTED;
+    if (a->dk > 128 || a->dv > 128) return FALCON_ERR_UNSUPPORTED;
+    const int w = is_windowed(a->rule) ? a->window : 1;
+    if (bwd_smem_bytes(a->dk, a->dv, w) > 232448) return FALCON_ERR_UNSUPPORTED;
+    return FALCON_OK;
+}
+
+}  // namespace
+
+size_t falcon_bwd_workspace_size(const falcon_args_t *a) {
+    if (check_bwd_args(a) != FALCON_OK) return 0;
+    if ((long long)a->B * a->H * a->T == 0) return 0;
+    return bwd_workspace_bytes(a->B, a->H, a->T, a->dk, a->dv, nullptr);
+}
+
+falcon_status_t falcon_bwd_recurrent(const falcon_args_t *a, const falcon_grads_t *g, void *workspace,
+                                     size_t workspace_bytes, falcon_stream_t stream) {
+    falcon_status_t st = check_bwd_args(a);
+    if (st != FALCON_OK) return st;
+    if (!g) return FALCON_ERR_INVALID_ARG;
+    const long long bh = (long long)a->B * a->H;
+    if (bh * a->T == 0) return FALCON_OK;
+    if (!g->dO || !g->dq || !g->dk || !g->dv || !g->dalpha || !g->deta) return FALCON_ERR_INVALID_ARG;
+    const void *ptrs[] = {g->dO, g->dS_T, g->dq, g->dk, g->dv, g->dalpha, g->deta, g->dS0, g->dk_prev};
+    for (const void *q : ptrs)
+        if (q && !aligned4(q)) return FALCON_ERR_INVALID_ARG;
+    int seg = 1;
+    const size_t need = bwd_workspace_bytes(a->B, a->H, a->T, a->dk, a->dv, &seg);
+    if (!workspace || workspace_bytes < need) return FALCON_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return FALCON_ERR_INVALID_ARG;
+
+    BwdParams p{};
+    p.B = a->B; p.H = a->H; p.T = a->T; p.dk = a->dk; p.dv = a->dv;
+    p.window = is_windowed(a->rule) ? a->window : 1;
+    p.seg = seg;
+    p.regression = is_regression(a->rule);
+    p.io_bf16 = a->io_dtype == FALCON_BF16;
+    p.same_step = same_step(a->rule);
+    p.q = a->q; p.k = a->k; p.v = a->v; p.k_prev = a->k_prev;
+    p.alpha = a->alpha; p.eta = a->eta; p.S0 = a->S0; p.eps = a->eps;
+    p.dO = g->dO; p.dS_T = g->dS_T;
+    p.dq = g->dq; p.dk_out = g->dk; p.dv_out = g->dv; p.dalpha = g->dalpha; p.deta = g->deta;
+    p.dS0 = g->dS0; p.dk_prev = g->dk_prev;
+    p.ws = static_cast<float *>(workspace);
+    int *err = nullptr;
+    int sms = 0;
+    if (!device_info(&err, &sms)) return FALCON_ERR_CUDA;
+    return launch_bwd_recurrent(p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? FALCON_OK
+                                                                                         : FALCON_ERR_CUDA;
+}
+
 falcon_status_t falcon_decode_step(int rule, int io_dtype, int N, int H, int dk, int dv, float *S,
                                    void *k_prev, const void *q, const void *k, const void *v,
                                    const float *alpha, const float *eta, float eps, void *o,

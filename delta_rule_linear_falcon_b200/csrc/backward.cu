@@ -1,0 +1,341 @@
+// backward.cu -- falcon_bwd_recurrent: gradients of the recurrent form (reverse mode
+// through the per-token recurrence of "Fast Weight Attention for Continual Learning",
+// authors' abstract; the pages give the forward rules only, so these are their
+// derivatives) for Falcon-1/1A/3/3A, with the same-step flag, an initial state and a
+// cached key. fp32 state and fp32 arithmetic; q, k, v in the I/O dtype, every gradient
+// in fp32.
+//
+// One CTA of 128 threads per (b, h). With U = dL/dS after step t (starting from dS_T),
+// step t (0-based, pairs j = t - m of window slot m, Sbar = alpha_t S_{t-1}) gives
+//   U += dO_t q_t^T,                       dq_t = S_t^T dO_t
+//   regression (r_m = Sbar x_m - y_m, S_t = Sbar - beta sum_m r_m x_m^T):
+//     dbeta = -sum_m r_m^T U x_m,   dr_m = -beta U x_m,   dy_m = -dr_m
+//     dx_m  = -beta U^T r_m + Sbar^T dr_m,   dSbar = U + sum_m dr_m x_m^T
+//   inner product (S_t = Sbar + beta sum_m y_m x_m^T):
+//     dbeta = sum_m y_m^T U x_m,   dy_m = beta U x_m,   dx_m = beta U^T y_m,   dSbar = U
+//   beta = eta_t / (N + eps), N = sum_m ||x_m||^2 (no gradient through it when N + eps = 0):
+//     deta_t = dbeta / (N + eps),   dx_m += -2 dbeta beta / (N + eps) x_m
+//   dalpha_t = <dSbar, S_{t-1}>,   U <- alpha_t dSbar
+// and dx_m, dy_m are scattered to the key and value rows of pair j (x_j = k_{j-1}, k_prev
+// for j = 0, or k_j with the same-step flag); dS0 is the last U.
+//
+// The states are not kept: a first forward pass stores S at the start of every segment of
+// C steps in the workspace, and the reverse sweep re-runs each segment forward from its
+// checkpoint into a buffer of C + 1 states before walking it backwards. U and the two
+// states a step needs (before and after it) sit in shared memory with rows padded to
+// d_k + 1 floats, so that a thread can walk a row (thread = value row i) or a column
+// (thread = key column c) without bank conflicts: row products (U x, Sbar x, the state
+// update) and column products (S^T dO, U^T r, Sbar^T dr) are both plain loops.
+#include <math.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace falcon {
+
+namespace {
+
+constexpr int kBwdThreads = 128;
+constexpr int kBwdWarps = kBwdThreads / 32;
+
+struct BwdSmem {
+    int LD, dk, dv, w;
+    // offsets in floats
+    size_t oU, oP, oA, oX, oY, oQ, oG, oUx, oR, oDr, oRed, total;
+};
+
+__host__ __device__ inline BwdSmem bwd_smem(int dk, int dv, int w) {
+    BwdSmem s;
+    s.LD = dk + 1; s.dk = dk; s.dv = dv; s.w = w;
+    const size_t mat = (size_t)dv * s.LD;
+    s.oU = 0; s.oP = mat; s.oA = 2 * mat;
+    s.oX = 3 * mat;
+    s.oY = s.oX + (size_t)w * dk;
+    s.oQ = s.oY + (size_t)w * dv;
+    s.oG = s.oQ + dk;
+    s.oUx = s.oG + dv;
+    s.oR = s.oUx + (size_t)w * dv;
+    s.oDr = s.oR + (size_t)w * dv;
+    s.oRed = s.oDr + (size_t)w * dv;
+    s.total = s.oRed + 2 * kBwdWarps + 4;
+    return s;
+}
+
+// Sum over the CTA; every thread gets the result. Two barriers.
+__device__ __forceinline__ float block_sum(float x, float *red) {
+    x = warp_sum(x);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();                 // earlier readers of red are done
+    if (lane == 0) red[warp] = x;
+    __syncthreads();
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < kBwdWarps; ++i) s += red[i];
+    return s;
+}
+
+template <typename IO>
+struct BwdCtx {
+    const BwdParams &p;
+    const IO *q, *k, *v, *kp;
+    const float *al, *et;
+    int T, dk, dv, w;
+    bool same;
+    // key row of pair j into dst (dk floats): k_{j-1}, k_prev for j = 0 (or 0), k_j with the flag
+    __device__ void pair_key(float *dst, long j) const {
+        const int tid = threadIdx.x;
+        const IO *src = nullptr;
+        size_t base = 0;
+        if (j >= 0) {
+            if (same) { src = k; base = (size_t)j * dk; }
+            else if (j >= 1) { src = k; base = (size_t)(j - 1) * dk; }
+            else if (kp) { src = kp; base = 0; }
+        }
+        for (int c = tid; c < dk; c += kBwdThreads) dst[c] = src ? Io<IO>::ld(src, base + c) : 0.f;
+    }
+    // stage the w pairs of step t (keys, values) into shared memory
+    __device__ void stage_pairs(float *sX, float *sY, long t) const {
+        const int tid = threadIdx.x;
+        for (int m = 0; m < w; ++m) {
+            pair_key(sX + (size_t)m * dk, t - m);
+            const long j = t - m;
+            for (int i = tid; i < dv; i += kBwdThreads)
+                sY[(size_t)m * dv + i] = j >= 0 ? Io<IO>::ld(v, (size_t)j * dv + i) : 0.f;
+        }
+    }
+};
+
+template <typename IO, bool REG>
+__global__ void __launch_bounds__(kBwdThreads)
+bwd_recurrent_kernel(BwdParams p) {
+    extern __shared__ __align__(16) float smem[];
+    const int dk = p.dk, dv = p.dv, w = p.window, T = p.T, C = p.seg;
+    const BwdSmem L = bwd_smem(dk, dv, w);
+    const int LD = L.LD;
+    float *sU = smem + L.oU, *sP = smem + L.oP, *sA = smem + L.oA;
+    float *sX = smem + L.oX, *sY = smem + L.oY, *sQ = smem + L.oQ, *sG = smem + L.oG;
+    float *sUx = smem + L.oUx, *sR = smem + L.oR, *sDr = smem + L.oDr, *sRed = smem + L.oRed;
+    const int tid = threadIdx.x;
+    const size_t bh = blockIdx.x;
+    const size_t DD = (size_t)dv * dk;
+
+    BwdCtx<IO> ctx{p,
+                   reinterpret_cast<const IO *>(p.q) + bh * T * dk,
+                   reinterpret_cast<const IO *>(p.k) + bh * T * dk,
+                   reinterpret_cast<const IO *>(p.v) + bh * T * dv,
+                   p.k_prev ? reinterpret_cast<const IO *>(p.k_prev) + bh * dk : nullptr,
+                   p.alpha + bh * T, p.eta + bh * T, T, dk, dv, w, p.same_step};
+    const IO *q = ctx.q;
+    const float *dO = p.dO + bh * T * dv;
+    float *gq = p.dq + bh * T * dk, *gk = p.dk_out + bh * T * dk, *gv = p.dv_out + bh * T * dv;
+    float *gal = p.dalpha + bh * T, *get = p.deta + bh * T;
+    float *gkp = (p.dk_prev && p.k_prev) ? p.dk_prev + bh * dk : nullptr;
+    const int nseg = (T + C - 1) / C;
+    float *ckpt = p.ws + bh * (size_t)(nseg + C + 1) * DD;   // nseg checkpoints, then C + 1 states
+    float *buf = ckpt + (size_t)nseg * DD;
+
+    // the key and value gradients accumulate over the w steps that read a pair
+    for (size_t e = tid; e < (size_t)T * dk; e += kBwdThreads) gk[e] = 0.f;
+    for (size_t e = tid; e < (size_t)T * dv; e += kBwdThreads) gv[e] = 0.f;
+    if (gkp)
+        for (int c = tid; c < dk; c += kBwdThreads) gkp[c] = 0.f;
+
+    auto store_state = [&](float *dst, const float *src) {   // padded shared rows -> dense dv x dk
+        for (size_t e = tid; e < DD; e += kBwdThreads) dst[e] = src[(e / dk) * LD + e % dk];
+    };
+    auto load_state = [&](float *dst, const float *src) {
+        for (size_t e = tid; e < DD; e += kBwdThreads) dst[(e / dk) * LD + e % dk] = src[e];
+    };
+    // beta of step t from the staged keys (every thread gets it) and its denominator
+    auto step_beta = [&](long t, float &beta, float &den) {
+        float part = 0.f;
+        for (int e = tid; e < w * dk; e += kBwdThreads) part += sX[e] * sX[e];
+        const float n = block_sum(part, sRed);
+        den = n + p.eps;
+        beta = den > 0.f ? ctx.et[t] / den : 0.f;
+    };
+    // one forward step on the state in sP (padded rows), in place
+    auto forward_step = [&](long t) {
+        __syncthreads();                   // sX / sY and sP are free
+        ctx.stage_pairs(sX, sY, t);
+        __syncthreads();
+        float beta, den;
+        step_beta(t, beta, den);
+        const float a = ctx.al[t];
+        for (int i = tid; i < dv; i += kBwdThreads) {
+            float *Si = sP + (size_t)i * LD;
+            for (int c = 0; c < dk; ++c) Si[c] *= a;
+            if (REG) {
+                for (int m = 0; m < w; ++m) {
+                    const float *x = sX + (size_t)m * dk;
+                    float r = -sY[(size_t)m * dv + i];
+                    for (int c = 0; c < dk; ++c) r = fmaf(Si[c], x[c], r);
+                    sR[(size_t)m * dv + i] = r;
+                }
+                for (int m = 0; m < w; ++m) {
+                    const float *x = sX + (size_t)m * dk;
+                    const float br = beta * sR[(size_t)m * dv + i];
+                    for (int c = 0; c < dk; ++c) Si[c] = fmaf(-br, x[c], Si[c]);
+                }
+            } else {
+                for (int m = 0; m < w; ++m) {
+                    const float *x = sX + (size_t)m * dk;
+                    const float by = beta * sY[(size_t)m * dv + i];
+                    for (int c = 0; c < dk; ++c) Si[c] = fmaf(by, x[c], Si[c]);
+                }
+            }
+        }
+    };
+
+    // ---- pass 1: checkpoints S_{s C}, s = 0 .. nseg-1
+    for (size_t e = tid; e < DD; e += kBwdThreads)
+        sP[(e / dk) * LD + e % dk] = p.S0 ? p.S0[bh * DD + e] : 0.f;
+    for (int s = 0; s < nseg; ++s) {
+        __syncthreads();
+        store_state(ckpt + (size_t)s * DD, sP);
+        if (s + 1 == nseg) break;
+        for (long t = (long)s * C; t < (long)(s + 1) * C; ++t) forward_step(t);
+    }
+
+    // ---- reverse sweep, segment by segment
+    for (size_t e = tid; e < DD; e += kBwdThreads)
+        sU[(e / dk) * LD + e % dk] = p.dS_T ? p.dS_T[bh * DD + e] : 0.f;
+    for (int s = nseg - 1; s >= 0; --s) {
+        const long t0 = (long)s * C, t1 = min((long)T, t0 + C);
+        __syncthreads();
+        load_state(sP, ckpt + (size_t)s * DD);
+        __syncthreads();
+        store_state(buf, sP);
+        for (long t = t0; t < t1; ++t) {
+            forward_step(t);
+            __syncthreads();
+            store_state(buf + (size_t)(t - t0 + 1) * DD, sP);
+        }
+        // sA = state after the last step of the segment
+        __syncthreads();
+        load_state(sA, buf + (size_t)(t1 - t0) * DD);
+        for (long t = t1 - 1; t >= t0; --t) {
+            __syncthreads();
+            load_state(sP, buf + (size_t)(t - t0) * DD);   // state before step t
+            ctx.stage_pairs(sX, sY, t);
+            for (int c = tid; c < dk; c += kBwdThreads) sQ[c] = Io<IO>::ld(q, (size_t)t * dk + c);
+            for (int i = tid; i < dv; i += kBwdThreads) sG[i] = dO[(size_t)t * dv + i];
+            __syncthreads();
+            float beta, den;
+            step_beta(t, beta, den);
+            const float a = ctx.al[t];
+            // rows: U += dO q^T; U x_m; residuals r_m at the decayed state
+            float part = 0.f;
+            for (int i = tid; i < dv; i += kBwdThreads) {
+                float *Ui = sU + (size_t)i * LD;
+                const float *Pi = sP + (size_t)i * LD;
+                const float g = sG[i];
+                for (int c = 0; c < dk; ++c) Ui[c] = fmaf(g, sQ[c], Ui[c]);
+                for (int m = 0; m < w; ++m) {
+                    const float *x = sX + (size_t)m * dk;
+                    float ux = 0.f, sx = 0.f;
+                    for (int c = 0; c < dk; ++c) {
+                        ux = fmaf(Ui[c], x[c], ux);
+                        sx = fmaf(Pi[c], x[c], sx);
+                    }
+                    sUx[(size_t)m * dv + i] = ux;
+                    if (REG) {
+                        const float r = a * sx - sY[(size_t)m * dv + i];
+                        sR[(size_t)m * dv + i] = r;
+                        part -= r * ux;
+                    } else {
+                        part += sY[(size_t)m * dv + i] * ux;
+                    }
+                }
+            }
+            const float dbeta = block_sum(part, sRed);
+            const bool has_den = den > 0.f;
+            const float dN = has_den ? -dbeta * beta / den : 0.f;
+            if (tid == 0) get[t] = has_den ? dbeta / den : 0.f;
+            // rows: dr_m, dy_m (scattered to the value row of pair j)
+            for (int i = tid; i < dv; i += kBwdThreads) {
+                for (int m = 0; m < w; ++m) {
+                    const float ux = sUx[(size_t)m * dv + i];
+                    if (REG) sDr[(size_t)m * dv + i] = -beta * ux;
+                    const long j = t - m;
+                    if (j >= 0) gv[(size_t)j * dv + i] += beta * ux;   // dy = -dr (regression) = beta U x
+                }
+            }
+            __syncthreads();
+            // columns: dq_t = S_t^T dO_t; dx_m (scattered to the key row of pair j)
+            for (int c = tid; c < dk; c += kBwdThreads) {
+                float acc = 0.f;
+                for (int i = 0; i < dv; ++i) acc = fmaf(sA[(size_t)i * LD + c], sG[i], acc);
+                gq[(size_t)t * dk + c] = acc;
+                for (int m = 0; m < w; ++m) {
+                    float dx = 0.f;
+                    if (REG) {
+                        const float *r = sR + (size_t)m * dv, *dr = sDr + (size_t)m * dv;
+                        for (int i = 0; i < dv; ++i) {
+                            dx = fmaf(-beta * sU[(size_t)i * LD + c], r[i], dx);
+                            dx = fmaf(a * sP[(size_t)i * LD + c], dr[i], dx);
+                        }
+                    } else {
+                        const float *y = sY + (size_t)m * dv;
+                        for (int i = 0; i < dv; ++i) dx = fmaf(beta * sU[(size_t)i * LD + c], y[i], dx);
+                    }
+                    dx = fmaf(2.f * dN, sX[(size_t)m * dk + c], dx);
+                    const long j = t - m;
+                    if (j < 0) continue;
+                    if (ctx.same) gk[(size_t)j * dk + c] += dx;
+                    else if (j >= 1) gk[(size_t)(j - 1) * dk + c] += dx;
+                    else if (gkp) gkp[c] += dx;
+                }
+            }
+            __syncthreads();
+            // rows: dSbar = U + sum_m dr_m x_m^T; dalpha = <dSbar, S_{t-1}>; U <- alpha dSbar
+            part = 0.f;
+            for (int i = tid; i < dv; i += kBwdThreads) {
+                float *Ui = sU + (size_t)i * LD;
+                const float *Pi = sP + (size_t)i * LD;
+                for (int c = 0; c < dk; ++c) {
+                    float d = Ui[c];
+                    if (REG)
+                        for (int m = 0; m < w; ++m) d = fmaf(sDr[(size_t)m * dv + i], sX[(size_t)m * dk + c], d);
+                    part = fmaf(d, Pi[c], part);
+                    Ui[c] = a * d;
+                }
+            }
+            const float dal = block_sum(part, sRed);
+            if (tid == 0) gal[t] = dal;
+            // the state before step t is the state after step t - 1
+            float *tmp = sA; sA = sP; sP = tmp;
+        }
+    }
+    __syncthreads();
+    if (p.dS0)
+        for (size_t e = tid; e < DD; e += kBwdThreads) p.dS0[bh * DD + e] = sU[(e / dk) * LD + e % dk];
+}
+
+}  // namespace
+
+size_t bwd_workspace_bytes(int B, int H, int T, int dk, int dv, int *seg_out) {
+    int C = (int)ceil(sqrt((double)(T > 0 ? T : 1)));
+    if (C < 1) C = 1;
+    const long long nseg = (T + C - 1) / C;
+    if (seg_out) *seg_out = C;
+    return (size_t)B * H * (size_t)(nseg + C + 1) * dv * dk * sizeof(float);
+}
+
+size_t bwd_smem_bytes(int dk, int dv, int w) { return bwd_smem(dk, dv, w).total * sizeof(float); }
+
+cudaError_t launch_bwd_recurrent(const BwdParams &p, cudaStream_t s) {
+    const size_t smem = bwd_smem_bytes(p.dk, p.dv, p.window);
+    auto pick = [&](auto kern) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<(unsigned)((long long)p.B * p.H), kBwdThreads, smem, s>>>(p);
+        return cudaGetLastError();
+    };
+    if (p.io_bf16)
+        return p.regression ? pick(bwd_recurrent_kernel<__nv_bfloat16, true>)
+                            : pick(bwd_recurrent_kernel<__nv_bfloat16, false>);
+    return p.regression ? pick(bwd_recurrent_kernel<float, true>) : pick(bwd_recurrent_kernel<float, false>);
+}
+
+}  // namespace falcon

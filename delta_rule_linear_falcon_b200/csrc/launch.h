@@ -22,6 +22,18 @@ struct RecParams {
     int *err;
 };
 
+struct BwdParams {
+    int B, H, T, dk, dv, window;  // window = 1 for Falcon-1/1A
+    int seg;                      // steps per checkpointed segment
+    bool regression, io_bf16, same_step;
+    const void *q, *k, *v, *k_prev;
+    const float *alpha, *eta, *S0;
+    float eps;
+    const float *dO, *dS_T;
+    float *dq, *dk_out, *dv_out, *dalpha, *deta, *dS0, *dk_prev;
+    float *ws;                    // per head: checkpoints, then one segment of states
+};
+
 struct DecodeParams {
     int N, H, dk, dv;
     bool regression, io_bf16;
@@ -60,6 +72,9 @@ constexpr long long kDefaultWaitBudget = 1ll << 31;  // SM clocks, about 1 s
 size_t recurrent_smem_bytes(int dk, int dv, int window);
 cudaError_t launch_recurrent(const RecParams &p, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, cudaStream_t s);
+size_t bwd_workspace_bytes(int B, int H, int T, int dk, int dv, int *seg_out);
+size_t bwd_smem_bytes(int dk, int dv, int window);
+cudaError_t launch_bwd_recurrent(const BwdParams &p, cudaStream_t s);
 cudaError_t launch_chunk(const ChunkParams &p, int num_sms, cudaStream_t s);
 // Warp-specialised tcgen05 / TMA kernel: d_k = d_v = 128, bf16 I/O, one pair per step, 64-token blocks.
 bool chunk_ws_supported(const ChunkParams &p);

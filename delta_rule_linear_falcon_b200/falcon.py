@@ -47,6 +47,16 @@ class FalconArgs(ctypes.Structure):
     ]
 
 
+class FalconGrads(ctypes.Structure):
+    """Mirror of falcon_grads_t."""
+    _fields_ = [
+        ("dO", ctypes.c_void_p), ("dS_T", ctypes.c_void_p),
+        ("dq", ctypes.c_void_p), ("dk", ctypes.c_void_p), ("dv", ctypes.c_void_p),
+        ("dalpha", ctypes.c_void_p), ("deta", ctypes.c_void_p),
+        ("dS0", ctypes.c_void_p), ("dk_prev", ctypes.c_void_p),
+    ]
+
+
 _lib = None
 _lock = threading.Lock()
 
@@ -68,6 +78,10 @@ def lib() -> ctypes.CDLL:
             L.falcon_fwd_chunk.restype = i
             L.falcon_fwd_recurrent.argtypes = [P, vp]
             L.falcon_fwd_recurrent.restype = i
+            L.falcon_bwd_workspace_size.argtypes = [P]
+            L.falcon_bwd_workspace_size.restype = ctypes.c_size_t
+            L.falcon_bwd_recurrent.argtypes = [P, ctypes.POINTER(FalconGrads), vp, ctypes.c_size_t, vp]
+            L.falcon_bwd_recurrent.restype = i
             L.falcon_decode_step.argtypes = [i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, vp, f, vp, vp]
             L.falcon_decode_step.restype = i
             L.falcon_status_string.argtypes = [i]
@@ -204,6 +218,45 @@ def falcon_fwd_recurrent(q, k, v, alpha, eta, *, rule, eps=1e-6, window=1, S0=No
     if st != FALCON_OK:
         raise FalconError(st, "falcon_fwd_recurrent")
     return o, S_out, k_last
+
+
+def falcon_bwd_workspace_size(args: FalconArgs) -> int:
+    return int(lib().falcon_bwd_workspace_size(ctypes.byref(args)))
+
+
+def falcon_bwd_recurrent(q, k, v, alpha, eta, dO, *, rule, eps=1e-6, window=1, S0=None, k_prev=None,
+                         dS_T=None, want_dS0=True, workspace=None, stream=None):
+    """Gradients of the recurrent form for upstream gradients dO (B, H, T, dv) fp32 of the
+    outputs and dS_T (B, H, dv, dk) fp32 (or None) of the final state. Returns a dict of fp32
+    tensors dq, dk, dv, dalpha, deta, dS0 (None unless want_dS0) and dk_prev (None without
+    k_prev). ``workspace``: a CUDA tensor of at least falcon_bwd_workspace_size(args) bytes, or
+    None to allocate one here for the call."""
+    B, H, T, dk = k.shape
+    dv = v.shape[-1]
+    dev = k.device
+    f32 = torch.float32
+    _need(dO, "dO", f32)
+    _need(dS_T, "dS_T", f32)
+    out = {"dq": torch.empty((B, H, T, dk), dtype=f32, device=dev),
+           "dk": torch.empty((B, H, T, dk), dtype=f32, device=dev),
+           "dv": torch.empty((B, H, T, dv), dtype=f32, device=dev),
+           "dalpha": torch.empty((B, H, T), dtype=f32, device=dev),
+           "deta": torch.empty((B, H, T), dtype=f32, device=dev),
+           "dS0": torch.empty((B, H, dv, dk), dtype=f32, device=dev) if want_dS0 else None,
+           "dk_prev": torch.empty((B, H, dk), dtype=f32, device=dev) if k_prev is not None else None}
+    args = make_args(q, k, v, alpha, eta, rule=rule, eps=eps, window=window, chunk=64, S0=S0, k_prev=k_prev)
+    grads = FalconGrads(dO.data_ptr(), _ptr(dS_T), out["dq"].data_ptr(), out["dk"].data_ptr(),
+                        out["dv"].data_ptr(), out["dalpha"].data_ptr(), out["deta"].data_ptr(),
+                        _ptr(out["dS0"]), _ptr(out["dk_prev"]))
+    need = falcon_bwd_workspace_size(args)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib().falcon_bwd_recurrent(ctypes.byref(args), ctypes.byref(grads), ws_ptr, ws_bytes, _stream(stream))
+    if st != FALCON_OK:
+        raise FalconError(st, "falcon_bwd_recurrent")
+    return out
 
 
 def falcon_decode_step(S, k_prev, q, k, v, alpha, eta, *, rule="falcon1", eps=1e-6, o=None,

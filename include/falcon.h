@@ -216,6 +216,50 @@ FALCON_API falcon_status_t falcon_fwd_chunk_noalloc(const falcon_args_t *args, f
 FALCON_API falcon_status_t falcon_fwd_recurrent(const falcon_args_t *args, falcon_stream_t stream);
 
 /*
+ * falcon_bwd_recurrent -- gradients of the recurrent form for a loss L, given the
+ * upstream gradients of the outputs and of the final state. The pages define the
+ * forward rules only (authors' abstract); these are their derivatives, taken step by
+ * step backwards through the same per-token recurrence (reverse mode):
+ *   U = dL/dS_t (U = dS_T after the last step), then for t = T..1:
+ *   U += dO_t q_t^T;  dq_t = S_t^T dO_t;
+ *   Falcon-1/3 (r_j = Sbar x_j - y_j):  dbeta = -sum_j r_j^T U x_j;
+ *     dy_j = beta U x_j;  dx_j = -beta U^T r_j - beta Sbar^T U x_j;  dSbar = U - beta sum_j U x_j x_j^T
+ *   Falcon-1A/3A:  dbeta = sum_j y_j^T U x_j;  dy_j = beta U x_j;  dx_j = beta U^T y_j;  dSbar = U
+ *   deta_t = dbeta / (N_t + eps);  dx_j += -2 dbeta beta / (N_t + eps) x_j  (N_t the pairs' squared norms;
+ *   nothing flows through beta when N_t + eps = 0);  dalpha_t = <dSbar, S_{t-1}>;  U <- alpha_t dSbar.
+ * dx of pair j goes to the key row it was read from (k_{j-1}; k_prev for the first pair, or k_j with
+ * FALCON_SAME_STEP), dy to v_j, and dS0 is the final U.
+ *
+ * `args` is the forward call's (q, k, v, alpha, eta, eps, window, S0, k_prev, rule with the
+ * flag); its outputs o, S_out, k_last and chunk are ignored. `grads` (every array fp32, dense,
+ * device memory; 4-byte alignment):
+ *   dO (B,H,T,dv) required; dS_T (B,H,dv,dk) or NULL (zero);
+ *   dq, dk (B,H,T,dk), dv (B,H,T,dv), dalpha, deta (B,H,T) written;
+ *   dS0 (B,H,dv,dk) written when not NULL; dk_prev (B,H,dk) written when not NULL and
+ *   args->k_prev is given.
+ * Workspace: falcon_bwd_workspace_size(args) bytes, 16-byte aligned (the states at the
+ * start of every segment of about sqrt(T) steps and one segment of recomputed states,
+ * fp32, per head). fp32 state and arithmetic; one CTA per (b, h).
+ * Supported: Falcon-1, 1A, 3, 3A (with or without FALCON_SAME_STEP); 1 <= dk, dv <= 128;
+ * windows whose staging fits in shared memory (w <= 8 at dk = dv = 128). Falcon-2/2A return
+ * UNSUPPORTED.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+typedef struct {
+    const float *dO;
+    const float *dS_T;
+    float *dq, *dk, *dv;
+    float *dalpha, *deta;
+    float *dS0;
+    float *dk_prev;
+} falcon_grads_t;
+
+FALCON_API size_t falcon_bwd_workspace_size(const falcon_args_t *args);
+FALCON_API falcon_status_t falcon_bwd_recurrent(const falcon_args_t *args, const falcon_grads_t *grads,
+                                                void *workspace, size_t workspace_bytes,
+                                                falcon_stream_t stream);
+
+/*
  * falcon_decode_step -- one token of the recurrence for N independent
  * sequences x H heads, in place: the recurrent form applied to a single step,
  * the incremental state update that the ai.info overview of "Fast Weight

@@ -40,23 +40,24 @@ def test_library_exports_every_declared_symbol(L):
         assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
 
 
-def test_struct_layout_matches_header(tmp_path):
-    """The binding's falcon_args_t mirror has the C compiler's offsets for every field of the
-    header's struct (a small C program compiled against include/falcon.h prints them)."""
+@pytest.mark.parametrize("mirror,ctype", [(F.FalconArgs, "falcon_args_t"), (F.FalconGrads, "falcon_grads_t")])
+def test_struct_layout_matches_header(tmp_path, mirror, ctype):
+    """The binding's struct mirrors have the C compiler's offsets for every field of the
+    header's structs (a small C program compiled against include/falcon.h prints them)."""
     import subprocess
-    fields = [name for name, _ in F.FalconArgs._fields_]
+    fields = [name for name, _ in mirror._fields_]
     src = tmp_path / "layout.c"
     src.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"falcon.h\"\nint main(void) {\n"
-                   + "".join(f'  printf("{f} %zu\\n", offsetof(falcon_args_t, {f}));\n' for f in fields)
-                   + '  printf("sizeof %zu\\n", sizeof(falcon_args_t));\n  return 0;\n}\n')
+                   + "".join(f'  printf("{f} %zu\\n", offsetof({ctype}, {f}));\n' for f in fields)
+                   + f'  printf("sizeof %zu\\n", sizeof({ctype}));\n  return 0;\n}}\n')
     exe = tmp_path / "layout"
     inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
     subprocess.run(["gcc", "-std=c99", "-I", inc, "-o", str(exe), str(src)], check=True)
     got = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True, text=True,
                                                         check=True).stdout.splitlines())
     for f in fields:
-        assert getattr(F.FalconArgs, f).offset == int(got[f]), f
-    assert ctypes.sizeof(F.FalconArgs) == int(got["sizeof"])
+        assert getattr(mirror, f).offset == int(got[f]), f
+    assert ctypes.sizeof(mirror) == int(got["sizeof"])
 
 
 def test_status_strings(L):
@@ -143,6 +144,54 @@ def test_decode_rejects_bad_arguments_on_host(L, kw, expect):
     assert _dec(L, **kw) == expect
 
 
+def _grads(**kw):
+    base = dict(dO=0x10000, dS_T=None, dq=0x11000, dk=0x12000, dv=0x13000, dalpha=0x14000,
+                deta=0x15000, dS0=None, dk_prev=None)
+    base.update(kw)
+    return F.FalconGrads(**base)
+
+
+@pytest.mark.parametrize("akw,gkw,ws,expect", [
+    (dict(rule=5), {}, 1 << 30, F.FALCON_ERR_UNSUPPORTED),       # Falcon-2/2A: forward only
+    (dict(rule=6 | 0x100), {}, 1 << 30, F.FALCON_ERR_UNSUPPORTED),
+    (dict(dk=129), {}, 1 << 30, F.FALCON_ERR_UNSUPPORTED),
+    (dict(dv=256), {}, 1 << 30, F.FALCON_ERR_UNSUPPORTED),
+    (dict(rule=3, window=16), {}, 1 << 30, F.FALCON_ERR_UNSUPPORTED),   # window staging too large
+    (dict(rule=3, window=0), {}, 1 << 30, F.FALCON_ERR_INVALID_ARG),
+    (dict(q=None), {}, 1 << 30, F.FALCON_ERR_INVALID_ARG),
+    (dict(eps=-1.0), {}, 1 << 30, F.FALCON_ERR_INVALID_ARG),
+    ({}, dict(dO=None), 1 << 30, F.FALCON_ERR_INVALID_ARG),
+    ({}, dict(deta=None), 1 << 30, F.FALCON_ERR_INVALID_ARG),
+    ({}, dict(dq=0x11002), 1 << 30, F.FALCON_ERR_INVALID_ARG),        # misaligned
+    ({}, {}, 0, F.FALCON_ERR_WORKSPACE),
+    ({}, {}, 1024, F.FALCON_ERR_WORKSPACE),
+    (dict(B=0), {}, 0, F.FALCON_OK),
+    (dict(T=0), {}, 0, F.FALCON_OK),
+])
+def test_backward_rejects_bad_arguments_on_host(L, akw, gkw, ws, expect):
+    a = _args(**{"o": None, **akw})
+    g = _grads(**gkw)
+    ws_ptr = 0x100000 if ws else None
+    assert L.falcon_bwd_recurrent(ctypes.byref(a), ctypes.byref(g), ws_ptr, ws, None) == expect
+    assert L.falcon_bwd_recurrent(None, ctypes.byref(g), ws_ptr, ws, None) == F.FALCON_ERR_INVALID_ARG
+    assert L.falcon_bwd_recurrent(ctypes.byref(_args(o=None)), None, ws_ptr, ws, None) in (
+        F.FALCON_ERR_INVALID_ARG, F.FALCON_OK)
+
+
+def test_backward_workspace_size(L):
+    """Checkpoints every C = ceil(sqrt(T)) steps plus one segment of C + 1 recomputed states, fp32,
+    per head."""
+    import math
+    for T, dk, dv in ((256, 32, 32), (100, 128, 64), (1, 16, 8), (4096, 128, 128)):
+        a = _args(T=T, dk=dk, dv=dv, o=None)
+        C = math.ceil(math.sqrt(T))
+        nseg = -(-T // C)
+        assert L.falcon_bwd_workspace_size(ctypes.byref(a)) == 2 * 3 * (nseg + C + 1) * dv * dk * 4
+    assert L.falcon_bwd_workspace_size(ctypes.byref(_args(T=0))) == 0
+    assert L.falcon_bwd_workspace_size(ctypes.byref(_args(rule=5))) == 0
+    assert L.falcon_bwd_workspace_size(None) == 0
+
+
 def test_empty_problems_launch_nothing(L):
     assert L.falcon_fwd_chunk(ctypes.byref(_args(B=0)), None, 0, None) == F.FALCON_OK
     assert L.falcon_fwd_recurrent(ctypes.byref(_args(H=0)), None) == F.FALCON_OK
@@ -156,6 +205,8 @@ def test_no_cpu_fallback_without_gpu(L):
     assert L.falcon_fwd_chunk(ctypes.byref(_args()), None, 0, None) == F.FALCON_ERR_CUDA
     assert L.falcon_fwd_recurrent(ctypes.byref(_args(dk=32, dv=32)), None) == F.FALCON_ERR_CUDA
     assert _dec(L) == F.FALCON_ERR_CUDA
+    assert L.falcon_bwd_recurrent(ctypes.byref(_args(o=None)), ctypes.byref(_grads()), 0x100000, 1 << 30,
+                                  None) == F.FALCON_ERR_CUDA
 
 
 def test_binding_raises_when_library_missing(monkeypatch, tmp_path):
