@@ -389,6 +389,45 @@ def bench_recurrent(args, D: Dist):
             "tokens_per_s": round(B * T / (ms * 1e-3), 1), "note": "latency bound, parity workload"}
 
 
+def bench_backward(args, D: Dist):
+    """Backward pass of the recurrent form (rank 0, CUDA events): Falcon-1, bf16 inputs, B1 H16 T1024
+    d128, with an initial state, a cached key and an upstream gradient of the final state. Latency
+    bound (one CTA walks each head's steps three times: checkpoints, recompute, reverse)."""
+    import numpy as np
+    import torch
+    from delta_rule_linear_falcon_b200 import falcon as F
+    from delta_rule_linear_falcon_b200 import inputs as I
+
+    B, H, T, d = 1, 16, 1024, 128
+    s = I.make_seq(1, B, H, T, d, d, seed=7, io_dtype="bf16", with_state=True, with_kprev=True)
+    dev = torch.device("cuda", D.local)
+    stream = torch.cuda.current_stream(dev)
+    bf = lambda x: torch.from_numpy(x).to(torch.bfloat16).to(dev)
+    f32 = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(dev)
+    q, k, v, kp = bf(s.q), bf(s.k), bf(s.v), bf(s.k_prev)
+    a, e, S0 = f32(s.alpha), f32(s.eta), f32(s.S0)
+    dO = f32(I.normal(8, 8, B * H * T * d).reshape(B, H, T, d))
+    dST = f32(I.normal(8, 9, B * H * d * d).reshape(B, H, d, d))
+    args_ = F.make_args(q, k, v, a, e, rule=1, eps=s.eps, S0=S0, k_prev=kp)
+    ws = torch.empty(F.falcon_bwd_workspace_size(args_), dtype=torch.uint8, device=dev)
+    run = lambda: F.falcon_bwd_recurrent(q, k, v, a, e, dO, rule=1, eps=s.eps, S0=S0, k_prev=kp, dS_T=dST,
+                                         workspace=ws, stream=stream)
+    for _ in range(2):
+        run()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(3):
+        run()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / 3
+    return {"workload": f"falcon1_bwd_recurrent_bf16_B{B}H{H}T{T}d{d}", "ms_per_call": round(ms, 3),
+            "tokens_per_s": round(B * T / (ms * 1e-3), 1), "workspace_bytes": int(ws.numel()),
+            "note": "latency bound: one CTA per head, forward to checkpoints, then recompute and reverse "
+                    "per segment"}
+
+
 def bench_more_chunk(args, D: Dist):
     """Secondary chunk workloads (rank 0, device-resident inputs, CUDA events): Falcon-3 and
     Falcon-3A (w = 4, B4 H16 T8192 d128), Falcon-1A on B1 H16 T32768 d128, and the benchmark
@@ -603,6 +642,7 @@ def main(argv=None):
     dec = bench_decode(args, D, clk)
     rec = bench_recurrent(args, D) if D.rank == 0 else None
     more = bench_more_chunk(args, D) if D.rank == 0 else None
+    bwd = bench_backward(args, D) if D.rank == 0 else None
 
     s = ch["s"]
     B, H, T, dk, dv = s.shape
@@ -650,6 +690,8 @@ def main(argv=None):
         line["recurrent"] = rec
     if more is not None:
         line["more_chunk"] = more
+    if bwd is not None:
+        line["backward"] = bwd
     if D.rank == 0 and D.world == 1:
         line["cpu_baseline"] = cpu_baseline(min_seconds=10.0)
     if D.rank == 0:

@@ -140,11 +140,15 @@ bwd_recurrent_kernel(BwdParams p) {
     if (gkp)
         for (int c = tid; c < dk; c += kBwdThreads) gkp[c] = 0.f;
 
-    auto store_state = [&](float *dst, const float *src) {   // padded shared rows -> dense dv x dk
-        for (size_t e = tid; e < DD; e += kBwdThreads) dst[e] = src[(e / dk) * LD + e % dk];
+    // dense dv x dk (global) <-> padded rows (shared): a warp per row, lanes along it
+    const int warp = tid >> 5, lane = tid & 31;
+    auto store_state = [&](float *dst, const float *src) {
+        for (int i = warp; i < dv; i += kBwdWarps)
+            for (int c = lane; c < dk; c += 32) dst[(size_t)i * dk + c] = src[i * LD + c];
     };
     auto load_state = [&](float *dst, const float *src) {
-        for (size_t e = tid; e < DD; e += kBwdThreads) dst[(e / dk) * LD + e % dk] = src[e];
+        for (int i = warp; i < dv; i += kBwdWarps)
+            for (int c = lane; c < dk; c += 32) dst[i * LD + c] = src ? src[(size_t)i * dk + c] : 0.f;
     };
     // beta of step t from the staged keys (every thread gets it) and its denominator
     auto step_beta = [&](long t, float &beta, float &den) {
@@ -188,8 +192,7 @@ bwd_recurrent_kernel(BwdParams p) {
     };
 
     // ---- pass 1: checkpoints S_{s C}, s = 0 .. nseg-1
-    for (size_t e = tid; e < DD; e += kBwdThreads)
-        sP[(e / dk) * LD + e % dk] = p.S0 ? p.S0[bh * DD + e] : 0.f;
+    load_state(sP, p.S0 ? p.S0 + bh * DD : nullptr);
     for (int s = 0; s < nseg; ++s) {
         __syncthreads();
         store_state(ckpt + (size_t)s * DD, sP);
@@ -198,8 +201,7 @@ bwd_recurrent_kernel(BwdParams p) {
     }
 
     // ---- reverse sweep, segment by segment
-    for (size_t e = tid; e < DD; e += kBwdThreads)
-        sU[(e / dk) * LD + e % dk] = p.dS_T ? p.dS_T[bh * DD + e] : 0.f;
+    load_state(sU, p.dS_T ? p.dS_T + bh * DD : nullptr);
     for (int s = nseg - 1; s >= 0; --s) {
         const long t0 = (long)s * C, t1 = min((long)T, t0 + C);
         __syncthreads();
@@ -308,8 +310,7 @@ bwd_recurrent_kernel(BwdParams p) {
         }
     }
     __syncthreads();
-    if (p.dS0)
-        for (size_t e = tid; e < DD; e += kBwdThreads) p.dS0[bh * DD + e] = sU[(e / dk) * LD + e % dk];
+    if (p.dS0) store_state(p.dS0 + bh * DD, sU);
 }
 
 }  // namespace
