@@ -88,10 +88,13 @@ constexpr uint32_t kSmem = oBar + 512 + 1024;
 static_assert(kSmem <= 232448, "shared memory");
 
 // TMEM columns
-// GP | slot 0 | slot 1 | A^T, B' | S (bf16) then -Z~ (bf16; R'^T for the inner-product rules' history)
+// GP | slot 0 | slot 1 | A^T, B' | S (bf16) then -Z~ (bf16)
 // Slot c & 1 holds [S X^T | S Q^T] of block c from (b); once the chain has read S X^T, (e') puts
-// R'^T B'^T in its place. dS of block c takes all of the other slot, free between the chain's read
-// of the outputs of block c-1 and (b) of block c+1.
+// R'^T B'^T in its place. Regression rules: dS of block c takes the AB columns once the chain has
+// copied A^T and B' of the block out of them, and frees them for (A), (B') of the next block when
+// the state update has read it, so the outputs of block c-1 can be read out of the other slot while
+// (b) and (A), (B') run. Inner-product rules: dS of block c takes all of the other slot, free
+// between the chain's read of the outputs of block c-1 and (b) of block c+1.
 constexpr uint32_t cGP = 0, cSXO = 64 /* + 128 * slot */, cAB = 320, cSR = 448, kTmemCols = 512;
 
 constexpr uint32_t kIdN64 = tc::idesc_bf16(128, 64, 0, 0);
@@ -119,7 +122,8 @@ enum {
     B_PRDY = 26,       // P~ ready -> MMA (B')
     B_TRDY = 27,       // T_f, T' (and the step sizes) ready -> MMA (A), (B')
     B_ABDONE = 28,     // (A), (B') done -> chain, local (T tiles free), helpers (P~ tile free)
-    B_EARDY = 29,      // A^T, B' in shared memory (8 warps) -> MMA (e'), (f')
+    B_EARDY = 29,      // the AB columns are free again (8 warps): regression rules after dS is read, inner
+                       // product after the outputs are read -> (A), (B') / dS of the next block
     B_BDONE = 30,      // (b) done -> chain
     B_RT = 31,         // -Z~ in TMEM (8 warps) -> MMA (e'), (f')
     B_EFDONE = 32,     // (f') done: dS in TMEM -> chain
@@ -1024,6 +1028,14 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 tc::mma_commit_elect(&bars[B_SQDONE]);
                 tc::mma_commit_elect(&bars[B_XQFREE + u]);   // (b) of the slot is done (the other arrival)
             }
+            // outputs of the previous block while (b) and (A), (B') run: their slot takes (b) of the
+            // next block
+            if (c >= 1) {
+                store_out(c - 1);
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[B_SCALFREE + (c - 1) % 4]);
+            }
             // A^T (rows d, columns i) and B' (rows i < 64) from TMEM to their shared-memory tiles
             if (!(ok = chain_wait(B_ABDONE, c & 1))) break;
             {
@@ -1039,22 +1051,15 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 }
             }
             tc::fence_proxy_async();
-            warp_arrive(&bars[B_EARDY]);    // the AB columns may take (A), (B') of the next block
-            // outputs of the previous block (their columns take dS of this block)
-            if (c >= 1) {
-                store_out(c - 1);
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[B_SCALFREE + (c - 1) % 4]);
-            }
-            // Y^T A, the state-independent half of dS, into slot s^1 once V has landed (the barrier also
-            // says that A^T is in shared memory and the outputs of block c-1 are read out of the slot)
+            tc::fence_before_sync();
+            // Y^T A, the state-independent half of dS, into the AB columns once V has landed (the
+            // barrier also says that A^T and B' have been read out of those columns)
             if (!(ok = chain_wait(B_FULLV + s, (c >> 1) & 1))) break;
             const uint64_t dY = tc::sdesc(tc::smem_u32(sm + oV + s * kVst), 8192, 1024);   // Y^T, MN-major A
             if (issuer) {
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16_elect(tbase + cSXO + 128 * (s ^ 1), dY + (uint64_t)(ks * 128), dAtC + (uint64_t)(ks * 2), kIdVA, ks > 0);
+                    tc::mma_bf16_elect(tbase + cAB, dY + (uint64_t)(ks * 128), dAtC + (uint64_t)(ks * 2), kIdVA, ks > 0);
             }
             // -Z~ = -(S X^T) diag(2^g), bf16 into TMEM: with dS = Y^T A - Z~ A and E = Y^T B'^T - Z~ B'^T the
             // values themselves only enter through the tensor cores. It replaces the bf16 state, which
@@ -1084,7 +1089,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 tc::fence_after_sync();
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * (s ^ 1), tbase + cSR + 8 * ks, dAtC + (uint64_t)(ks * 2), kIdN128, true);
+                    tc::mma_bf16_ts_elect(tbase + cAB, tbase + cSR + 8 * ks, dAtC + (uint64_t)(ks * 2), kIdN128, true);
                 tc::mma_commit_elect(&bars[B_EFDONE]);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
@@ -1099,7 +1104,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             if (!(ok = chain_wait(B_EFDONE, c & 1))) break;
             {
                 const float dl = exp2f(sGL[u4]);
-                const uint32_t cds = cSXO + 128 * (s ^ 1) + 64 * hf;
+                const uint32_t cds = cAB + 64 * hf;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float v[32];
@@ -1108,6 +1113,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                     for (int j = 0; j < 32; ++j) S[32 * hh + j] = dl * S[32 * hh + j] + v[j];
                 }
             }
+            warp_arrive(&bars[B_EARDY]);    // dS read: the AB columns may take (A), (B') of the next block
             // (e') still reads -Z~ from the columns the bf16 state takes
             if (!(ok = chain_wait(B_EDONE, c & 1))) break;
             store_S();
