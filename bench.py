@@ -385,8 +385,32 @@ def bench_recurrent(args, D: Dist):
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / 20
     B, H, T, dk, dv = s.shape
-    return {"workload": s.name, "ms_per_call": round(ms, 4),
-            "tokens_per_s": round(B * T / (ms * 1e-3), 1), "note": "latency bound, parity workload"}
+    out = {"workload": s.name, "ms_per_call": round(ms, 4),
+           "tokens_per_s": round(B * T / (ms * 1e-3), 1), "note": "latency bound, parity workload"}
+    # The per-column rules (Falcon-2 / 2A) run on the recurrent kernel only: one head per CTA walks
+    # its tokens one by one, so a full-width problem shows that path's own rate.
+    per_col = {}
+    for rule, name in ((5, "falcon2"), (6, "falcon2a")):
+        s2 = I.make_seq(rule, 1, 16, 4096, 128, 128, seed=11, io_dtype="bf16")
+        q2, k2, v2 = (torch.from_numpy(x).to(torch.bfloat16).to(dev) for x in (s2.q, s2.k, s2.v))
+        a2, e2 = (torch.from_numpy(x).to(dev) for x in (s2.alpha, s2.eta))
+        n_out = torch.empty((1, 16, 128), dtype=torch.float32, device=dev)
+        run2 = lambda: F.falcon_fwd_recurrent(q2, k2, v2, a2, e2, rule=rule, eps=s2.eps, n_out=n_out,
+                                              stream=stream)
+        for _ in range(2):
+            run2()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(3):
+            run2()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        ms2 = t0.elapsed_time(t1) / 3
+        per_col[f"{name}_recurrent_bf16_B1H16T4096d128"] = {
+            "ms_per_call": round(ms2, 3), "tokens_per_s": round(4096 / (ms2 * 1e-3), 1),
+            "note": "recurrent kernel (the only path of the per-column rules), latency bound"}
+    out["per_column_rules"] = per_col
+    return out
 
 
 def bench_backward(args, D: Dist):
