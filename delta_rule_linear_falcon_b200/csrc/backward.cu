@@ -5,7 +5,7 @@
 // cached key. fp32 state and fp32 arithmetic; q, k, v in the I/O dtype, every gradient
 // in fp32.
 //
-// One CTA of 128 threads per (b, h). With U = dL/dS after step t (starting from dS_T),
+// One CTA of 512 threads per (b, h). With U = dL/dS after step t (starting from dS_T),
 // step t (0-based, pairs j = t - m of window slot m, Sbar = alpha_t S_{t-1}) gives
 //   U += dO_t q_t^T,                       dq_t = S_t^T dO_t
 //   regression (r_m = Sbar x_m - y_m, S_t = Sbar - beta sum_m r_m x_m^T):
@@ -22,10 +22,12 @@
 // The states are not kept: a first forward pass stores S at the start of every segment of
 // C steps in the workspace, and the reverse sweep re-runs each segment forward from its
 // checkpoint into a buffer of C + 1 states before walking it backwards. U and the two
-// states a step needs (before and after it) sit in shared memory with rows padded to
-// d_k + 1 floats, so that a thread can walk a row (thread = value row i) or a column
-// (thread = key column c) without bank conflicts: row products (U x, Sbar x, the state
-// update) and column products (S^T dO, U^T r, Sbar^T dr) are both plain loops.
+// states a step needs (before and after it) sit in shared memory. Row products (U x, Sbar x,
+// the state update) take four threads per value row i, each every fourth column, reduced
+// with two shuffles; the row stride is 4 more than a multiple of 32 floats, so the 32 threads
+// of a warp (8 rows x 4 column phases) hit 32 different banks. Column products (S^T dO,
+// U^T r, Sbar^T dr) take one thread per key column c in each of four row groups, reduced
+// through shared memory.
 #include <math.h>
 
 #include "common.cuh"
@@ -35,18 +37,19 @@ namespace falcon {
 
 namespace {
 
-constexpr int kBwdThreads = 128;
+constexpr int kBwdThreads = 512;
 constexpr int kBwdWarps = kBwdThreads / 32;
+constexpr int kRowGroups = kBwdThreads / 128;   // column products: four row groups of 128 columns
 
 struct BwdSmem {
     int LD, dk, dv, w;
     // offsets in floats
-    size_t oU, oP, oA, oX, oY, oQ, oG, oUx, oR, oDr, oRed, total;
+    size_t oU, oP, oA, oX, oY, oQ, oG, oUx, oR, oDr, oPart, oRed, total;
 };
 
 __host__ __device__ inline BwdSmem bwd_smem(int dk, int dv, int w) {
     BwdSmem s;
-    s.LD = dk + 1; s.dk = dk; s.dv = dv; s.w = w;
+    s.LD = ((dk + 27) / 32) * 32 + 4; s.dk = dk; s.dv = dv; s.w = w;
     const size_t mat = (size_t)dv * s.LD;
     s.oU = 0; s.oP = mat; s.oA = 2 * mat;
     s.oX = 3 * mat;
@@ -56,7 +59,8 @@ __host__ __device__ inline BwdSmem bwd_smem(int dk, int dv, int w) {
     s.oUx = s.oG + dv;
     s.oR = s.oUx + (size_t)w * dv;
     s.oDr = s.oR + (size_t)w * dv;
-    s.oRed = s.oDr + (size_t)w * dv;
+    s.oPart = s.oDr + (size_t)w * dv;                 // kRowGroups x (1 + w) x dk partial column sums
+    s.oRed = s.oPart + (size_t)kRowGroups * (1 + w) * dk;
     s.total = s.oRed + 2 * kBwdWarps + 4;
     return s;
 }
@@ -72,6 +76,13 @@ __device__ __forceinline__ float block_sum(float x, float *red) {
 #pragma unroll
     for (int i = 0; i < kBwdWarps; ++i) s += red[i];
     return s;
+}
+
+// Sum over the four threads of a value row (lanes 4i .. 4i + 3); all four get it.
+__device__ __forceinline__ float quad_sum(float x) {
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    return x;
 }
 
 template <typename IO>
@@ -115,7 +126,11 @@ bwd_recurrent_kernel(BwdParams p) {
     float *sU = smem + L.oU, *sP = smem + L.oP, *sA = smem + L.oA;
     float *sX = smem + L.oX, *sY = smem + L.oY, *sQ = smem + L.oQ, *sG = smem + L.oG;
     float *sUx = smem + L.oUx, *sR = smem + L.oR, *sDr = smem + L.oDr, *sRed = smem + L.oRed;
+    float *sPart = smem + L.oPart;
     const int tid = threadIdx.x;
+    const int ri = tid >> 2, rq = tid & 3;          // row products: value row ri, columns rq, rq + 4, ..
+    const bool rok = ri < dv;
+    const int cc = tid & 127, rg = tid >> 7;        // column products: key column cc, rows rg, rg + 4, ..
     const size_t bh = blockIdx.x;
     const size_t DD = (size_t)dv * dk;
 
@@ -166,27 +181,31 @@ bwd_recurrent_kernel(BwdParams p) {
         float beta, den;
         step_beta(t, beta, den);
         const float a = ctx.al[t];
-        for (int i = tid; i < dv; i += kBwdThreads) {
-            float *Si = sP + (size_t)i * LD;
-            for (int c = 0; c < dk; ++c) Si[c] *= a;
-            if (REG) {
+        float *Si = sP + (size_t)(rok ? ri : 0) * LD;
+        if (rok)
+            for (int c = rq; c < dk; c += 4) Si[c] *= a;
+        if (REG) {
+            // residuals at the decayed state first (every window pair), then the update
+            for (int m = 0; m < w; ++m) {
+                const float *x = sX + (size_t)m * dk;
+                float r = 0.f;
+                if (rok)
+                    for (int c = rq; c < dk; c += 4) r = fmaf(Si[c], x[c], r);
+                r = quad_sum(r);
+                if (rok && rq == 0) sR[(size_t)m * dv + ri] = r - sY[(size_t)m * dv + ri];
+            }
+            __syncwarp();
+            if (rok)
                 for (int m = 0; m < w; ++m) {
                     const float *x = sX + (size_t)m * dk;
-                    float r = -sY[(size_t)m * dv + i];
-                    for (int c = 0; c < dk; ++c) r = fmaf(Si[c], x[c], r);
-                    sR[(size_t)m * dv + i] = r;
+                    const float br = beta * sR[(size_t)m * dv + ri];
+                    for (int c = rq; c < dk; c += 4) Si[c] = fmaf(-br, x[c], Si[c]);
                 }
-                for (int m = 0; m < w; ++m) {
-                    const float *x = sX + (size_t)m * dk;
-                    const float br = beta * sR[(size_t)m * dv + i];
-                    for (int c = 0; c < dk; ++c) Si[c] = fmaf(-br, x[c], Si[c]);
-                }
-            } else {
-                for (int m = 0; m < w; ++m) {
-                    const float *x = sX + (size_t)m * dk;
-                    const float by = beta * sY[(size_t)m * dv + i];
-                    for (int c = 0; c < dk; ++c) Si[c] = fmaf(by, x[c], Si[c]);
-                }
+        } else if (rok) {
+            for (int m = 0; m < w; ++m) {
+                const float *x = sX + (size_t)m * dk;
+                const float by = beta * sY[(size_t)m * dv + ri];
+                for (int c = rq; c < dk; c += 4) Si[c] = fmaf(by, x[c], Si[c]);
             }
         }
     };
@@ -228,25 +247,32 @@ bwd_recurrent_kernel(BwdParams p) {
             const float a = ctx.al[t];
             // rows: U += dO q^T; U x_m; residuals r_m at the decayed state
             float part = 0.f;
-            for (int i = tid; i < dv; i += kBwdThreads) {
-                float *Ui = sU + (size_t)i * LD;
-                const float *Pi = sP + (size_t)i * LD;
-                const float g = sG[i];
-                for (int c = 0; c < dk; ++c) Ui[c] = fmaf(g, sQ[c], Ui[c]);
+            {
+                float *Ui = sU + (size_t)(rok ? ri : 0) * LD;
+                const float *Pi = sP + (size_t)(rok ? ri : 0) * LD;
+                if (rok) {
+                    const float g = sG[ri];
+                    for (int c = rq; c < dk; c += 4) Ui[c] = fmaf(g, sQ[c], Ui[c]);
+                }
                 for (int m = 0; m < w; ++m) {
                     const float *x = sX + (size_t)m * dk;
                     float ux = 0.f, sx = 0.f;
-                    for (int c = 0; c < dk; ++c) {
-                        ux = fmaf(Ui[c], x[c], ux);
-                        sx = fmaf(Pi[c], x[c], sx);
-                    }
-                    sUx[(size_t)m * dv + i] = ux;
-                    if (REG) {
-                        const float r = a * sx - sY[(size_t)m * dv + i];
-                        sR[(size_t)m * dv + i] = r;
-                        part -= r * ux;
-                    } else {
-                        part += sY[(size_t)m * dv + i] * ux;
+                    if (rok)
+                        for (int c = rq; c < dk; c += 4) {
+                            ux = fmaf(Ui[c], x[c], ux);
+                            sx = fmaf(Pi[c], x[c], sx);
+                        }
+                    ux = quad_sum(ux);
+                    sx = quad_sum(sx);
+                    if (rok && rq == 0) {
+                        sUx[(size_t)m * dv + ri] = ux;
+                        if (REG) {
+                            const float r = a * sx - sY[(size_t)m * dv + ri];
+                            sR[(size_t)m * dv + ri] = r;
+                            part -= r * ux;
+                        } else {
+                            part += sY[(size_t)m * dv + ri] * ux;
+                        }
                     }
                 }
             }
@@ -255,50 +281,62 @@ bwd_recurrent_kernel(BwdParams p) {
             const float dN = has_den ? -dbeta * beta / den : 0.f;
             if (tid == 0) get[t] = has_den ? dbeta / den : 0.f;
             // rows: dr_m, dy_m (scattered to the value row of pair j)
-            for (int i = tid; i < dv; i += kBwdThreads) {
-                for (int m = 0; m < w; ++m) {
-                    const float ux = sUx[(size_t)m * dv + i];
-                    if (REG) sDr[(size_t)m * dv + i] = -beta * ux;
+            if (rok)
+                for (int m = rq; m < w; m += 4) {
+                    const float ux = sUx[(size_t)m * dv + ri];
+                    if (REG) sDr[(size_t)m * dv + ri] = -beta * ux;
                     const long j = t - m;
-                    if (j >= 0) gv[(size_t)j * dv + i] += beta * ux;   // dy = -dr (regression) = beta U x
+                    if (j >= 0) gv[(size_t)j * dv + ri] += beta * ux;   // dy = -dr (regression) = beta U x
                 }
-            }
             __syncthreads();
             // columns: dq_t = S_t^T dO_t; dx_m (scattered to the key row of pair j)
-            for (int c = tid; c < dk; c += kBwdThreads) {
+            if (cc < dk) {   // partial sums over the rows of this thread's group
                 float acc = 0.f;
-                for (int i = 0; i < dv; ++i) acc = fmaf(sA[(size_t)i * LD + c], sG[i], acc);
-                gq[(size_t)t * dk + c] = acc;
+                for (int i = rg; i < dv; i += kRowGroups) acc = fmaf(sA[(size_t)i * LD + cc], sG[i], acc);
+                sPart[(size_t)rg * (1 + w) * dk + cc] = acc;
                 for (int m = 0; m < w; ++m) {
                     float dx = 0.f;
                     if (REG) {
                         const float *r = sR + (size_t)m * dv, *dr = sDr + (size_t)m * dv;
-                        for (int i = 0; i < dv; ++i) {
-                            dx = fmaf(-beta * sU[(size_t)i * LD + c], r[i], dx);
-                            dx = fmaf(a * sP[(size_t)i * LD + c], dr[i], dx);
+                        for (int i = rg; i < dv; i += kRowGroups) {
+                            dx = fmaf(-beta * sU[(size_t)i * LD + cc], r[i], dx);
+                            dx = fmaf(a * sP[(size_t)i * LD + cc], dr[i], dx);
                         }
                     } else {
                         const float *y = sY + (size_t)m * dv;
-                        for (int i = 0; i < dv; ++i) dx = fmaf(beta * sU[(size_t)i * LD + c], y[i], dx);
+                        for (int i = rg; i < dv; i += kRowGroups) dx = fmaf(beta * sU[(size_t)i * LD + cc], y[i], dx);
                     }
-                    dx = fmaf(2.f * dN, sX[(size_t)m * dk + c], dx);
-                    const long j = t - m;
-                    if (j < 0) continue;
-                    if (ctx.same) gk[(size_t)j * dk + c] += dx;
-                    else if (j >= 1) gk[(size_t)(j - 1) * dk + c] += dx;
-                    else if (gkp) gkp[c] += dx;
+                    sPart[((size_t)rg * (1 + w) + 1 + m) * dk + cc] = dx;
                 }
+            }
+            __syncthreads();
+            for (int e = tid; e < (1 + w) * dk; e += kBwdThreads) {   // e = slot * dk + c
+                const int slot = e / dk, c = e - slot * dk;
+                float v = 0.f;
+#pragma unroll
+                for (int g = 0; g < kRowGroups; ++g) v += sPart[(size_t)g * (1 + w) * dk + e];
+                if (slot == 0) {
+                    gq[(size_t)t * dk + c] = v;
+                    continue;
+                }
+                const int m = slot - 1;
+                const float dx = fmaf(2.f * dN, sX[(size_t)m * dk + c], v);
+                const long j = t - m;
+                if (j < 0) continue;
+                if (ctx.same) gk[(size_t)j * dk + c] += dx;
+                else if (j >= 1) gk[(size_t)(j - 1) * dk + c] += dx;
+                else if (gkp) gkp[c] += dx;
             }
             __syncthreads();
             // rows: dSbar = U + sum_m dr_m x_m^T; dalpha = <dSbar, S_{t-1}>; U <- alpha dSbar
             part = 0.f;
-            for (int i = tid; i < dv; i += kBwdThreads) {
-                float *Ui = sU + (size_t)i * LD;
-                const float *Pi = sP + (size_t)i * LD;
-                for (int c = 0; c < dk; ++c) {
+            if (rok) {
+                float *Ui = sU + (size_t)ri * LD;
+                const float *Pi = sP + (size_t)ri * LD;
+                for (int c = rq; c < dk; c += 4) {
                     float d = Ui[c];
                     if (REG)
-                        for (int m = 0; m < w; ++m) d = fmaf(sDr[(size_t)m * dv + i], sX[(size_t)m * dk + c], d);
+                        for (int m = 0; m < w; ++m) d = fmaf(sDr[(size_t)m * dv + ri], sX[(size_t)m * dk + c], d);
                     part = fmaf(d, Pi[c], part);
                     Ui[c] = a * d;
                 }
