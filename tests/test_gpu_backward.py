@@ -98,3 +98,11 @@ def test_backward_refuses_falcon2(F):
     with pytest.raises(F.FalconError) as ei:
         _gpu(F, s, dO, None)
     assert ei.value.status == F.FALCON_ERR_UNSUPPORTED
+
+
+def test_backward_bench_workload_heads(F):
+    """The benchmark's backward shape (bf16, T1024 d128, initial state, cached key, dS_T), two of its
+    heads: 32 checkpointed segments of 32 steps."""
+    s = I.make_seq(1, 1, 2, 1024, 128, 128, seed=7, io_dtype="bf16", with_state=True, with_kprev=True)
+    dO, dST = _upstream(680, 1, 2, 1024, 128, 128, True)
+    _check(F, s, dO, dST)

@@ -79,3 +79,15 @@ def test_falcon2_refused_by_chunk_and_decode(F):
         F.falcon_decode_step(S, kp, q[:, :, 0].contiguous(), k[:, :, 0].contiguous(), v[:, :, 0].contiguous(),
                              a[:, :, 0].contiguous(), e[:, :, 0].contiguous(), rule=6)
     assert ei.value.status == F.FALCON_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("rule", [5, 6])
+def test_falcon2_bench_shape(F, rule):
+    """The benchmark's Falcon-2 / 2A shape (bf16, T4096 d128), two heads: outputs at the bf16
+    tolerance, the fp32 state and column energies at 1e-4."""
+    s = I.make_seq(rule, 1, 2, 4096, 128, 128, seed=11, io_dtype="bf16")
+    o, S, kl, n = _run(F, s, None)
+    o_r, S_r, kl_r, n_r = oracle.falcon2(rule, s.q, s.k, s.v, s.alpha, s.eta, s.eps)
+    assert relerr(o, o_r) <= TOL_BF16
+    assert relerr(S, S_r) <= TOL_F32
+    assert relerr(n, n_r) <= TOL_F32
