@@ -237,10 +237,14 @@ def bench_chunk(args, D: Dist, clk):
     S = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
     kl = torch.empty((B, H, dk), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
+    # the two-pass path's tiles (every block's solved T_f, T'), allocated once like the outputs
+    need = F.falcon_workspace_size(F.make_args(q, k, v, a, e, rule=1, eps=s.eps, chunk=64, o=o, S_out=S,
+                                               k_last=kl))
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
 
     def step():
         F.falcon_fwd_chunk(q, k, v, a, e, rule=1, eps=s.eps, chunk=64, o=o, S_out=S, k_last=kl,
-                           stream=stream)
+                           workspace=ws, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -301,7 +305,7 @@ def bench_chunk(args, D: Dist, clk):
             qq, kk, vv, aa, ee = ins[b]
             oo, SS, kk_last = outs[b]
             F.falcon_fwd_chunk(qq, kk, vv, aa, ee, rule=1, eps=s.eps, chunk=64, o=oo, S_out=SS,
-                               k_last=kk_last, stream=stream)
+                               k_last=kk_last, workspace=ws, stream=stream)
             used[b].record(stream)
             down.wait_event(used[b])
             with torch.cuda.stream(down):
@@ -326,7 +330,8 @@ def bench_chunk(args, D: Dist, clk):
     assert torch.equal(ho[(n_e2e - 1) % 2], o.cpu())
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, ha, he))
     d2h = ho[0].numel() * ho[0].element_size() + hS[0].numel() * hS[0].element_size()
-    return dict(s=s, total_ms=total_ms, kern_ms=kern_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h)
+    return dict(s=s, total_ms=total_ms, kern_ms=kern_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
+                launches=2 if need else 1, workspace_bytes=need)
 
 
 def bench_decode(args, D: Dist, clk):
@@ -500,8 +505,9 @@ def bench_more_chunk(args, D: Dist):
                       "t_roofline_us": round(t_roof * 1e6, 2),
                       "roofline_bound": "hbm" if nbytes / (hbm * 1e9) >= flops / (tf * 1e12) else "tensor",
                       "roofline_frac": round(t_roof / (ms * 1e-3), 4), "launches": n,
-                      # the sequence split of the inner-product rule: state pass, scan, chunk kernel
-                      "kernels_per_call": 3 if need else 1, "workspace_bytes": need}
+                      # the sequence split of the inner-product rule: state pass, scan, chunk kernel;
+                      # the two-pass path of the regression rules: solve pass, chain kernel
+                      "kernels_per_call": (2 if rule & 1 else 3) if need else 1, "workspace_bytes": need}
         del q, k, v, a, e, o, S, kl, ws
 
     s3 = I.workload_chunk_f3()
@@ -678,7 +684,9 @@ def main(argv=None):
     flops = chunk_algorithmic_flops(B, H, T, dk, dv)
     achieved = nbytes / (ch["kern_ms"] * 1e-3) / 1e9
     t_roof = max(nbytes / (hbm * 1e9), flops / (tf * 1e12))
-    traffic = recorded_traffic("chunk_ws_kernel", CHUNK_KERNEL_SOURCES)
+    two_pass = ch["launches"] == 2
+    traffic = recorded_traffic("chunk_two_pass" if two_pass else "chunk_ws_kernel", CHUNK_KERNEL_SOURCES)
+    kname = "chunk_local_kernel + chunk_ws_kernel (one call)" if two_pass else "chunk_ws_kernel"
     dbytes = decode_algorithmic_bytes(dec["N"], dec["H"], dec["dk"], dec["dv"])
     dgbs = dbytes / (dec["ms"] * 1e-3) / 1e9
 
@@ -690,8 +698,9 @@ def main(argv=None):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(achieved / hbm, 4), "traffic": traffic,
                      "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else src,
-                     "algorithmic_bytes_per_launch": nbytes, "kernel": "chunk_ws_kernel",
-                     "kernel_ms": round(ch["kern_ms"], 4)},
+                     "algorithmic_bytes_per_launch": nbytes, "kernel": kname,
+                     "kernel_ms": round(ch["kern_ms"], 4), "launches_per_step": ch["launches"],
+                     "workspace_bytes": ch["workspace_bytes"]},
         "roofline_flops_and_bytes": {"flops": flops, "bytes": nbytes, "t_roofline_us": round(t_roof * 1e6, 2),
                                 "frac": round(t_roof / (ch["kern_ms"] * 1e-3), 4),
                                 "tflops": round(flops / (ch["kern_ms"] * 1e-3) / 1e12, 2),
@@ -701,7 +710,7 @@ def main(argv=None):
                 "h2d_bytes_per_step": ch["h2d"], "d2h_bytes_per_step": ch["d2h"],
                 "ms_per_step": round(ch["e2e_ms"], 3)},
         "clocks": clk.summary(),
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * ch["launches"],
         "decode": {"workload": f"falcon1_decode_N{dec['N']}H{dec['H']}d{dec['dk']}", "value": round(dgbs, 1),
                    "unit": "GB/s", "ms_per_step": round(dec["ms"], 4), "steps": dec["steps"],
                    "gpu_launches": dec["steps"],

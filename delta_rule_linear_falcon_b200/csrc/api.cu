@@ -157,7 +157,8 @@ size_t falcon_workspace_size(const falcon_args_t *a) {
     ChunkParams p = chunk_params(a);
     int sms = 0;
     if (!device_info(&p.err, &sms)) return 0;
-    return seg_plan(p, sms).bytes;
+    const size_t seg = seg_plan(p, sms).bytes;
+    return seg ? seg : chunk_tile_bytes(p);
 }
 
 falcon_status_t falcon_fwd_chunk(const falcon_args_t *a, void *workspace, size_t workspace_bytes,
@@ -188,6 +189,13 @@ falcon_status_t falcon_fwd_chunk(const falcon_args_t *a, void *workspace, size_t
         if (!workspace || workspace_bytes < plan.bytes) return FALCON_ERR_WORKSPACE;
         if (!aligned16(workspace)) return FALCON_ERR_INVALID_ARG;
         return launch_chunk_seg(p, plan, workspace, s) == cudaSuccess ? FALCON_OK : FALCON_ERR_CUDA;
+    }
+    // Regression rules: the two-pass path when the workspace holds every block's T tiles, the
+    // single-kernel path otherwise (NULL or a smaller workspace is not an error here).
+    const size_t tile_bytes = chunk_tile_bytes(p);
+    if (tile_bytes > 0 && workspace && workspace_bytes >= tile_bytes) {
+        if (!aligned16(workspace)) return FALCON_ERR_INVALID_ARG;
+        p.tiles = workspace;
     }
     return launch_chunk(p, sms, s) == cudaSuccess ? FALCON_OK : FALCON_ERR_CUDA;
 }

@@ -56,6 +56,7 @@
 // are loaded and only TB outputs are written per block.
 #include <cuda.h>
 
+#include "chunk_mma.cuh"
 #include "common.cuh"
 #include "launch.h"
 #include "tc_common.cuh"
@@ -131,7 +132,12 @@ enum {
     B_SRDY = 34,       // S bf16 in TMEM, dS read, O of the previous block read (8 warps) -> MMA (b)
     B_FINAL = 35,      // drain of the chain MMA warp's MMAs at exit
     B_SQDONE = 36,     // S Q^T done (it reads the bf16 state that -Z~ replaces) -> chain
-    B_COUNT = 37
+    B_FULLT = 37,      // [2] two-pass path: the block's T_f, T' tiles landed -> MMA (A), (B')
+    B_TFREE = 39,      // [2] two-pass path: (A), (B') that read the tile slot are done -> tile loads
+    B_OUTFREE = 41,    // [2] two-pass path: outputs of the slot's block read (4 output warps) -> (b)
+    B_EDONES = 43,     // [2] two-pass path: (e') of the slot's block done -> chain, output warps (one
+                       // barrier per slot, so that a slow output warp never sees a later phase)
+    B_COUNT = 45
 };
 
 __device__ __forceinline__ void named_bar(int id, int n) {
@@ -176,6 +182,38 @@ __device__ __forceinline__ float pick_lane(const float (&v)[64], int lane) {
 #pragma unroll
     for (int k = 0; k < 2; ++k) t2[k] = (lane & 2) ? t4[2 + k] : t4[k];
     return (lane & 1) ? t2[1] : t2[0];
+}
+
+// O^T of block c (TMEM slot c & 1: S Q^T scaled by 2^g per token, plus R'^T B'^T) to global memory
+// for value row `row` (TMEM lane base tl) and the query tokens 32 hf .. 32 hf + 31 of the block's TB:
+// for each token a warp stores the bf16 outputs of its 32 consecutive value rows, 64 contiguous bytes
+// per store instruction. dg2 holds 2^g of the block's tokens.
+template <int TB>
+__device__ __forceinline__ void store_out_rows(void *out, int bh, int T, int c, int row, uint32_t tl, int hf,
+                                               const float *dg2) {
+    constexpr int D = 128;
+    const int t0 = c * TB, nval = min(TB, T - t0);
+    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(out) + ((size_t)bh * T + t0) * D + row;
+#pragma unroll 1
+    for (int h = 0; h < 4; ++h) {          // 8 tokens at a time
+        const int i0 = 32 * hf + 8 * h;
+        if (i0 >= TB) break;               // a block has TB query tokens
+        // the scales first, so that their shared-memory latency overlaps the TMEM loads
+        const float4 da = *reinterpret_cast<const float4 *>(dg2 + i0);
+        const float4 db = *reinterpret_cast<const float4 *>(dg2 + i0 + 4);
+        const float dg[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+        float v[8], w[8];
+        tc::tmem_ld8x2(tl + cSXO + 128 * (c & 1) + 64 + i0, tl + cSXO + 128 * (c & 1) + i0, v, w);
+        __nv_bfloat16 *oi = o + (size_t)i0 * D;
+        if (i0 + 8 <= nval) {              // whole group (every group but the sequence's last)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) oi[j * D] = __float2bfloat16_rn(dg[j] * v[j] + w[j]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (i0 + j < nval) oi[j * D] = __float2bfloat16_rn(dg[j] * v[j] + w[j]);
+        }
+    }
 }
 
 // ---- tf32 warp MMA for the 16 x 16 blocks of the triangular solve
@@ -232,9 +270,11 @@ __device__ __forceinline__ void store16(float *C, const float (&acc)[2][4], int 
 //     round A: T_10, T_21, T_32 and W_20 T_00;  round B: T_20, T_31 and W_30 T_00 + W_31 T_10;
 //     round C: T_30.
 // Entries above the block diagonal of Tf are zero on entry and stay zero.
+// PACKED (a throughput-bound caller): the diagonal blocks go to two warps, 16 lanes per block.
+template <bool PACKED = false>
 __device__ __forceinline__ void solve_local(float *sL, float *sTf, int lt, int lw, int lane) {
-    if (lane < 16) {  // column j of the inverse of diagonal block b = warp, left-looking, rows of L as float4
-        const int b = lw, j = lane;
+    if (PACKED ? lw < 2 : lane < 16) {  // column j of the inverse of diagonal block b, left-looking, rows of L as float4
+        const int b = PACKED ? 2 * lw + (lane >> 4) : lw, j = lane & 15;
         const float *Lb = sL + (16 * b) * LDF + 16 * b;
         float x[16];
 #pragma unroll
@@ -313,9 +353,259 @@ __device__ __forceinline__ void solve_local(float *sL, float *sTf, int lt, int l
     named_bar(2, 128);
 }
 
+// ---- two-pass path of the regression rules, pass 1 (chunk_local_kernel)
+constexpr int kLocThreads = 128;
+constexpr int kLocCtasPerSm = 4;
+constexpr uint32_t kTileBytes = 16384;              // T_f then T', bf16 64 x 64 each, 128-byte swizzled
+constexpr uint32_t oLX = 0;                         // keys: 2 swizzled atoms of 64 rows
+constexpr uint32_t oLT = 16384;                     // T fp32 64 x LDF
+constexpr uint32_t oLL = oLT + 64 * LDF * 4;        // L / W fp32 64 x LDF, then the output tiles
+constexpr uint32_t oLS = oLL + 64 * LDF * 4;        // beta[64], g[64], 2^(g_last - g)[64], cf[64], carry, barrier
+constexpr uint32_t kLocSmem = oLS + 4 * 256 + 32 + 1024;   // + alignment of the base to 1024 bytes
+
+// One bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) into shared memory,
+// completing on the mbarrier's transaction count.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(tc::smem_u32(dst)), "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                 "r"(tc::smem_u32(src)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4_addr(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
 }  // namespace
 
-template <bool REG, int W>
+// Pass 1 of the two-pass path of the regression rules (window 1). The chunk-local step depends only
+// on a block's keys and gates, so it runs for every block at once before any state chain starts.
+// Persistent CTAs of 128 threads walk the (head, block) items; per item they form G = X X^T (bf16
+// mma.sync, fp32 accumulation), the step sizes from its diagonal, L = diag(beta)(Gamma o G) and
+// T = (I + L)^-1 (solve_local), and write T_f = diag(2^(g_last - g)) T diag(beta) and
+// T' = T diag(beta) as two bf16 tiles in the 128-byte swizzled order the tensor cores read, 16 KB
+// per item at tiles + (head * nblk + block) * 16 KB. The arithmetic is the one the single-kernel
+// path does on its local and helper warps. The keys of the next item are loaded by TMA (128-byte
+// swizzled, which also makes the ldmatrix reads of G conflict-free; rows before or past the sequence
+// read as zero) as soon as G of the current item has read its own, and the tiles leave by a bulk
+// copy that is only waited for before their buffer is written again, so the loads and stores of
+// one item overlap the arithmetic of the next.
+__global__ void __launch_bounds__(kLocThreads, kLocCtasPerSm)
+chunk_local_kernel(const __grid_constant__ CUtensorMap tmK, const ChunkParams p, const int nblk) {
+    extern __shared__ __align__(1024) uint8_t lsm_raw[];
+    uint8_t *lsm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(lsm_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sX = lsm + oLX;
+    float *sT = reinterpret_cast<float *>(lsm + oLT);
+    float *sL = reinterpret_cast<float *>(lsm + oLL);
+    uint8_t *sOut = lsm + oLL;
+    float *sBeta = reinterpret_cast<float *>(lsm + oLS);
+    float *sG = sBeta + 64, *sFr = sBeta + 128, *sCF = sBeta + 192, *sCarry = sBeta + 256;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sBeta + 260);
+
+    const int lt = threadIdx.x, lw = lt >> 5, lane = lt & 31;
+    const int T = p.T;
+    const int kshift = p.same_step ? 0 : 1;
+    constexpr int D = 128;
+    const long long items = (long long)p.B * p.H * nblk;
+    const volatile int no_abort = 0;
+
+    auto load_keys = [&](long long it) {   // thread 0: TMA of item it's key rows t0 - kshift ..
+        const int bh = (int)(it / nblk), c = (int)(it % nblk);
+        tc::mbar_arrive_expect_tx(bar, 16384);
+        tc::tma_load_3d(sX, &tmK, 0, c * kBlk - kshift, bh, bar);
+        tc::tma_load_3d(sX + 8192, &tmK, 64, c * kBlk - kshift, bh, bar);
+    };
+    // gates of an item for the threads of rows 0..63 (alpha, eta; 1 and 0 past the sequence)
+    auto load_gates = [&](long long it, float &a, float &e) {
+        const int bh = (int)(it / nblk), c = (int)(it % nblk), t = c * kBlk + lt;
+        const bool valid = lt < 64 && it < items && t < T;
+        a = valid ? p.alpha[(size_t)bh * T + t] : 1.f;
+        e = valid ? p.eta[(size_t)bh * T + t] : 0.f;
+    };
+
+    long long it = blockIdx.x;
+    if (lt == 0) {
+        tc::mbar_init(bar, 1);
+        tc::mbar_fence_init();
+        if (it < items) load_keys(it);
+    }
+    float ga, ge;
+    load_gates(it, ga, ge);
+    __syncthreads();
+    for (uint32_t k = 0; it < items; ++k, it += gridDim.x) {
+        const int bh = (int)(it / nblk), c = (int)(it % nblk);
+        const int t0 = c * kBlk, nval = min(kBlk, T - t0);
+        const long long nx = it + gridDim.x;
+        // cumulative log2 decay of the block (rows past the sequence add nothing)
+        float la = 0.f;
+        if (lt < 64) {
+            la = lt < nval ? log2f(ga) : 0.f;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, la, off);
+                if (lane >= off) la += y;
+            }
+            if (lt == 31) sCarry[0] = la;
+        }
+        const float ge_c = ge;
+        load_gates(nx, ga, ge);   // the next item's gates, in flight during this one
+        const bool landed = tc::mbar_wait(bar, k & 1, &no_abort, kDefaultWaitBudget);
+        if (landed && c == 0 && kshift == 1 && p.k_prev && lt < 16) {
+            // pair 0 = (k_prev, v_0): key row -1 is the cached key
+            const uint4 v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(p.k_prev) +
+                                                              (size_t)bh * D + lt * 8);
+            *reinterpret_cast<uint4 *>(sX + (lt >> 3) * 8192 + tc::sw128_chunk(0, lt & 7)) = v;
+        }
+        if (lt == 0) tc::tma_store_wait_read0();   // the previous item's tiles have left the L buffer
+        if (__syncthreads_or(!landed)) {
+            if (lt == 0) set_error(p.err, kDevErrTimeout);
+            break;
+        }
+        if (lt >= 32 && lt < 64) la += sCarry[0];
+        if (lt < 64) sG[lt] = la;
+
+        // G = X X^T, the 16 x 16 blocks on and below the diagonal: warp lw takes rows 16 lw .. 16 lw + 15.
+        // Lane l of an ldmatrix.x4 addresses row (l & 7) + 8 ((l >> 3) & 1) (A) or + 8 (l >> 4) (B) of
+        // its 16-row group and the 8-column chunk 2 k + (l >> 4) (A) or 2 k + ((l >> 3) & 1) (B).
+        {
+            const uint32_t xb = tc::smem_u32(sX);
+            auto chunk_addr = [&](int r, int ch) -> uint32_t {   // 16-byte chunk ch (0..15) of key row r
+                return xb + (uint32_t)((ch >> 3) * 8192 + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+            };
+            float acc[4][2][4];
+#pragma unroll
+            for (int np = 0; np < 4; ++np)
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[np][h][e] = 0.f;
+            const int ra = 16 * lw + (lane & 7) + 8 * ((lane >> 3) & 1), ca = lane >> 4;
+            const int rbo = (lane & 7) + 8 * (lane >> 4), cb = (lane >> 3) & 1;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                uint32_t a[4];
+                ldsm_x4_addr(a, chunk_addr(ra, 2 * ks + ca));
+#pragma unroll
+                for (int np = 0; np < 4; ++np) {
+                    if (np <= lw) {
+                        uint32_t b[4];
+                        ldsm_x4_addr(b, chunk_addr(16 * np + rbo, 2 * ks + cb));
+                        mma_bf16_16816(acc[np][0], a, b[0], b[1]);
+                        mma_bf16_16816(acc[np][1], a, b[2], b[3]);
+                    }
+                }
+            }
+            const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                if (np <= lw) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int col = 16 * np + 8 * h + 2 * t;
+                        *reinterpret_cast<float2 *>(sL + (16 * lw + g) * LDF + col) = make_float2(acc[np][h][0], acc[np][h][1]);
+                        *reinterpret_cast<float2 *>(sL + (16 * lw + g + 8) * LDF + col) = make_float2(acc[np][h][2], acc[np][h][3]);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        if (lt == 0 && nx < items) {   // the keys are read: the next item's may land in their place
+            tc::fence_proxy_async();
+            load_keys(nx);
+        }
+        if (lt < 64) {   // step sizes from the key norms on the diagonal; decay tables
+            const float nrm = sL[lt * LDF + lt];
+            sBeta[lt] = lt < nval ? step_size(ge_c, nrm, p.eps) : 0.f;
+            const float gl = sG[nval - 1];
+            sFr[lt] = exp2f(gl - la);
+            sCF[lt] = exp2f(sG[lt | 15] - la);
+        }
+        // T starts at zero (the solve writes only the blocks on and below the diagonal)
+        for (int idx = lt; idx < 64 * LDF / 4; idx += kLocThreads)
+            reinterpret_cast<float4 *>(sT)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+        __syncthreads();
+        {   // L = diag(beta)(Gamma o G) in place: thread (row r, half h) takes columns 32 h .. 32 h + 31
+            // (decay factors as in the single-kernel path: through the last index of a column block
+            // below the diagonal blocks, directly inside them)
+            const int r = lt >> 1, h = lt & 1, rb = r >> 4;
+            const float be = sBeta[r], gri = sG[r];
+            float *Lr = sL + r * LDF;
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int jb = 2 * h + jj;
+                if (jb < rb) {
+                    const float fac = be * exp2f(fminf(gri - sG[16 * jb + 15], 0.f));
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int j = 16 * jb + 4 * q;
+                        const float4 c4 = *reinterpret_cast<const float4 *>(sCF + j);
+                        float4 x = *reinterpret_cast<float4 *>(Lr + j);
+                        x.x *= fac * c4.x; x.y *= fac * c4.y; x.z *= fac * c4.z; x.w *= fac * c4.w;
+                        *reinterpret_cast<float4 *>(Lr + j) = x;
+                    }
+                } else if (jb == rb) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int j = 16 * jb + 4 * q;
+                        const float4 g4 = *reinterpret_cast<const float4 *>(sG + j);
+                        float4 x = *reinterpret_cast<float4 *>(Lr + j);
+                        x.x *= be * exp2f(fminf(gri - g4.x, 0.f));
+                        x.y *= be * exp2f(fminf(gri - g4.y, 0.f));
+                        x.z *= be * exp2f(fminf(gri - g4.z, 0.f));
+                        x.w *= be * exp2f(fminf(gri - g4.w, 0.f));
+                        *reinterpret_cast<float4 *>(Lr + j) = x;
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        solve_local<true>(sL, sT, lt, lw, lane);   // ends with a barrier of all 128 threads
+        {   // thread (row rr, half h) writes columns 32 h .. 32 h + 31 of both tiles: T' = T diag(beta)
+            // and T_f = 2^(g_last - g_rr) T'; chunks above the diagonal are zero
+            const int rr = lt >> 1, h = lt & 1;
+            const float fr = sFr[rr];
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+                const int cc = 4 * h + k4, j0 = 8 * cc;
+                float t8[8], f8[8];
+                if (j0 <= rr) {
+                    const float4 x0 = *reinterpret_cast<const float4 *>(sT + rr * LDF + j0);
+                    const float4 x1 = *reinterpret_cast<const float4 *>(sT + rr * LDF + j0 + 4);
+                    const float4 b0 = *reinterpret_cast<const float4 *>(sBeta + j0);
+                    const float4 b1 = *reinterpret_cast<const float4 *>(sBeta + j0 + 4);
+                    t8[0] = x0.x * b0.x; t8[1] = x0.y * b0.y; t8[2] = x0.z * b0.z; t8[3] = x0.w * b0.w;
+                    t8[4] = x1.x * b1.x; t8[5] = x1.y * b1.y; t8[6] = x1.z * b1.z; t8[7] = x1.w * b1.w;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) f8[q] = fr * t8[q];
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) t8[q] = f8[q] = 0.f;
+                }
+                st_chunk8(sOut, tc::sw128_chunk(rr, cc), f8);
+                st_chunk8(sOut + 8192, tc::sw128_chunk(rr, cc), t8);
+            }
+        }
+        tc::fence_proxy_async();
+        __syncthreads();
+        if (lt == 0) {
+            bulk_store(reinterpret_cast<uint8_t *>(p.tiles) + (size_t)it * kTileBytes, sOut, kTileBytes);
+            tc::tma_store_commit();
+        }
+    }
+    if (lt == 0) tc::tma_store_wait_read0();   // shared memory stays until the last copy has read it
+}
+
+// PRE (regression rules): T_f and T' of every block were written by chunk_local_kernel; the feed
+// warp brings them into a 2-slot ring with one bulk copy per block, and neither the local warps nor
+// the helpers form them.
+template <bool REG, int W, bool PRE>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                 const __grid_constant__ CUtensorMap tmV, ChunkParams p) {
@@ -348,7 +638,13 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             const bool chain_arrivals = (i >= B_SCALFREE && i < B_SCALFREE + 4) || i == B_EARDY || i == B_RT ||
                                         i == B_SRDY;
             const bool two = i >= B_XQFREE && i < B_XQFREE + 3;
-            tc::mbar_init(&bars[i], chain_arrivals ? kChainWarps : (i == B_GPFREE ? 3 : (two ? 2 : 1)));
+            const bool scal = i >= B_SCALFREE && i < B_SCALFREE + 4;
+            const bool outw = i == B_OUTFREE || i == B_OUTFREE + 1;
+            // two-pass path: the chain and the four output warps both read a scalar slot
+            const uint32_t n = (PRE && scal) ? kChainWarps + 4
+                               : chain_arrivals ? kChainWarps
+                               : outw ? 4 : (i == B_GPFREE ? (PRE ? 1 : 3) : (two ? 2 : 1));
+            tc::mbar_init(&bars[i], n);
         }
         *abort_flag = 0;
         tc::mbar_fence_init();
@@ -436,9 +732,12 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         const uint64_t dXmn0 = tc::sdesc(tc::smem_u32(sm + oXQ), 16384, 1024);  // X as an MN-major A
         const uint64_t dTF = tc::sdesc(tc::smem_u32(sTF), 8192, 1024);          // MN-major B, one N atom
         const uint64_t dTP = tc::sdesc(tc::smem_u32(sTP), 8192, 1024);
+        // two-pass path: tile slot 1 in the fp32 L / T buffers, which no solve uses then
+        const uint64_t dTF1 = tc::sdesc(tc::smem_u32(sm + oL), 8192, 1024);
+        const uint64_t dTP1 = tc::sdesc(tc::smem_u32(sm + oL + 8192), 8192, 1024);
         const uint64_t dPB = tc::sdesc(tc::smem_u32(sPB), 16, 1024);            // [P~; B'] K-major
         const int kshift = p.same_step ? 0 : 1;   // prefix-aligned key rows of block j start at t0 - 1
-        int kx = 0, kv = 0;
+        int kx = 0, kv = 0, kt = 0;
         bool ok = true;
         for (int j = 0; j <= nblk + 1 && ok; ++j) {
             // (a) first: it only needs its own slot (loaded in the previous iteration), so a slot that is
@@ -453,6 +752,19 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 for (int ks = 0; ks < 8; ++ks) tc::mma_bf16_elect(tbase + cGP, d + kmaj(ks), d + kmaj(ks), kIdN64, ks > 0);
                 tc::mma_commit_elect(&bars[B_ADONE]);
                 if (!REG) tc::mma_commit_elect(&bars[B_XQFREE + ja % 3]);   // one of the slot's two arrivals
+            }
+            const int jt = j - 1;   // two-pass path: the tiles of block j-1, one iteration before (A), (B')
+            if (PRE && jt >= 0 && jt < nblk) {
+                if (jt >= 2 && !(ok = wait_all(B_TFREE + (jt & 1), ((jt >> 1) - 1) & 1))) break;
+                if (lane == 0) {
+                    uint64_t *fb = &bars[B_FULLT + (jt & 1)];
+                    tc::mbar_arrive_expect_tx(fb, kTileBytes);
+                    bulk_load(sm + ((jt & 1) ? oL : oTF),
+                              reinterpret_cast<const uint8_t *>(p.tiles) + ((size_t)bh * nblk + jt) * kTileBytes,
+                              kTileBytes, fb);
+                }
+                __syncwarp();
+                kt = jt + 1;
             }
             if (j < nblk) {
                 if (j == p.dbg_stall_block) break;  // test hook: this block is never loaded
@@ -481,19 +793,22 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             }
             const int jb = j - 2;   // (A) A^T = X^T T_f and (B') B' = P~ T' into the AB columns, free once
             if (REG && jb >= 0 && jb < nblk) {  // the chain copied A^T, B' of the block before
-                if (!(ok = wait_all(B_TRDY, jb & 1) && wait_all(B_PRDY, jb & 1) &&
-                           (jb == 0 || wait_all(B_EARDY, (jb - 1) & 1))))
+                if (!(ok = (PRE ? wait_all(B_FULLT + (jb & 1), (jb >> 1) & 1) : wait_all(B_TRDY, jb & 1)) &&
+                           wait_all(B_PRDY, jb & 1) && (jb == 0 || wait_all(B_EARDY, (jb - 1) & 1))))
                     break;
                 tc::fence_after_sync();
                 const int u = jb % 3;
+                const bool t1 = PRE && (jb & 1);
+                const uint64_t dtf = t1 ? dTF1 : dTF, dtp = t1 ? dTP1 : dTP;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16_elect(tbase + cAB, dXmn0 + slot_off(u) + (uint64_t)(ks * 128), dTF + (uint64_t)(ks * 128), kIdAT, ks > 0);
+                    tc::mma_bf16_elect(tbase + cAB, dXmn0 + slot_off(u) + (uint64_t)(ks * 128), dtf + (uint64_t)(ks * 128), kIdAT, ks > 0);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc::mma_bf16_elect(tbase + cAB + 64, dPB + (uint64_t)(ks * 2), dTP + (uint64_t)(ks * 128), kIdBP, ks > 0);
+                    tc::mma_bf16_elect(tbase + cAB + 64, dPB + (uint64_t)(ks * 2), dtp + (uint64_t)(ks * 128), kIdBP, ks > 0);
                 tc::mma_commit_elect(&bars[B_ABDONE]);
                 tc::mma_commit_elect(&bars[B_XQFREE + u]);   // (a), (A) of the slot are done (one of two arrivals)
+                if (PRE) tc::mma_commit_elect(&bars[B_TFREE + (jb & 1)]);
             }
         }
         if (!ok) *abort_flag = 1;
@@ -506,6 +821,8 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
                 tc::mbar_wait(&bars[B_FULLXQ + c % 3], (c / 3) & 1, &no_abort, kDrainBudget);
             for (int c = kv - 2 < 0 ? 0 : kv - 2; c < kv; ++c)
                 tc::mbar_wait(&bars[B_FULLV + (c & 1)], (c >> 1) & 1, &no_abort, kDrainBudget);
+            for (int c = kt - 2 < 0 ? 0 : kt - 2; c < kt; ++c)
+                tc::mbar_wait(&bars[B_FULLT + (c & 1)], (c >> 1) & 1, &no_abort, kDrainBudget);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -715,7 +1032,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             tc::fence_proxy_async();
             named_bar(1, 64);
             if (leader) mbar_arrive(&bars[B_PRDY]);
-            if (REG) {
+            if (REG && !PRE) {
                 // T_f = diag(2^(g_last - g)) T diag(beta) and T' = T diag(beta) (bf16, m-major order) from
                 // the solved T; the tiles are free since (A), (B') of block c-1 are done (waited above)
                 if (!(ok = role_wait(&bars[B_SOLVED], c & 1, leader, 1, 64))) break;
@@ -780,6 +1097,24 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             // the block after next: its slot frees once (b) of block c-1 is done
             if (c + 2 < nblk && !(ok = prep(c + 2))) break;
         }
+    } else if (warp < 8 && PRE) {
+        // ================================================================ outputs (two-pass path)
+        // The local warps have no solve to run; they store the outputs of each block once (e') is done,
+        // which takes that work off the chain. Warp 4 + q reads TMEM lanes 32 q .. 32 q + 31.
+        const int qd = warp & 3, row = 32 * qd + lane;
+        const uint32_t tl = tbase + ((uint32_t)(32 * qd) << 16);
+        for (int c = 0; c < nblk; ++c) {
+            if (!warp_wait(&bars[B_EDONES + (c & 1)], (c >> 1) & 1)) break;
+            tc::fence_after_sync();
+            store_out_rows<TB>(p.o, bh, T, c, row, tl, 0, sScal + (c % 4) * 256 + 64);
+            store_out_rows<TB>(p.o, bh, T, c, row, tl, 1, sScal + (c % 4) * 256 + 64);
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars[B_OUTFREE + (c & 1)]);   // (b) of block c + 2 may take the slot
+                mbar_arrive(&bars[B_SCALFREE + c % 4]);
+            }
+        }
     } else if (warp < 8) {
         // ================================================================ local (128 threads)
         const int lt = tid - 128, lw = warp - 4;
@@ -789,7 +1124,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         const float *eta_h = p.eta + (size_t)bh * T;
         const int rs = r % TB;             // token of row r (rows of one token share its step size)
         float ge = (lw < 2 && rs < T) ? eta_h[rs] : 0.f;  // step-size gate of row r's token, one block ahead
-        for (int c = 0; c < nblk; ++c) {
+        for (int c = 0; c < nblk && !PRE; ++c) {   // (the two-pass path has no work for these warps)
             const int u4 = c % 4;
             // (a) of the block follows the helpers' readiness of it, which follows its decay scalars:
             // ADONE alone says both
@@ -932,33 +1267,8 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(S[2 * j], S[2 * j + 1]);
             tc::tmem_st32(tl + cSR + 32 * hf, pk);
         };
-        // O^T of block c (TMEM slot c & 1: S Q^T scaled by 2^g per token, plus R'^T B'^T) to global
-        // memory: for each token a warp stores the bf16 outputs of its 32 consecutive value rows, 64
-        // contiguous bytes per store instruction.
         auto store_out = [&](int c) {
-            const int t0 = c * TB, nval = min(TB, T - t0);
-            __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.o) + ((size_t)bh * T + t0) * D + row;
-#pragma unroll 1
-            for (int h = 0; h < 4; ++h) {          // 8 tokens at a time
-                const int i0 = 32 * hf + 8 * h;
-                if (i0 >= TB) break;               // a block has TB query tokens
-                const float *d2 = sScal + (c % 4) * 256 + 64 + i0;   // 2^g of the tokens
-                // the scales first, so that their shared-memory latency overlaps the TMEM loads
-                const float4 da = *reinterpret_cast<const float4 *>(d2);
-                const float4 db = *reinterpret_cast<const float4 *>(d2 + 4);
-                const float dg[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
-                float v[8], w[8];
-                tc::tmem_ld8x2(tl + cSXO + 128 * (c & 1) + 64 + i0, tl + cSXO + 128 * (c & 1) + i0, v, w);
-                __nv_bfloat16 *oi = o + (size_t)i0 * D;
-                if (i0 + 8 <= nval) {              // whole group (every group but the sequence's last)
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) oi[j * D] = __float2bfloat16_rn(dg[j] * v[j] + w[j]);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        if (i0 + j < nval) oi[j * D] = __float2bfloat16_rn(dg[j] * v[j] + w[j]);
-                }
-            }
+            store_out_rows<TB>(p.o, bh, T, c, row, tl, hf, sScal + (c % 4) * 256 + 64);
         };
         {
             const float *S0 = p.S0 ? p.S0 + ((size_t)bh * D + row) * D + 64 * hf : nullptr;
@@ -1011,7 +1321,110 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         };
         const uint64_t dAtC = tc::sdesc(tc::smem_u32(sA), 16, 1024);          // A^T, K-major B of dS
         const uint64_t dBpC = tc::sdesc(tc::smem_u32(sPB + 8192), 16, 1024);  // B', K-major B of E
-        for (int c = 0; c < nblk && REG; ++c) {
+        // Two-pass path: the output warps store the outputs, so the chain only runs the state chain.
+        // (b) is one group of N = 128 ([X;Q] as the B operand), and A^T, B' are copied out first:
+        // their (A), (B') ran during the previous block's state update.
+        for (int c = 0; c < nblk && REG && PRE; ++c) {
+            const int s = c & 1, u = c % 3, u4 = c % 4;
+            {   // the block's [X;Q] slot is ready, and the outputs of block c-2 have left slot s
+                bool failed = false;
+                if (ct == 32) {
+                    failed = !tc::mbar_wait(&bars[B_XQRDY + u], (c / 3) & 1, abort_flag, p.wait_budget) ||
+                             (c >= 2 && !tc::mbar_wait(&bars[B_OUTFREE + s], ((c >> 1) - 1) & 1, abort_flag,
+                                                       p.wait_budget));
+                    if (failed) *abort_flag = 1;
+                }
+                if (!(ok = !named_bar_or(4, 256, failed))) break;
+                tc::fence_after_sync();
+            }
+            if (issuer) {
+                const uint64_t dXQ = dXQ0 + slot_off(u);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dXQ + kmaj(ks), kIdN128, ks > 0);
+                tc::mma_commit_elect(&bars[B_BDONE]);
+                tc::mma_commit_elect(&bars[B_XQFREE + u]);   // (b) of the slot is done (the other arrival)
+            }
+            if (!(ok = chain_wait(B_ABDONE, c & 1))) break;
+            {
+                float v[32];
+                tc::tmem_ld32(tl + cAB + 32 * hf, v);
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) st_chunk8(sA, tc::sw128_chunk(row, 4 * hf + cc), v + 8 * cc);
+                if (qd < 2) {
+                    tc::tmem_ld32(tl + cAB + 64 + 32 * hf, v);
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc)
+                        st_chunk8(sPB + 8192, tc::sw128_chunk(row, 4 * hf + cc), v + 8 * cc);
+                }
+            }
+            tc::fence_proxy_async();
+            tc::fence_before_sync();
+            if (!(ok = chain_wait(B_FULLV + s, (c >> 1) & 1))) break;
+            const uint64_t dY = tc::sdesc(tc::smem_u32(sm + oV + s * kVst), 8192, 1024);   // Y^T, MN-major A
+            if (issuer) {
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16_elect(tbase + cAB, dY + (uint64_t)(ks * 128), dAtC + (uint64_t)(ks * 2), kIdVA, ks > 0);
+            }
+            // -Z~ = -(S X^T) diag(2^g) in place of the bf16 state, which (b) has finished reading
+            if (!(ok = chain_wait(B_BDONE, c & 1))) break;
+            {
+                const float *dg = sScal + u4 * 256 + 64 + 32 * hf;
+                uint32_t pk[16];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float x[16];
+                    tc::tmem_ld16(tl + cSXO + 128 * s + 32 * hf + 16 * hh, x);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 d4 = *reinterpret_cast<const float4 *>(dg + 16 * hh + 4 * q4);
+                        pk[8 * hh + 2 * q4] = pack_bf16x2(-d4.x * x[4 * q4], -d4.y * x[4 * q4 + 1]);
+                        pk[8 * hh + 2 * q4 + 1] = pack_bf16x2(-d4.z * x[4 * q4 + 2], -d4.w * x[4 * q4 + 3]);
+                    }
+                }
+                tc::tmem_st16(tl + cSR + 16 * hf, pk);
+            }
+            tc::fence_before_sync();
+            if ((ok = !named_bar_or(4, 256, false)) && issuer) {
+                tc::fence_after_sync();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16_ts_elect(tbase + cAB, tbase + cSR + 8 * ks, dAtC + (uint64_t)(ks * 2), kIdN128, true);
+                tc::mma_commit_elect(&bars[B_EFDONE]);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16_elect(tbase + cSXO + 128 * s, dY + (uint64_t)(ks * 128), dBpC + (uint64_t)(ks * 2), kIdVP, ks > 0);
+                tc::mma_commit_elect(&bars[B_VFREE + s]);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc::mma_bf16_ts_elect(tbase + cSXO + 128 * s, tbase + cSR + 8 * ks, dBpC + (uint64_t)(ks * 2), kIdN64, true);
+                tc::mma_commit_elect(&bars[B_EDONES + s]);
+            }
+            if (!ok) break;
+            if (!(ok = chain_wait(B_EFDONE, c & 1))) break;
+            {
+                const float dl = exp2f(sGL[u4]);
+                const uint32_t cds = cAB + 64 * hf;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float v[32];
+                    tc::tmem_ld32(tl + cds + 32 * hh, v);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) S[32 * hh + j] = dl * S[32 * hh + j] + v[j];
+                }
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars[B_EARDY]);          // dS read: the AB columns may take (A), (B') of the next block
+                mbar_arrive(&bars[B_SCALFREE + u4]);  // the chain's reads of the scalar slot are done
+            }
+            if (!(ok = chain_wait(B_EDONES + s, (c >> 1) & 1))) break;
+            store_S();
+            tc::fence_before_sync();
+        }
+        for (int c = 0; c < nblk && REG && !PRE; ++c) {
             const int s = c & 1, u = c % 3, u4 = c % 4;
             // (b) Z = S X^T then S Q^T -> slot s, S (bf16) from TMEM: the block's [X;Q] slot is ready (and
             // so are its decay scalars), and every chain thread's bf16 state is in TMEM (barrier).
@@ -1126,7 +1539,7 @@ chunk_ws_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             tc::mbar_wait(&bars[B_FINAL], 0, &no_abort, kDrainBudget);
             __syncwarp();
         }
-        if (REG && ok && nblk > 0 && !*abort_flag) {
+        if (REG && !PRE && ok && nblk > 0 && !*abort_flag) {
             store_out(nblk - 1);
             tc::fence_before_sync();
         }
@@ -1171,14 +1584,36 @@ cudaError_t launch_chunk_ws_w(const ChunkParams &p, cudaStream_t s) {
     if (!map_head_rows(&mK, p.k, p.T, BH, TB) || !map_head_rows(&mQ, p.q, p.T, BH, TB) ||
         !map_head_rows(&mV, p.v, p.T, BH, TB))
         return cudaErrorInvalidValue;
-    auto kern = p.regression ? chunk_ws_kernel<true, W> : chunk_ws_kernel<false, W>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+    const bool two_pass = p.tiles != nullptr && chunk_tile_bytes(p) > 0;
+    cudaError_t e;
+    auto kern = p.regression ? chunk_ws_kernel<true, W, false> : chunk_ws_kernel<false, W, false>;
+    if (two_pass) {
+        if constexpr (W == 1) {
+            const int nblk = (p.T + kBlk - 1) / kBlk;
+            e = cudaFuncSetAttribute(chunk_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLocSmem);
+            if (e != cudaSuccess) return e;
+            int dev = 0, sms = 0;
+            if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+            if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+            const long long items = BH * nblk, slots = (long long)sms * kLocCtasPerSm;
+            chunk_local_kernel<<<(unsigned)(items < slots ? items : slots), kLocThreads, kLocSmem, s>>>(mK, p, nblk);
+            kern = chunk_ws_kernel<true, W, true>;
+        }
+    }
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)BH, kThreads, kSmem, s>>>(mK, mQ, mV, p);
     return cudaGetLastError();
 }
 
 }  // namespace
+
+size_t chunk_tile_bytes(const ChunkParams &p) {
+    if (!p.regression || p.window != 1 || !chunk_ws_supported(p)) return 0;
+    const long long blocks = (long long)p.B * p.H * ((p.T + kBlk - 1) / kBlk);
+    if (blocks <= 0 || blocks > 0x7fffffffLL) return 0;
+    return (size_t)blocks * kTileBytes;
+}
 
 cudaError_t launch_chunk_ws(const ChunkParams &p, cudaStream_t s) {
     switch (p.window) {

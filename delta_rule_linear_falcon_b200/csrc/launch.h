@@ -59,6 +59,10 @@ struct ChunkParams {
     void *o, *k_last;
     float *S_out;
     int *err;
+    // Regression rules on the warp-specialised kernel: when set, a first launch writes the solved
+    // T_f and T' tiles of every block here (chunk_tile_bytes) and the chain kernel reads them instead
+    // of solving each block itself.
+    void *tiles;
     // Bounded waits of the tensor-core kernels give up after wait_budget SM clocks. A test hook
     // (falcon_debug_stall_next_call) shortens it and makes the TMA producers stop loading at
     // block dbg_stall_block, so that the timeout path runs without faulting or hanging the GPU;
@@ -79,6 +83,8 @@ cudaError_t launch_chunk(const ChunkParams &p, int num_sms, cudaStream_t s);
 // Warp-specialised tcgen05 / TMA kernel: d_k = d_v = 128, bf16 I/O, one pair per step, 64-token blocks.
 bool chunk_ws_supported(const ChunkParams &p);
 cudaError_t launch_chunk_ws(const ChunkParams &p, cudaStream_t s);
+// Workspace of the two-pass path of the regression rules (0 where it does not apply).
+size_t chunk_tile_bytes(const ChunkParams &p);
 
 // Sequence split of the inner-product rule (seg_state.cu): the segments of each head run
 // as heads of their own, started from states that a parallel pass and a scan provide.

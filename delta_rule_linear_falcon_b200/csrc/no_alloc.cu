@@ -48,14 +48,17 @@ extern "C" {
 
 FALCON_API falcon_status_t falcon_fwd_chunk_noalloc(const falcon_args_t *args, falcon_stream_t stream) {
     // Argument errors are reported by falcon_fwd_chunk itself; a size of 0 means no scratch.
+    // falcon_fwd_chunk decides what the array's size allows: a sequence split that needs more
+    // is refused before anything runs, and the regression rules' two-pass path runs only when
+    // every block's tiles fit (their single-kernel path otherwise).
     const size_t need = falcon_workspace_size(args);
     if (need == 0) return falcon_fwd_chunk(args, nullptr, 0, stream);
-    if (need > kFalconStaticScratchBytes) return FALCON_ERR_WORKSPACE;
     void *ws = scratch_on_current_device();
     if (!ws) return FALCON_ERR_CUDA;
     // Nothing in the scratch has to start at zero: every byte a call reads (the pieces'
-    // state increments and decays, the segment start states, the cached keys) is written
-    // earlier in the same call, so stale contents of a previous call are never read.
+    // state increments and decays, the segment start states, the cached keys, the blocks'
+    // tiles) is written earlier in the same call, so stale contents of a previous call are
+    // never read.
     return falcon_fwd_chunk(args, ws, kFalconStaticScratchBytes, stream);
 }
 

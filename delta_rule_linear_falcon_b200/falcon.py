@@ -180,11 +180,13 @@ def falcon_fwd_chunk(q, k, v, alpha, eta, *, rule, eps=1e-6, window=1, chunk=64,
     """Chunk-parallel forward pass. Returns (o, S_out, k_last).
 
     ``workspace`` is an optional contiguous CUDA tensor of at least
-    ``falcon_workspace_size(args)`` bytes (nonzero only where the library splits the
-    sequence of an inner-product problem with few heads); when it is needed and not
+    ``falcon_workspace_size(args)`` bytes (nonzero where the library splits the sequence of
+    an inner-product problem with few heads, and for the two-pass path of the regression
+    rules, whose blocks' solved tiles it holds); when the size is nonzero and no tensor is
     given, one is allocated here with torch for the call (on the current stream, recorded
     on ``stream`` when that is another torch stream; pass your own when ``stream`` is a raw
-    handle of a different stream)."""
+    handle of a different stream). A smaller tensor runs the regression rules in one
+    kernel."""
     o, S_out, k_last = _outputs(k, v, o, S_out, k_last, want_state)
     args = make_args(q, k, v, alpha, eta, rule=rule, eps=eps, window=window, chunk=chunk, S0=S0,
                      k_prev=k_prev, o=o, S_out=S_out, k_last=k_last)

@@ -122,13 +122,19 @@ typedef struct {
 } falcon_args_t;
 
 /*
- * Bytes of device workspace falcon_fwd_chunk needs for these arguments on the
- * current device (0 when it needs none). Returns 0 for invalid arguments as
- * well; the call itself reports those. Nonzero only for the sequence split of
- * the inner-product rules described at falcon_fwd_chunk: about
- * (B*H*T/piece + B*H*nseg) * dv*dk*4 bytes, a few tens of MB for 16 heads of
- * 32768 tokens. The caller allocates it (16-byte aligned) and owns it; the
- * call only uses it while its kernels run on `stream`.
+ * Bytes of device workspace falcon_fwd_chunk uses for these arguments on the
+ * current device (0 when it uses none). Returns 0 for invalid arguments as
+ * well; the call itself reports those. Nonzero in two cases, both described at
+ * falcon_fwd_chunk:
+ *   - the sequence split of the inner-product rules, which needs it: about
+ *     (B*H*T/piece + B*H*nseg) * dv*dk*4 bytes, a few tens of MB for 16 heads of
+ *     32768 tokens;
+ *   - the two-pass path of the regression rules (Falcon-1/3 at window 1 on the
+ *     dk = dv = 128 bf16 kernel), which is optional: 16 KB per block of 64
+ *     tokens per head, B*H*ceil(T/64)*16384 bytes (134 MB for 128 heads of 4096
+ *     tokens); given less, or NULL, those rules run in one kernel instead.
+ * The caller allocates it (16-byte aligned) and owns it; the call only uses it
+ * while its kernels run on `stream`.
  */
 FALCON_API size_t falcon_workspace_size(const falcon_args_t *args);
 
@@ -164,9 +170,18 @@ FALCON_API size_t falcon_workspace_size(const falcon_args_t *args);
  * The result is the same up to rounding; falcon_workspace_size() says when
  * this path is taken and how much workspace it needs.
  *
+ * Two-pass path (regression write, window 1, dk = dv = 128, bf16, chunk 64,
+ * when the workspace holds falcon_workspace_size() bytes): the chunk-local step
+ * of a block (its Gram matrix, step sizes, L and T = (I + L)^-1) depends only on
+ * the block's keys and gates, so a first launch solves every block of every
+ * head at once and leaves its two bf16 T tiles in the workspace; the second
+ * launch runs the state recurrence over the blocks and reads them. Both paths
+ * do the same arithmetic; with less workspace, or NULL, the single kernel runs.
+ *
  * `workspace` may be NULL when falcon_workspace_size() is 0.
  * Errors: INVALID_ARG (also a workspace not 16-byte aligned), UNSUPPORTED,
- * WORKSPACE (NULL or smaller than falcon_workspace_size()), CUDA.
+ * WORKSPACE (NULL or smaller than falcon_workspace_size() where the sequence
+ * split needs it), CUDA.
  */
 FALCON_API falcon_status_t falcon_fwd_chunk(const falcon_args_t *args, void *workspace,
                                  size_t workspace_bytes, falcon_stream_t stream);
@@ -184,12 +199,13 @@ FALCON_API falcon_status_t falcon_fwd_chunk(const falcon_args_t *args, void *wor
  * counterpart; this is a deployment convenience of this library.
  *
  * Arguments, results and errors are those of falcon_fwd_chunk. Where that call
- * needs workspace (falcon_workspace_size() > 0), this one uses a fixed array of
+ * uses workspace (falcon_workspace_size() > 0), this one uses a fixed array of
  * FALCON_NOALLOC_SCRATCH_BYTES in the library's device image instead; every
- * GPU that uses the library holds that array until the process exits. Larger
- * needs are rejected before anything runs with FALCON_ERR_WORKSPACE (use
- * falcon_fwd_chunk with your own workspace then). The call allocates and frees
- * nothing.
+ * GPU that uses the library holds that array until the process exits. A
+ * sequence split that needs more is rejected before anything runs with
+ * FALCON_ERR_WORKSPACE (use falcon_fwd_chunk with your own workspace then);
+ * the regression rules' two-pass path runs when its tiles fit in the array and
+ * their single-kernel path otherwise. The call allocates and frees nothing.
  *
  * The array is reserved on a device no later than the first call there (with
  * lazy module loading, the CUDA default, that first call loads it; with eager

@@ -20,8 +20,11 @@ pytestmark = pytest.mark.gpu
 BUDGET = 2_000_000   # SM clocks a wait may take in the stalled call (about 1 ms)
 
 CASES = {
-    # warp-specialised chunk kernel, Falcon-1: 10 blocks of 64 tokens, the 5th never loaded
+    # Falcon-1 on the two-pass path: the solve pass completes, the chain kernel's 5th of 10 blocks
+    # of 64 tokens is never loaded
     "falcon1_chunk": dict(rule=1, H=2, T=640, window=1, alpha_mu=4.0, block=4),
+    # the same on the single-kernel path (a workspace too small for the two-pass tiles)
+    "falcon1_single_kernel": dict(rule=1, H=2, T=640, window=1, alpha_mu=4.0, block=4, single=True),
     # the same kernel for the windowed rule: 20 blocks of 16 tokens (w = 4)
     "falcon3_chunk": dict(rule=3, H=2, T=320, window=4, alpha_mu=4.0, block=7),
     # Falcon-1A with few heads takes the sequence split: the state pass (seg_piece_kernel) and the
@@ -36,11 +39,13 @@ def _problem(c):
                       with_state=True, with_kprev=True)
 
 
-def _call(F, s):
+def _call(F, s, single=False):
     q, k, v = (dev(x, torch.bfloat16) for x in (s.q, s.k, s.v))
     a, e = dev(s.alpha, torch.float32), dev(s.eta, torch.float32)
     S0, kp = dev(s.S0, torch.float32), dev(s.k_prev, torch.bfloat16)
-    F.falcon_fwd_chunk(q, k, v, a, e, rule=s.rule, eps=s.eps, window=s.window, chunk=64, S0=S0, k_prev=kp)
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda") if single else None
+    F.falcon_fwd_chunk(q, k, v, a, e, rule=s.rule, eps=s.eps, window=s.window, chunk=64, S0=S0, k_prev=kp,
+                       workspace=ws)
 
 
 @pytest.mark.parametrize("name", list(CASES))
@@ -48,7 +53,7 @@ def test_stalled_load_times_out_and_the_gpu_stays_usable(F, name):
     s = _problem(CASES[name])
     assert F.falcon_check_device_errors() == F.FALCON_OK
     assert F.falcon_debug_stall_next_call(CASES[name]["block"], BUDGET) == F.FALCON_OK
-    _call(F, s)                      # launches normally; its waits run out on the device
+    _call(F, s, CASES[name].get("single", False))   # launches normally; its waits run out on the device
     torch.cuda.synchronize()         # the kernels returned
     assert F.falcon_check_device_errors() == F.FALCON_ERR_TIMEOUT
     assert F.falcon_check_device_errors() == F.FALCON_OK      # the error word was cleared

@@ -29,7 +29,8 @@ def test_split_is_chosen_only_where_it_applies(F):
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     assert _ws_bytes(F, 2, 1, 2, 4096) > 0                  # inner-product rule, few heads
     assert _ws_bytes(F, 2 | SS, 1, 2, 4096) > 0
-    assert _ws_bytes(F, 1, 1, 2, 4096) == 0                 # regression rule: no split
+    # regression rule: no split; its workspace is the two-pass path's tiles, 16 KB per block
+    assert _ws_bytes(F, 1, 1, 2, 4096) == 2 * 64 * 16384
     assert _ws_bytes(F, 2, 1, 2, 4096 + 9) == 0             # ragged length
     assert _ws_bytes(F, 2, 1, 2, 448) == 0                  # too short for two segments of 8 blocks
     assert _ws_bytes(F, 2, 1, 2, 4096, chunk=32) == 0       # not the 64-token tensor-core kernel

@@ -6,8 +6,10 @@ which a cudaMalloc could synchronise the device).
 Called through the C ABI and compared with falcon_fwd_chunk on a workspace of the
 caller's own, on two calls in a row with different inputs (the second call finds the
 first one's leftovers in the shared array), on a smaller problem without state outputs
-after a larger one, on a problem that needs no scratch, and on a
-problem whose scratch would not fit, which must be refused before anything runs. This
+after a larger one, on a problem that needs no scratch, on the regression rules' two-pass
+path with its tiles in the array and with tiles that would not fit (the single kernel runs),
+and on a sequence split whose scratch would not fit, which must be refused before anything
+runs. This
 file is collected last so that a run stopping at its first failure has run every other
 test; it passes alone in a fresh process as well.
 """
@@ -106,9 +108,30 @@ def test_noalloc_smaller_problem_without_state_after_a_larger_one(F):
 
 
 def test_noalloc_without_scratch_runs_the_plain_pass(F):
-    s = I.make_seq(1, 1, 2, 1024, 128, 128, seed=770, io_dtype="bf16", with_state=True)
+    """Falcon-1A with 15 blocks per head is too short to split: no scratch at all."""
+    s = I.make_seq(2, 1, 2, 960, 128, 128, seed=770, io_dtype="bf16", normalise_qk=False, with_state=True)
     need, ref = _run(F, s, noalloc=False)
     assert need == 0
+    _same(_run(F, s, noalloc=True)[1], ref)
+
+
+def test_noalloc_two_pass_tiles_in_the_scratch(F):
+    """Falcon-1: every block's solved tiles (16 KB per block) fit in the array, so the two-pass
+    path runs on it, and a second call with other inputs overwrites the first one's tiles."""
+    cases = [I.make_seq(1, 1, 2, 1024, 128, 128, seed=seed, io_dtype="bf16", with_state=True,
+                        with_kprev=True) for seed in (771, 772)]
+    for s in cases:
+        need, ref = _run(F, s, noalloc=False)
+        assert need == 2 * 16 * 16384
+        _same(_run(F, s, noalloc=True)[1], ref)
+
+
+def test_noalloc_two_pass_beyond_the_scratch_runs_one_kernel(F):
+    """Falcon-1 with 16 heads of 8704 tokens would need 34.8 MB of tiles: the call is not refused
+    (that workspace is optional) and runs the single-kernel path."""
+    s = I.make_seq(1, 1, 16, 8704, 128, 128, seed=773, io_dtype="bf16", with_state=True)
+    need, ref = _run(F, s, noalloc=False)
+    assert need == 16 * 136 * 16384 > SCRATCH_BYTES
     _same(_run(F, s, noalloc=True)[1], ref)
 
 
