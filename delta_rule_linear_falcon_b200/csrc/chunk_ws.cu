@@ -360,8 +360,8 @@ constexpr uint32_t kTileBytes = 16384;              // T_f then T', bf16 64 x 64
 constexpr uint32_t oLX = 0;                         // keys: 2 swizzled atoms of 64 rows
 constexpr uint32_t oLT = 16384;                     // T fp32 64 x LDF
 constexpr uint32_t oLL = oLT + 64 * LDF * 4;        // L / W fp32 64 x LDF, then the output tiles
-constexpr uint32_t oLS = oLL + 64 * LDF * 4;        // beta[64], g[64], 2^(g_last - g)[64], cf[64], carry, barrier
-constexpr uint32_t kLocSmem = oLS + 4 * 256 + 32 + 1024;   // + alignment of the base to 1024 bytes
+constexpr uint32_t oLS = oLL + 64 * LDF * 4;        // beta[64], g[64], 2^(g_last - g)[64], cf[64], carry, barriers, TMEM slot
+constexpr uint32_t kLocSmem = oLS + 4 * 256 + 64 + 1024;   // + alignment of the base to 1024 bytes
 
 // One bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) into shared memory,
 // completing on the mbarrier's transaction count.
@@ -387,16 +387,16 @@ __device__ __forceinline__ void ldsm_x4_addr(uint32_t (&r)[4], uint32_t addr) {
 
 // Pass 1 of the two-pass path of the regression rules (window 1). The chunk-local step depends only
 // on a block's keys and gates, so it runs for every block at once before any state chain starts.
-// Persistent CTAs of 128 threads walk the (head, block) items; per item they form G = X X^T (bf16
-// mma.sync, fp32 accumulation), the step sizes from its diagonal, L = diag(beta)(Gamma o G) and
+// Persistent CTAs of 128 threads walk the (head, block) items; per item they form G = X X^T on the
+// tensor cores (tcgen05, fp32 accumulation in 64 TMEM columns), the step sizes from its diagonal and
+// L = diag(beta)(Gamma o G) from the rows in registers (warps 0-1, which own TMEM lanes 0-63),
 // T = (I + L)^-1 (solve_local), and write T_f = diag(2^(g_last - g)) T diag(beta) and
 // T' = T diag(beta) as two bf16 tiles in the 128-byte swizzled order the tensor cores read, 16 KB
 // per item at tiles + (head * nblk + block) * 16 KB. The arithmetic is the one the single-kernel
 // path does on its local and helper warps. The keys of the next item are loaded by TMA (128-byte
-// swizzled, which also makes the ldmatrix reads of G conflict-free; rows before or past the sequence
-// read as zero) as soon as G of the current item has read its own, and the tiles leave by a bulk
-// copy that is only waited for before their buffer is written again, so the loads and stores of
-// one item overlap the arithmetic of the next.
+// swizzled; rows before or past the sequence read as zero) as soon as G of the current item is
+// done, and the tiles leave by a bulk copy that is only waited for before their buffer is written
+// again, so the loads and stores of one item overlap the arithmetic of the next.
 __global__ void __launch_bounds__(kLocThreads, kLocCtasPerSm)
 chunk_local_kernel(const __grid_constant__ CUtensorMap tmK, const ChunkParams p, const int nblk) {
     extern __shared__ __align__(1024) uint8_t lsm_raw[];
@@ -407,42 +407,63 @@ chunk_local_kernel(const __grid_constant__ CUtensorMap tmK, const ChunkParams p,
     uint8_t *sOut = lsm + oLL;
     float *sBeta = reinterpret_cast<float *>(lsm + oLS);
     float *sG = sBeta + 64, *sFr = sBeta + 128, *sCF = sBeta + 192, *sCarry = sBeta + 256;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sBeta + 260);
+    uint64_t *bar_k = reinterpret_cast<uint64_t *>(sBeta + 260), *bar_m = bar_k + 1;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_k + 2);
 
     const int lt = threadIdx.x, lw = lt >> 5, lane = lt & 31;
     const int T = p.T;
     const int kshift = p.same_step ? 0 : 1;
     constexpr int D = 128;
-    const long long items = (long long)p.B * p.H * nblk;
+    const int items = p.B * p.H * nblk;   // below 2^31 (the host checks the workspace size)
     const volatile int no_abort = 0;
+    // K-major [X] descriptor (128-byte swizzle, 8-row groups 1024 bytes apart); a K step of 16 moves
+    // 32 bytes inside an atom of 64 columns, the second atom is 8 KB further. With M = 128 the A
+    // operand's rows 64-127 run past the keys into the T buffer: their products land in TMEM lanes
+    // 64-127, which nothing reads.
+    const uint64_t dX = tc::sdesc(tc::smem_u32(sX), 16, 1024);
+    auto kstep = [](int ks) -> uint64_t { return (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4); };
+    constexpr uint32_t kIdG = tc::idesc_bf16(128, 64, 0, 0);
 
-    auto load_keys = [&](long long it) {   // thread 0: TMA of item it's key rows t0 - kshift ..
-        const int bh = (int)(it / nblk), c = (int)(it % nblk);
-        tc::mbar_arrive_expect_tx(bar, 16384);
-        tc::tma_load_3d(sX, &tmK, 0, c * kBlk - kshift, bh, bar);
-        tc::tma_load_3d(sX + 8192, &tmK, 64, c * kBlk - kshift, bh, bar);
+    auto load_keys = [&](int it) {   // thread 0: TMA of item it's key rows t0 - kshift ..
+        const int bh = it / nblk, c = it - bh * nblk;
+        tc::mbar_arrive_expect_tx(bar_k, 16384);
+        tc::tma_load_3d(sX, &tmK, 0, c * kBlk - kshift, bh, bar_k);
+        tc::tma_load_3d(sX + 8192, &tmK, 64, c * kBlk - kshift, bh, bar_k);
     };
     // gates of an item for the threads of rows 0..63 (alpha, eta; 1 and 0 past the sequence)
-    auto load_gates = [&](long long it, float &a, float &e) {
-        const int bh = (int)(it / nblk), c = (int)(it % nblk), t = c * kBlk + lt;
-        const bool valid = lt < 64 && it < items && t < T;
-        a = valid ? p.alpha[(size_t)bh * T + t] : 1.f;
-        e = valid ? p.eta[(size_t)bh * T + t] : 0.f;
+    auto load_gates = [&](int it, float &a, float &e) {
+        a = 1.f;
+        e = 0.f;
+        if (lt < 64 && it < items) {
+            const int bh = it / nblk, t = (it - bh * nblk) * kBlk + lt;
+            if (t < T) {
+                a = p.alpha[(size_t)bh * T + t];
+                e = p.eta[(size_t)bh * T + t];
+            }
+        }
     };
 
-    long long it = blockIdx.x;
+    int it = blockIdx.x;
     if (lt == 0) {
-        tc::mbar_init(bar, 1);
+        tc::mbar_init(bar_k, 1);
+        tc::mbar_init(bar_m, 1);
         tc::mbar_fence_init();
         if (it < items) load_keys(it);
     }
+    if (lw == 0) {
+        tc::tmem_alloc(tslot, 64);
+        tc::tmem_relinquish();
+    }
     float ga, ge;
     load_gates(it, ga, ge);
+    tc::fence_before_sync();
     __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = *tslot;
     for (uint32_t k = 0; it < items; ++k, it += gridDim.x) {
-        const int bh = (int)(it / nblk), c = (int)(it % nblk);
+        const int bh = it / nblk, c = it - bh * nblk;
         const int t0 = c * kBlk, nval = min(kBlk, T - t0);
-        const long long nx = it + gridDim.x;
+        const int nx = it + gridDim.x;
         // cumulative log2 decay of the block (rows past the sequence add nothing)
         float la = 0.f;
         if (lt < 64) {
@@ -456,116 +477,93 @@ chunk_local_kernel(const __grid_constant__ CUtensorMap tmK, const ChunkParams p,
         }
         const float ge_c = ge;
         load_gates(nx, ga, ge);   // the next item's gates, in flight during this one
-        const bool landed = tc::mbar_wait(bar, k & 1, &no_abort, kDefaultWaitBudget);
+        const bool landed = tc::mbar_wait(bar_k, k & 1, &no_abort, kDefaultWaitBudget);
         if (landed && c == 0 && kshift == 1 && p.k_prev && lt < 16) {
             // pair 0 = (k_prev, v_0): key row -1 is the cached key
             const uint4 v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(p.k_prev) +
                                                               (size_t)bh * D + lt * 8);
             *reinterpret_cast<uint4 *>(sX + (lt >> 3) * 8192 + tc::sw128_chunk(0, lt & 7)) = v;
+            tc::fence_proxy_async();   // the tensor cores read it
         }
         if (lt == 0) tc::tma_store_wait_read0();   // the previous item's tiles have left the L buffer
+        tc::fence_before_sync();
         if (__syncthreads_or(!landed)) {
             if (lt == 0) set_error(p.err, kDevErrTimeout);
             break;
         }
+        tc::fence_after_sync();
         if (lt >= 32 && lt < 64) la += sCarry[0];
         if (lt < 64) sG[lt] = la;
-
-        // G = X X^T, the 16 x 16 blocks on and below the diagonal: warp lw takes rows 16 lw .. 16 lw + 15.
-        // Lane l of an ldmatrix.x4 addresses row (l & 7) + 8 ((l >> 3) & 1) (A) or + 8 (l >> 4) (B) of
-        // its 16-row group and the 8-column chunk 2 k + (l >> 4) (A) or 2 k + ((l >> 3) & 1) (B).
-        {
-            const uint32_t xb = tc::smem_u32(sX);
-            auto chunk_addr = [&](int r, int ch) -> uint32_t {   // 16-byte chunk ch (0..15) of key row r
-                return xb + (uint32_t)((ch >> 3) * 8192 + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
-            };
-            float acc[4][2][4];
+        if (lw == 0) {   // G = X X^T -> TMEM columns 0-63, lanes 0-63
 #pragma unroll
-            for (int np = 0; np < 4; ++np)
-#pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[np][h][e] = 0.f;
-            const int ra = 16 * lw + (lane & 7) + 8 * ((lane >> 3) & 1), ca = lane >> 4;
-            const int rbo = (lane & 7) + 8 * (lane >> 4), cb = (lane >> 3) & 1;
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                uint32_t a[4];
-                ldsm_x4_addr(a, chunk_addr(ra, 2 * ks + ca));
-#pragma unroll
-                for (int np = 0; np < 4; ++np) {
-                    if (np <= lw) {
-                        uint32_t b[4];
-                        ldsm_x4_addr(b, chunk_addr(16 * np + rbo, 2 * ks + cb));
-                        mma_bf16_16816(acc[np][0], a, b[0], b[1]);
-                        mma_bf16_16816(acc[np][1], a, b[2], b[3]);
-                    }
-                }
-            }
-            const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-            for (int np = 0; np < 4; ++np) {
-                if (np <= lw) {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int col = 16 * np + 8 * h + 2 * t;
-                        *reinterpret_cast<float2 *>(sL + (16 * lw + g) * LDF + col) = make_float2(acc[np][h][0], acc[np][h][1]);
-                        *reinterpret_cast<float2 *>(sL + (16 * lw + g + 8) * LDF + col) = make_float2(acc[np][h][2], acc[np][h][3]);
-                    }
-                }
-            }
+            for (int ks = 0; ks < 8; ++ks) tc::mma_bf16_elect(tbase, dX + kstep(ks), dX + kstep(ks), kIdG, ks > 0);
+            tc::mma_commit_elect(bar_m);
         }
         __syncthreads();
-        if (lt == 0 && nx < items) {   // the keys are read: the next item's may land in their place
-            tc::fence_proxy_async();
-            load_keys(nx);
-        }
-        if (lt < 64) {   // step sizes from the key norms on the diagonal; decay tables
-            const float nrm = sL[lt * LDF + lt];
-            sBeta[lt] = lt < nval ? step_size(ge_c, nrm, p.eps) : 0.f;
+        if (lt < 64) {   // decay tables
             const float gl = sG[nval - 1];
             sFr[lt] = exp2f(gl - la);
             sCF[lt] = exp2f(sG[lt | 15] - la);
         }
-        // T starts at zero (the solve writes only the blocks on and below the diagonal)
-        for (int idx = lt; idx < 64 * LDF / 4; idx += kLocThreads)
-            reinterpret_cast<float4 *>(sT)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
-        __syncthreads();
-        {   // L = diag(beta)(Gamma o G) in place: thread (row r, half h) takes columns 32 h .. 32 h + 31
-            // (decay factors as in the single-kernel path: through the last index of a column block
-            // below the diagonal blocks, directly inside them)
-            const int r = lt >> 1, h = lt & 1, rb = r >> 4;
-            const float be = sBeta[r], gri = sG[r];
+        const bool mok = tc::mbar_wait(bar_m, k & 1, &no_abort, kDefaultWaitBudget);
+        if (lt == 0 && mok && nx < items) load_keys(nx);   // G has read the keys: the next item's may land
+        if (__syncthreads_or(!mok)) {
+            if (lt == 0) set_error(p.err, kDevErrTimeout);
+            break;
+        }
+        tc::fence_after_sync();
+        if (lw < 2) {   // G row r = lt from TMEM: step size, then L = diag(beta)(Gamma o G) row r
+            const int r = lt, rb = r >> 4;
+            float v[64];
+            {
+                float h0[32], h1[32];
+                const uint32_t tl = tbase + ((uint32_t)(32 * lw) << 16);
+                tc::tmem_ld32(tl, h0);
+                tc::tmem_ld32(tl + 32, h1);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) { v[j] = h0[j]; v[32 + j] = h1[j]; }
+            }
+            // ||x_r||^2 is the diagonal entry G[r][r] = v[32 lw + lane] (a warp-uniform branch on lw
+            // keeps v in registers)
+            const float nrm = lw == 0 ? pick_lane<0>(v, lane) : pick_lane<32>(v, lane);
+            const float be = r < nval ? step_size(ge_c, nrm, p.eps) : 0.f;
+            sBeta[r] = be;
+            // decay factors 2^(g_r - g_j), j < r: below the 16 x 16 diagonal blocks through the last
+            // index of column block jb (2^(g_r - g_{16jb+15}) cf[j]), directly inside them; entries on
+            // and above the diagonal are left as they come (the solve reads the strictly lower part)
+            const float gri = sG[r];
+            float gd[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 g4 = *reinterpret_cast<const float4 *>(sG + 16 * rb + 4 * q);
+                gd[4 * q] = be * exp2f(fminf(gri - g4.x, 0.f));
+                gd[4 * q + 1] = be * exp2f(fminf(gri - g4.y, 0.f));
+                gd[4 * q + 2] = be * exp2f(fminf(gri - g4.z, 0.f));
+                gd[4 * q + 3] = be * exp2f(fminf(gri - g4.w, 0.f));
+            }
             float *Lr = sL + r * LDF;
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const int jb = 2 * h + jj;
-                if (jb < rb) {
-                    const float fac = be * exp2f(fminf(gri - sG[16 * jb + 15], 0.f));
+            for (int jb = 0; jb < 4; ++jb) {   // the solve reads no block above the row's diagonal one
+                if (jb > rb) break;
+                const float fac = be * exp2f(fminf(gri - sG[16 * jb + 15], 0.f));
+                const bool below = jb < rb;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int j = 16 * jb + 4 * q;
-                        const float4 c4 = *reinterpret_cast<const float4 *>(sCF + j);
-                        float4 x = *reinterpret_cast<float4 *>(Lr + j);
-                        x.x *= fac * c4.x; x.y *= fac * c4.y; x.z *= fac * c4.z; x.w *= fac * c4.w;
-                        *reinterpret_cast<float4 *>(Lr + j) = x;
-                    }
-                } else if (jb == rb) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int j = 16 * jb + 4 * q;
-                        const float4 g4 = *reinterpret_cast<const float4 *>(sG + j);
-                        float4 x = *reinterpret_cast<float4 *>(Lr + j);
-                        x.x *= be * exp2f(fminf(gri - g4.x, 0.f));
-                        x.y *= be * exp2f(fminf(gri - g4.y, 0.f));
-                        x.z *= be * exp2f(fminf(gri - g4.z, 0.f));
-                        x.w *= be * exp2f(fminf(gri - g4.w, 0.f));
-                        *reinterpret_cast<float4 *>(Lr + j) = x;
-                    }
+                for (int q = 0; q < 4; ++q) {
+                    const int j = 16 * jb + 4 * q;
+                    const float4 c4 = *reinterpret_cast<const float4 *>(sCF + j);
+                    const float w0 = below ? fac * c4.x : gd[4 * q];
+                    const float w1 = below ? fac * c4.y : gd[4 * q + 1];
+                    const float w2 = below ? fac * c4.z : gd[4 * q + 2];
+                    const float w3 = below ? fac * c4.w : gd[4 * q + 3];
+                    *reinterpret_cast<float4 *>(Lr + j) =
+                        make_float4(w0 * v[j], w1 * v[j + 1], w2 * v[j + 2], w3 * v[j + 3]);
                 }
             }
         }
+        tc::fence_before_sync();
         __syncthreads();
+        // T = (I + L)^-1; its blocks above the diagonal are never written and never read (the tiles
+        // below take only the chunks on and below the diagonal)
         solve_local<true>(sL, sT, lt, lw, lane);   // ends with a barrier of all 128 threads
         {   // thread (row rr, half h) writes columns 32 h .. 32 h + 31 of both tiles: T' = T diag(beta)
             // and T_f = 2^(g_last - g_rr) T'; chunks above the diagonal are zero
@@ -600,6 +598,9 @@ chunk_local_kernel(const __grid_constant__ CUtensorMap tmK, const ChunkParams p,
         }
     }
     if (lt == 0) tc::tma_store_wait_read0();   // shared memory stays until the last copy has read it
+    tc::fence_before_sync();
+    __syncthreads();
+    if (lw == 0) tc::tmem_dealloc(tbase, 64);
 }
 
 // PRE (regression rules): T_f and T' of every block were written by chunk_local_kernel; the feed
@@ -1595,7 +1596,7 @@ cudaError_t launch_chunk_ws_w(const ChunkParams &p, cudaStream_t s) {
             int dev = 0, sms = 0;
             if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
             if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-            const long long items = BH * nblk, slots = (long long)sms * kLocCtasPerSm;
+            const long long items = BH * nblk, slots = (long long)sms * kLocCtasPerSm;   // items < 2^31
             chunk_local_kernel<<<(unsigned)(items < slots ? items : slots), kLocThreads, kLocSmem, s>>>(mK, p, nblk);
             kern = chunk_ws_kernel<true, W, true>;
         }
@@ -1611,7 +1612,7 @@ cudaError_t launch_chunk_ws_w(const ChunkParams &p, cudaStream_t s) {
 size_t chunk_tile_bytes(const ChunkParams &p) {
     if (!p.regression || p.window != 1 || !chunk_ws_supported(p)) return 0;
     const long long blocks = (long long)p.B * p.H * ((p.T + kBlk - 1) / kBlk);
-    if (blocks <= 0 || blocks > 0x7fffffffLL) return 0;
+    if (blocks <= 0 || blocks > (1LL << 30)) return 0;
     return (size_t)blocks * kTileBytes;
 }
 
