@@ -360,8 +360,8 @@ constexpr uint32_t kTileBytes = 16384;              // T_f then T', bf16 64 x 64
 constexpr uint32_t oLX = 0;                         // keys: 2 swizzled atoms of 64 rows
 constexpr uint32_t oLT = 16384;                     // T fp32 64 x LDF
 constexpr uint32_t oLL = oLT + 64 * LDF * 4;        // L / W fp32 64 x LDF, then the output tiles
-constexpr uint32_t oLS = oLL + 64 * LDF * 4;        // beta[64], g[64], 2^(g_last - g)[64], cf[64], carry, barriers, TMEM slot
-constexpr uint32_t kLocSmem = oLS + 4 * 256 + 64 + 1024;   // + alignment of the base to 1024 bytes
+constexpr uint32_t oLS = oLL + 64 * LDF * 4;        // beta[64], g[64], 2^(g_last - g)[64], cf[64], carry[36], barriers, TMEM slot
+constexpr uint32_t kLocSmem = oLS + 4 * 256 + 36 * 4 + 32 + 1024;   // + alignment of the base to 1024 bytes
 
 // One bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) into shared memory,
 // completing on the mbarrier's transaction count.
@@ -385,20 +385,24 @@ __device__ __forceinline__ void ldsm_x4_addr(uint32_t (&r)[4], uint32_t addr) {
 
 }  // namespace
 
-// Pass 1 of the two-pass path of the regression rules (window 1). The chunk-local step depends only
-// on a block's keys and gates, so it runs for every block at once before any state chain starts.
+// Pass 1 of the two-pass path of the regression rules. The chunk-local step depends only on a
+// block's keys and gates, so it runs for every block at once before any state chain starts.
 // Persistent CTAs of 128 threads walk the (head, block) items; per item they form G = X X^T on the
 // tensor cores (tcgen05, fp32 accumulation in 64 TMEM columns), the step sizes from its diagonal and
 // L = diag(beta)(Gamma o G) from the rows in registers (warps 0-1, which own TMEM lanes 0-63),
 // T = (I + L)^-1 (solve_local), and write T_f = diag(2^(g_last - g)) T diag(beta) and
 // T' = T diag(beta) as two bf16 tiles in the 128-byte swizzled order the tensor cores read, 16 KB
 // per item at tiles + (head * nblk + block) * 16 KB. The arithmetic is the one the single-kernel
-// path does on its local and helper warps. The keys of the next item are loaded by TMA (128-byte
+// path does on its local and helper warps, including the windowed layout (W pairs per step: rows in
+// m-major order, L and T in token-major order, the tiles permuted back). The keys of the next item
+// are loaded by TMA (128-byte
 // swizzled; rows before or past the sequence read as zero) as soon as G of the current item is
 // done, and the tiles leave by a bulk copy that is only waited for before their buffer is written
 // again, so the loads and stores of one item overlap the arithmetic of the next.
+template <int W>
 __global__ void __launch_bounds__(kLocThreads, kLocCtasPerSm)
 chunk_local_kernel(const __grid_constant__ CUtensorMap tmK, const ChunkParams p, const int nblk) {
+    constexpr int TB = kBlk / W;   // tokens per block
     extern __shared__ __align__(1024) uint8_t lsm_raw[];
     uint8_t *lsm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(lsm_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sX = lsm + oLX;
@@ -407,7 +411,8 @@ chunk_local_kernel(const __grid_constant__ CUtensorMap tmK, const ChunkParams p,
     uint8_t *sOut = lsm + oLL;
     float *sBeta = reinterpret_cast<float *>(lsm + oLS);
     float *sG = sBeta + 64, *sFr = sBeta + 128, *sCF = sBeta + 192, *sCarry = sBeta + 256;
-    uint64_t *bar_k = reinterpret_cast<uint64_t *>(sBeta + 260), *bar_m = bar_k + 1;
+    float *sNrm = sCF;   // windowed rules: squared key norms of the rows (the cf table is W = 1 only)
+    uint64_t *bar_k = reinterpret_cast<uint64_t *>(sBeta + 292), *bar_m = bar_k + 1;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar_k + 2);
 
     const int lt = threadIdx.x, lw = lt >> 5, lane = lt & 31;
@@ -424,18 +429,24 @@ chunk_local_kernel(const __grid_constant__ CUtensorMap tmK, const ChunkParams p,
     auto kstep = [](int ks) -> uint64_t { return (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4); };
     constexpr uint32_t kIdG = tc::idesc_bf16(128, 64, 0, 0);
 
-    auto load_keys = [&](int it) {   // thread 0: TMA of item it's key rows t0 - kshift ..
+    // thread 0: TMA of item it's keys; rows m TB .. hold the pairs t0 - m .., i.e. key rows
+    // t0 - m - kshift (W boxes of TB rows per 64-column atom)
+    auto load_keys = [&](int it) {
         const int bh = it / nblk, c = it - bh * nblk;
         tc::mbar_arrive_expect_tx(bar_k, 16384);
-        tc::tma_load_3d(sX, &tmK, 0, c * kBlk - kshift, bh, bar_k);
-        tc::tma_load_3d(sX + 8192, &tmK, 64, c * kBlk - kshift, bh, bar_k);
+#pragma unroll
+        for (int m = 0; m < W; ++m) {
+            tc::tma_load_3d(sX + m * TB * 128, &tmK, 0, c * TB - m - kshift, bh, bar_k);
+            tc::tma_load_3d(sX + 8192 + m * TB * 128, &tmK, 64, c * TB - m - kshift, bh, bar_k);
+        }
     };
-    // gates of an item for the threads of rows 0..63 (alpha, eta; 1 and 0 past the sequence)
+    // gates of an item for the threads of rows 0..63: those of the row's token r % TB (alpha, eta;
+    // 1 and 0 past the sequence)
     auto load_gates = [&](int it, float &a, float &e) {
         a = 1.f;
         e = 0.f;
         if (lt < 64 && it < items) {
-            const int bh = it / nblk, t = (it - bh * nblk) * kBlk + lt;
+            const int bh = it / nblk, t = (it - bh * nblk) * TB + lt % TB;
             if (t < T) {
                 a = p.alpha[(size_t)bh * T + t];
                 e = p.eta[(size_t)bh * T + t];
@@ -460,14 +471,21 @@ chunk_local_kernel(const __grid_constant__ CUtensorMap tmK, const ChunkParams p,
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tbase = *tslot;
+    if constexpr (W > 1) {
+        // T starts at zero once: in token-major order the solve writes only the blocks on and below
+        // the diagonal, and the permuted tiles read every entry
+        for (int idx = lt; idx < 64 * LDF / 4; idx += kLocThreads)
+            reinterpret_cast<float4 *>(sT)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     for (uint32_t k = 0; it < items; ++k, it += gridDim.x) {
         const int bh = it / nblk, c = it - bh * nblk;
-        const int t0 = c * kBlk, nval = min(kBlk, T - t0);
+        const int t0 = c * TB, nval = min(TB, T - t0);
         const int nx = it + gridDim.x;
-        // cumulative log2 decay of the block (rows past the sequence add nothing)
+        // cumulative log2 decay of the block's tokens (tokens past the sequence add nothing); for
+        // W > 1 the TB <= 32 tokens are scanned by warp 0
         float la = 0.f;
-        if (lt < 64) {
-            la = lt < nval ? log2f(ga) : 0.f;
+        if (W == 1 ? lt < 64 : lt < 32) {
+            la = (lt < TB && lt < nval) ? log2f(ga) : 0.f;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const float y = __shfl_up_sync(0xffffffffu, la, off);
@@ -478,11 +496,12 @@ chunk_local_kernel(const __grid_constant__ CUtensorMap tmK, const ChunkParams p,
         const float ge_c = ge;
         load_gates(nx, ga, ge);   // the next item's gates, in flight during this one
         const bool landed = tc::mbar_wait(bar_k, k & 1, &no_abort, kDefaultWaitBudget);
-        if (landed && c == 0 && kshift == 1 && p.k_prev && lt < 16) {
-            // pair 0 = (k_prev, v_0): key row -1 is the cached key
+        if (landed && c == 0 && kshift == 1 && p.k_prev && lt < 16 * W) {
+            // pair 0 = (k_prev, v_0) sits in row m TB + m for every m < W: its key is the cached key
+            const int m = lt >> 4, ch = lt & 15;
             const uint4 v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(p.k_prev) +
-                                                              (size_t)bh * D + lt * 8);
-            *reinterpret_cast<uint4 *>(sX + (lt >> 3) * 8192 + tc::sw128_chunk(0, lt & 7)) = v;
+                                                              (size_t)bh * D + ch * 8);
+            *reinterpret_cast<uint4 *>(sX + (ch >> 3) * 8192 + tc::sw128_chunk(m * TB + m, ch & 7)) = v;
             tc::fence_proxy_async();   // the tensor cores read it
         }
         if (lt == 0) tc::tma_store_wait_read0();   // the previous item's tiles have left the L buffer
@@ -492,8 +511,12 @@ chunk_local_kernel(const __grid_constant__ CUtensorMap tmK, const ChunkParams p,
             break;
         }
         tc::fence_after_sync();
-        if (lt >= 32 && lt < 64) la += sCarry[0];
-        if (lt < 64) sG[lt] = la;
+        if constexpr (W == 1) {
+            if (lt >= 32 && lt < 64) la += sCarry[0];
+            if (lt < 64) sG[lt] = la;
+        } else {
+            if (lt < TB) sCarry[1 + lt] = la;   // token decays g_s in sCarry[1 + s]
+        }
         if (lw == 0) {   // G = X X^T -> TMEM columns 0-63, lanes 0-63
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) tc::mma_bf16_elect(tbase, dX + kstep(ks), dX + kstep(ks), kIdG, ks > 0);
@@ -501,9 +524,15 @@ chunk_local_kernel(const __grid_constant__ CUtensorMap tmK, const ChunkParams p,
         }
         __syncthreads();
         if (lt < 64) {   // decay tables
-            const float gl = sG[nval - 1];
-            sFr[lt] = exp2f(gl - la);
-            sCF[lt] = exp2f(sG[lt | 15] - la);
+            if constexpr (W == 1) {
+                const float gl = sG[nval - 1];
+                sFr[lt] = exp2f(gl - la);
+                sCF[lt] = exp2f(sG[lt | 15] - la);
+            } else {   // every row takes its token's decay
+                const float g = sCarry[1 + lt % TB], gl = sCarry[nval];
+                sG[lt] = g;
+                sFr[lt] = exp2f(gl - g);
+            }
         }
         const bool mok = tc::mbar_wait(bar_m, k & 1, &no_abort, kDefaultWaitBudget);
         if (lt == 0 && mok && nx < items) load_keys(nx);   // G has read the keys: the next item's may land
@@ -525,9 +554,36 @@ chunk_local_kernel(const __grid_constant__ CUtensorMap tmK, const ChunkParams p,
             }
             // ||x_r||^2 is the diagonal entry G[r][r] = v[32 lw + lane] (a warp-uniform branch on lw
             // keeps v in registers)
-            const float nrm = lw == 0 ? pick_lane<0>(v, lane) : pick_lane<32>(v, lane);
-            const float be = r < nval ? step_size(ge_c, nrm, p.eps) : 0.f;
+            float nrm = lw == 0 ? pick_lane<0>(v, lane) : pick_lane<32>(v, lane);
+            if constexpr (W > 1) {   // the token's window: rows m TB + r % TB, m < W
+                sNrm[r] = nrm;
+                named_bar(3, 64);
+                nrm = 0.f;
+#pragma unroll
+                for (int m = 0; m < W; ++m) nrm += sNrm[m * TB + r % TB];
+            }
+            const float be = r % TB < nval ? step_size(ge_c, nrm, p.eps) : 0.f;
             sBeta[r] = be;
+          if constexpr (W > 1) {
+            // row u = s W + m of L in token-major order (s = r % TB, m = r / TB) couples to the rows of
+            // earlier tokens s' < s only: L[u][s' W + m'] = beta 2^(g_s - g_s') G[r][m' TB + s']
+            const int rs = r % TB;
+            const float gri = sG[r];
+            float gd[TB];
+#pragma unroll
+            for (int sp = 0; sp < TB; ++sp) gd[sp] = sp < rs ? be * exp2f(fminf(gri - sG[sp], 0.f)) : 0.f;
+            float *Lr = sL + (rs * W + r / TB) * LDF;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                float w4[4];
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const int up = 4 * q + kk, sp = up / W, mp = up % W;
+                    w4[kk] = gd[sp] * v[mp * TB + sp];
+                }
+                *reinterpret_cast<float4 *>(Lr + 4 * q) = make_float4(w4[0], w4[1], w4[2], w4[3]);
+            }
+          } else {
             // decay factors 2^(g_r - g_j), j < r: below the 16 x 16 diagonal blocks through the last
             // index of column block jb (2^(g_r - g_{16jb+15}) cf[j]), directly inside them; entries on
             // and above the diagonal are left as they come (the solve reads the strictly lower part)
@@ -559,27 +615,39 @@ chunk_local_kernel(const __grid_constant__ CUtensorMap tmK, const ChunkParams p,
                         make_float4(w0 * v[j], w1 * v[j + 1], w2 * v[j + 2], w3 * v[j + 3]);
                 }
             }
+          }
         }
         tc::fence_before_sync();
         __syncthreads();
         // T = (I + L)^-1; its blocks above the diagonal are never written and never read (the tiles
         // below take only the chunks on and below the diagonal)
         solve_local<true>(sL, sT, lt, lw, lane);   // ends with a barrier of all 128 threads
-        {   // thread (row rr, half h) writes columns 32 h .. 32 h + 31 of both tiles: T' = T diag(beta)
-            // and T_f = 2^(g_last - g_rr) T'; chunks above the diagonal are zero
+        {   // thread (row rr, half h) writes columns 32 h .. 32 h + 31 of both tiles (m-major order):
+            // T' = T diag(beta) and T_f = 2^(g_last - g) T'; for W = 1 the chunks above the diagonal
+            // are zero, for W > 1 T is read in token-major order (row rr is token-major row
+            // (rr % TB) W + rr / TB; the eight columns j0.. of a chunk share m' = j0 / TB and take
+            // tokens j0 % TB + k, a stride of W)
             const int rr = lt >> 1, h = lt & 1;
             const float fr = sFr[rr];
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
                 const int cc = 4 * h + k4, j0 = 8 * cc;
                 float t8[8], f8[8];
-                if (j0 <= rr) {
-                    const float4 x0 = *reinterpret_cast<const float4 *>(sT + rr * LDF + j0);
-                    const float4 x1 = *reinterpret_cast<const float4 *>(sT + rr * LDF + j0 + 4);
+                if (W > 1 || j0 <= rr) {
+                    if constexpr (W == 1) {
+                        const float4 x0 = *reinterpret_cast<const float4 *>(sT + rr * LDF + j0);
+                        const float4 x1 = *reinterpret_cast<const float4 *>(sT + rr * LDF + j0 + 4);
+                        t8[0] = x0.x; t8[1] = x0.y; t8[2] = x0.z; t8[3] = x0.w;
+                        t8[4] = x1.x; t8[5] = x1.y; t8[6] = x1.z; t8[7] = x1.w;
+                    } else {
+                        const float *Trow = sT + ((rr % TB) * W + rr / TB) * LDF + (j0 % TB) * W + j0 / TB;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) t8[q] = Trow[q * W];
+                    }
                     const float4 b0 = *reinterpret_cast<const float4 *>(sBeta + j0);
                     const float4 b1 = *reinterpret_cast<const float4 *>(sBeta + j0 + 4);
-                    t8[0] = x0.x * b0.x; t8[1] = x0.y * b0.y; t8[2] = x0.z * b0.z; t8[3] = x0.w * b0.w;
-                    t8[4] = x1.x * b1.x; t8[5] = x1.y * b1.y; t8[6] = x1.z * b1.z; t8[7] = x1.w * b1.w;
+                    t8[0] *= b0.x; t8[1] *= b0.y; t8[2] *= b0.z; t8[3] *= b0.w;
+                    t8[4] *= b1.x; t8[5] *= b1.y; t8[6] *= b1.z; t8[7] *= b1.w;
 #pragma unroll
                     for (int q = 0; q < 8; ++q) f8[q] = fr * t8[q];
                 } else {
@@ -1589,15 +1657,15 @@ cudaError_t launch_chunk_ws_w(const ChunkParams &p, cudaStream_t s) {
     cudaError_t e;
     auto kern = p.regression ? chunk_ws_kernel<true, W, false> : chunk_ws_kernel<false, W, false>;
     if (two_pass) {
-        if constexpr (W == 1) {
-            const int nblk = (p.T + kBlk - 1) / kBlk;
-            e = cudaFuncSetAttribute(chunk_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLocSmem);
+        {
+            const int nblk = (p.T + TB - 1) / TB;
+            e = cudaFuncSetAttribute(chunk_local_kernel<W>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLocSmem);
             if (e != cudaSuccess) return e;
             int dev = 0, sms = 0;
             if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
             if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
             const long long items = BH * nblk, slots = (long long)sms * kLocCtasPerSm;   // items < 2^31
-            chunk_local_kernel<<<(unsigned)(items < slots ? items : slots), kLocThreads, kLocSmem, s>>>(mK, p, nblk);
+            chunk_local_kernel<W><<<(unsigned)(items < slots ? items : slots), kLocThreads, kLocSmem, s>>>(mK, p, nblk);
             kern = chunk_ws_kernel<true, W, true>;
         }
     }
@@ -1610,8 +1678,9 @@ cudaError_t launch_chunk_ws_w(const ChunkParams &p, cudaStream_t s) {
 }  // namespace
 
 size_t chunk_tile_bytes(const ChunkParams &p) {
-    if (!p.regression || p.window != 1 || !chunk_ws_supported(p)) return 0;
-    const long long blocks = (long long)p.B * p.H * ((p.T + kBlk - 1) / kBlk);
+    if (!p.regression || !chunk_ws_supported(p)) return 0;
+    const int tb = kBlk / p.window;   // tokens per block
+    const long long blocks = (long long)p.B * p.H * ((p.T + tb - 1) / tb);
     if (blocks <= 0 || blocks > (1LL << 30)) return 0;
     return (size_t)blocks * kTileBytes;
 }

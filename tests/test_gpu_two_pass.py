@@ -2,8 +2,9 @@
 every block's solved tiles) against the single-kernel path (a smaller workspace) and the fp64
 oracle: both paths within the bf16 tolerance of the oracle and within a small fraction of it of
 each other, over several blocks with a ragged tail, lengths around one block, an initial state
-and a cached key, the same-step flag, Falcon-3 at window 1, strong and tiny decays, and the
-benchmark workload at full size."""
+and a cached key, the same-step flag, Falcon-3 at windows 1, 2 and 4 (the windowed layout:
+rows in m-major order, the solve in token-major order), strong and tiny decays, and the
+Falcon-1 and Falcon-3 benchmark workloads at full size."""
 import ctypes
 
 import numpy as np
@@ -51,13 +52,14 @@ def _check(s, out, heads=None):
     assert np.array_equal(k1, k2)
 
 
-@pytest.mark.parametrize("rule", [1, 3, 1 | SS])
-@pytest.mark.parametrize("T", [1, 63, 64, 65, 201, 640])
-def test_two_pass_matches_single_kernel_and_oracle(F, rule, T):
-    s = I.make_seq(rule, 2, 3, T, 128, 128, seed=1100 + T + rule, io_dtype="bf16", window=1,
+@pytest.mark.parametrize("rule,w", [(1, 1), (3, 1), (1 | SS, 1), (3, 2), (3, 4), (3 | SS, 4)])
+@pytest.mark.parametrize("T", [1, 2, 5, 15, 16, 17, 63, 64, 65, 201, 640])
+def test_two_pass_matches_single_kernel_and_oracle(F, rule, w, T):
+    s = I.make_seq(rule, 2, 3, T, 128, 128, seed=1100 + T + rule + 7 * w, io_dtype="bf16", window=w,
                    with_state=True, with_kprev=True)
     need, out = _both(F, s)
-    assert need == 2 * 3 * ((T + 63) // 64) * 16384
+    tb = 64 // w
+    assert need == 2 * 3 * ((T + tb - 1) // tb) * 16384
     _check(s, out)
 
 
@@ -89,7 +91,9 @@ def test_two_pass_workspace_sizes(F):
     assert size(1, 2, 3, 130, 128) == 2 * 3 * 3 * 16384
     assert size(3, 1, 2, 64, 128, window=1) == 2 * 16384
     assert size(1 | SS, 1, 1, 65, 128) == 2 * 16384
-    assert size(3, 1, 2, 256, 128, window=4) == 0     # windowed: the single kernel solves in place
+    assert size(3, 1, 2, 256, 128, window=4) == 2 * 16 * 16384   # 16 tokens per block
+    assert size(3, 1, 2, 100, 128, window=2) == 2 * 4 * 16384     # 32 tokens per block
+    assert size(3, 1, 2, 256, 128, window=3) == 0     # w = 3: the mma.sync kernel
     assert size(1, 1, 2, 256, 64) == 0                # d = 64: the mma.sync kernel
     assert size(1, 1, 2, 256, 128, chunk=32) == 0
     assert size(4, 1, 2, 256, 128, window=1) == 0     # inner-product rules have no solve
@@ -111,3 +115,20 @@ def test_two_pass_full_benchmark_workload(F):
     for o, S in ((o1, S1), (o2, S2)):
         assert relerr(o[b, h][None], ref[0]) <= TOL_BF16
         assert relerr(S[b, h][None], ref[1]) <= TOL_BF16
+
+
+def test_two_pass_full_falcon3_workload(F):
+    """Falcon-3 (w = 4) at B4 H16 T8192 d128: both paths over all heads against each other, 16 sampled
+    heads of the two-pass result against the oracle."""
+    s = _full("f3")
+    need, out = _both(F, s)
+    assert need == 4 * 16 * 512 * 16384
+    (o1, S1, k1), (o2, S2, k2) = out["two_pass"], out["single"]
+    assert relerr(o1, o2) <= TOL_PATHS and relerr(S1, S2) <= TOL_PATHS and np.array_equal(k1, k2)
+    pairs = _spread_heads(4, 16)
+    b = np.array([p[0] for p in pairs])
+    h = np.array([p[1] for p in pairs])
+    g = _gather(s, pairs)
+    ref = run_oracle(g)
+    assert relerr(o1[b, h][None], ref[0]) <= TOL_BF16
+    assert relerr(S1[b, h][None], ref[1]) <= TOL_BF16
