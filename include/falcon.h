@@ -129,10 +129,11 @@ typedef struct {
  *   - the sequence split of the inner-product rules, which needs it: about
  *     (B*H*T/piece + B*H*nseg) * dv*dk*4 bytes, a few tens of MB for 16 heads of
  *     32768 tokens;
- *   - the two-pass path of the regression rules (Falcon-1/3 at window 1 on the
- *     dk = dv = 128 bf16 kernel), which is optional: 16 KB per block of 64
- *     tokens per head, B*H*ceil(T/64)*16384 bytes (134 MB for 128 heads of 4096
- *     tokens); given less, or NULL, those rules run in one kernel instead.
+ *   - the two-pass path of the regression rules (Falcon-1, and Falcon-3 at
+ *     window 1, 2 or 4, on the dk = dv = 128 bf16 kernel), which is optional:
+ *     16 KB per block of 64 / window tokens per head, B*H*ceil(T*window/64)*16384
+ *     bytes (134 MB for 128 heads of 4096 tokens at window 1); given less, or
+ *     NULL, those rules run in one kernel instead.
  * The caller allocates it (16-byte aligned) and owns it; the call only uses it
  * while its kernels run on `stream`.
  */
@@ -170,8 +171,8 @@ FALCON_API size_t falcon_workspace_size(const falcon_args_t *args);
  * The result is the same up to rounding; falcon_workspace_size() says when
  * this path is taken and how much workspace it needs.
  *
- * Two-pass path (regression write, window 1, dk = dv = 128, bf16, chunk 64,
- * when the workspace holds falcon_workspace_size() bytes): the chunk-local step
+ * Two-pass path (regression write, window 1, 2 or 4, dk = dv = 128, bf16, chunk
+ * 64, when the workspace holds falcon_workspace_size() bytes): the chunk-local step
  * of a block (its Gram matrix, step sizes, L and T = (I + L)^-1) depends only on
  * the block's keys and gates, so a first launch solves every block of every
  * head at once and leaves its two bf16 T tiles in the workspace; the second
