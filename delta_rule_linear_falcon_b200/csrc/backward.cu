@@ -165,6 +165,44 @@ bwd_recurrent_kernel(BwdParams p) {
         for (int i = warp; i < dv; i += kBwdWarps)
             for (int c = lane; c < dk; c += 32) dst[i * LD + c] = src ? src[(size_t)i * dk + c] : 0.f;
     };
+    // The states the kernel keeps in its workspace (16-byte aligned, d_k a multiple of 4) move as
+    // 16-byte words, with a batch of loads in flight per thread before any is stored: one memory
+    // latency per state rather than one per row.
+    const bool vec = (dk & 3) == 0;
+    const int q4 = dk >> 2, n4 = dv * q4;
+    constexpr int kBatch = 4;
+    auto load_ws_state = [&](float *dst, const float *src) {
+        if (!vec) {
+            load_state(dst, src);
+            return;
+        }
+        for (int base = tid; base < n4; base += kBwdThreads * kBatch) {
+            float4 r[kBatch];
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+                const int e = base + b * kBwdThreads;
+                if (e < n4) r[b] = reinterpret_cast<const float4 *>(src)[e];
+            }
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+                const int e = base + b * kBwdThreads;
+                if (e < n4) {
+                    const int i = e / q4, c4 = e - i * q4;
+                    *reinterpret_cast<float4 *>(dst + i * LD + 4 * c4) = r[b];
+                }
+            }
+        }
+    };
+    auto store_ws_state = [&](float *dst, const float *src) {
+        if (!vec) {
+            store_state(dst, src);
+            return;
+        }
+        for (int e = tid; e < n4; e += kBwdThreads) {
+            const int i = e / q4, c4 = e - i * q4;
+            reinterpret_cast<float4 *>(dst)[e] = *reinterpret_cast<const float4 *>(src + i * LD + 4 * c4);
+        }
+    };
     // beta of step t from the staged keys (every thread gets it) and its denominator
     auto step_beta = [&](long t, float &beta, float &den) {
         float part = 0.f;
@@ -214,7 +252,7 @@ bwd_recurrent_kernel(BwdParams p) {
     load_state(sP, p.S0 ? p.S0 + bh * DD : nullptr);
     for (int s = 0; s < nseg; ++s) {
         __syncthreads();
-        store_state(ckpt + (size_t)s * DD, sP);
+        store_ws_state(ckpt + (size_t)s * DD, sP);
         if (s + 1 == nseg) break;
         for (long t = (long)s * C; t < (long)(s + 1) * C; ++t) forward_step(t);
     }
@@ -224,20 +262,20 @@ bwd_recurrent_kernel(BwdParams p) {
     for (int s = nseg - 1; s >= 0; --s) {
         const long t0 = (long)s * C, t1 = min((long)T, t0 + C);
         __syncthreads();
-        load_state(sP, ckpt + (size_t)s * DD);
+        load_ws_state(sP, ckpt + (size_t)s * DD);
         __syncthreads();
-        store_state(buf, sP);
+        store_ws_state(buf, sP);
         for (long t = t0; t < t1; ++t) {
             forward_step(t);
             __syncthreads();
-            store_state(buf + (size_t)(t - t0 + 1) * DD, sP);
+            store_ws_state(buf + (size_t)(t - t0 + 1) * DD, sP);
         }
         // sA = state after the last step of the segment
         __syncthreads();
-        load_state(sA, buf + (size_t)(t1 - t0) * DD);
+        load_ws_state(sA, buf + (size_t)(t1 - t0) * DD);
         for (long t = t1 - 1; t >= t0; --t) {
             __syncthreads();
-            load_state(sP, buf + (size_t)(t - t0) * DD);   // state before step t
+            load_ws_state(sP, buf + (size_t)(t - t0) * DD);   // state before step t
             ctx.stage_pairs(sX, sY, t);
             for (int c = tid; c < dk; c += kBwdThreads) sQ[c] = Io<IO>::ld(q, (size_t)t * dk + c);
             for (int i = tid; i < dv; i += kBwdThreads) sG[i] = dO[(size_t)t * dv + i];
@@ -286,7 +324,11 @@ bwd_recurrent_kernel(BwdParams p) {
                     const float ux = sUx[(size_t)m * dv + ri];
                     if (REG) sDr[(size_t)m * dv + ri] = -beta * ux;
                     const long j = t - m;
-                    if (j >= 0) gv[(size_t)j * dv + ri] += beta * ux;   // dy = -dr (regression) = beta U x
+                    // dy = -dr (regression) = beta U x; with one pair per step a value row has one term
+                    if (j >= 0) {
+                        if (w == 1) gv[(size_t)j * dv + ri] = beta * ux;
+                        else gv[(size_t)j * dv + ri] += beta * ux;
+                    }
                 }
             __syncthreads();
             // columns: dq_t = S_t^T dO_t; dx_m (scattered to the key row of pair j)
@@ -323,9 +365,12 @@ bwd_recurrent_kernel(BwdParams p) {
                 const float dx = fmaf(2.f * dN, sX[(size_t)m * dk + c], v);
                 const long j = t - m;
                 if (j < 0) continue;
-                if (ctx.same) gk[(size_t)j * dk + c] += dx;
-                else if (j >= 1) gk[(size_t)(j - 1) * dk + c] += dx;
-                else if (gkp) gkp[c] += dx;
+                // with one pair per step a key row has one term (no read of the zero it starts from)
+                float *dst = ctx.same ? gk + (size_t)j * dk + c
+                                      : (j >= 1 ? gk + (size_t)(j - 1) * dk + c : gkp ? gkp + c : nullptr);
+                if (!dst) continue;
+                if (w == 1) *dst = dx;
+                else *dst += dx;
             }
             __syncthreads();
             // rows: dSbar = U + sum_m dr_m x_m^T; dalpha = <dSbar, S_{t-1}>; U <- alpha dSbar
