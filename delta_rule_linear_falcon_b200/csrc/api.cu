@@ -239,6 +239,7 @@ falcon_status_t check_bwd_args(const falcon_args_t *a) {
     if (is_per_column(a->rule)) return FALCON_ERR_UNSUPPORTED;
     if (a->dk > 128 || a->dv > 128) return FALCON_ERR_UNSUPPORTED;
     const int w = is_windowed(a->rule) ? a->window : 1;
+    if (w > 8) return FALCON_ERR_UNSUPPORTED;   // the step inputs held in registers
     if (bwd_smem_bytes(a->dk, a->dv, w) > 232448) return FALCON_ERR_UNSUPPORTED;
     return FALCON_OK;
 }

@@ -40,6 +40,7 @@ namespace {
 constexpr int kBwdThreads = 512;
 constexpr int kBwdWarps = kBwdThreads / 32;
 constexpr int kRowGroups = kBwdThreads / 128;   // column products: four row groups of 128 columns
+constexpr int kBwdMaxWindow = 8;                // pairs per step the register prefetch holds
 
 struct BwdSmem {
     int LD, dk, dv, w;
@@ -103,6 +104,13 @@ struct BwdCtx {
             else if (kp) { src = kp; base = 0; }
         }
         for (int c = tid; c < dk; c += kBwdThreads) dst[c] = src ? Io<IO>::ld(src, base + c) : 0.f;
+    }
+    // element c of the key row of pair j (0 for j < 0, or for the first pair without k_prev)
+    __device__ float key_elem(long j, int c) const {
+        if (j < 0) return 0.f;
+        if (same) return Io<IO>::ld(k, (size_t)j * dk + c);
+        if (j >= 1) return Io<IO>::ld(k, (size_t)(j - 1) * dk + c);
+        return kp ? Io<IO>::ld(kp, c) : 0.f;
     }
     // stage the w pairs of step t (keys, values) into shared memory
     __device__ void stage_pairs(float *sX, float *sY, long t) const {
@@ -203,22 +211,61 @@ bwd_recurrent_kernel(BwdParams p) {
             reinterpret_cast<float4 *>(dst)[e] = *reinterpret_cast<const float4 *>(src + i * LD + 4 * c4);
         }
     };
-    // beta of step t from the staged keys (every thread gets it) and its denominator
-    auto step_beta = [&](long t, float &beta, float &den) {
+    // The inputs of a step, loaded one step ahead into registers (thread tid < dk holds key and
+    // query element tid, tid < dv value and dO element tid; d_k, d_v <= 128 < 512 threads), so
+    // that their memory latency overlaps the step before instead of sitting on the chain of steps.
+    struct StepIn {
+        float a, e, q, g, x[kBwdMaxWindow], y[kBwdMaxWindow];
+    };
+    auto fetch = [&](long t, StepIn &in, bool qg) {
+        in.a = 1.f; in.e = 0.f; in.q = 0.f; in.g = 0.f;
+#pragma unroll
+        for (int m = 0; m < kBwdMaxWindow; ++m) in.x[m] = in.y[m] = 0.f;
+        if (t < 0 || t >= T) return;
+        in.a = ctx.al[t];
+        in.e = ctx.et[t];
+        if (qg) {
+            if (tid < dk) in.q = Io<IO>::ld(q, (size_t)t * dk + tid);
+            if (tid < dv) in.g = dO[(size_t)t * dv + tid];
+        }
+#pragma unroll
+        for (int m = 0; m < kBwdMaxWindow; ++m) {
+            if (m < w) {
+                const long j = t - m;
+                if (tid < dk) in.x[m] = ctx.key_elem(j, tid);
+                if (tid < dv && j >= 0) in.y[m] = Io<IO>::ld(ctx.v, (size_t)j * dv + tid);
+            }
+        }
+    };
+    auto commit = [&](const StepIn &in, bool qg) {   // into sX, sY (and sQ, sG)
+#pragma unroll
+        for (int m = 0; m < kBwdMaxWindow; ++m) {
+            if (m < w) {
+                if (tid < dk) sX[(size_t)m * dk + tid] = in.x[m];
+                if (tid < dv) sY[(size_t)m * dv + tid] = in.y[m];
+            }
+        }
+        if (qg) {
+            if (tid < dk) sQ[tid] = in.q;
+            if (tid < dv) sG[tid] = in.g;
+        }
+    };
+    // beta of a step from the staged keys (every thread gets it) and its denominator
+    auto step_beta = [&](float eta_t, float &beta, float &den) {
         float part = 0.f;
         for (int e = tid; e < w * dk; e += kBwdThreads) part += sX[e] * sX[e];
         const float n = block_sum(part, sRed);
         den = n + p.eps;
-        beta = den > 0.f ? ctx.et[t] / den : 0.f;
+        beta = den > 0.f ? eta_t / den : 0.f;
     };
     // one forward step on the state in sP (padded rows), in place
-    auto forward_step = [&](long t) {
+    auto forward_step = [&](const StepIn &in) {
         __syncthreads();                   // sX / sY and sP are free
-        ctx.stage_pairs(sX, sY, t);
+        commit(in, false);
         __syncthreads();
         float beta, den;
-        step_beta(t, beta, den);
-        const float a = ctx.al[t];
+        step_beta(in.e, beta, den);
+        const float a = in.a;
         float *Si = sP + (size_t)(rok ? ri : 0) * LD;
         if (rok)
             for (int c = rq; c < dk; c += 4) Si[c] *= a;
@@ -250,11 +297,17 @@ bwd_recurrent_kernel(BwdParams p) {
 
     // ---- pass 1: checkpoints S_{s C}, s = 0 .. nseg-1
     load_state(sP, p.S0 ? p.S0 + bh * DD : nullptr);
+    StepIn cur, nxt;
+    fetch(0, cur, false);
     for (int s = 0; s < nseg; ++s) {
         __syncthreads();
         store_ws_state(ckpt + (size_t)s * DD, sP);
         if (s + 1 == nseg) break;
-        for (long t = (long)s * C; t < (long)(s + 1) * C; ++t) forward_step(t);
+        for (long t = (long)s * C; t < (long)(s + 1) * C; ++t) {
+            fetch(t + 1, nxt, false);
+            forward_step(cur);
+            cur = nxt;
+        }
     }
 
     // ---- reverse sweep, segment by segment
@@ -265,24 +318,27 @@ bwd_recurrent_kernel(BwdParams p) {
         load_ws_state(sP, ckpt + (size_t)s * DD);
         __syncthreads();
         store_ws_state(buf, sP);
+        fetch(t0, cur, false);
         for (long t = t0; t < t1; ++t) {
-            forward_step(t);
+            fetch(t + 1 < t1 ? t + 1 : -1, nxt, false);
+            forward_step(cur);
             __syncthreads();
             store_ws_state(buf + (size_t)(t - t0 + 1) * DD, sP);
+            cur = nxt;
         }
         // sA = state after the last step of the segment
         __syncthreads();
         load_ws_state(sA, buf + (size_t)(t1 - t0) * DD);
+        fetch(t1 - 1, cur, true);
         for (long t = t1 - 1; t >= t0; --t) {
+            fetch(t - 1 >= t0 ? t - 1 : -1, nxt, true);
             __syncthreads();
             load_ws_state(sP, buf + (size_t)(t - t0) * DD);   // state before step t
-            ctx.stage_pairs(sX, sY, t);
-            for (int c = tid; c < dk; c += kBwdThreads) sQ[c] = Io<IO>::ld(q, (size_t)t * dk + c);
-            for (int i = tid; i < dv; i += kBwdThreads) sG[i] = dO[(size_t)t * dv + i];
+            commit(cur, true);
             __syncthreads();
             float beta, den;
-            step_beta(t, beta, den);
-            const float a = ctx.al[t];
+            step_beta(cur.e, beta, den);
+            const float a = cur.a;
             // rows: U += dO q^T; U x_m; residuals r_m at the decayed state
             float part = 0.f;
             {
@@ -390,6 +446,7 @@ bwd_recurrent_kernel(BwdParams p) {
             if (tid == 0) gal[t] = dal;
             // the state before step t is the state after step t - 1
             float *tmp = sA; sA = sP; sP = tmp;
+            cur = nxt;
         }
     }
     __syncthreads();

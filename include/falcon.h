@@ -258,7 +258,7 @@ FALCON_API falcon_status_t falcon_fwd_recurrent(const falcon_args_t *args, falco
  * start of every segment of about sqrt(T) steps and one segment of recomputed states,
  * fp32, per head). fp32 state and arithmetic; one CTA of 512 threads per (b, h).
  * Supported: Falcon-1, 1A, 3, 3A (with or without FALCON_SAME_STEP); 1 <= dk, dv <= 128;
- * windows whose staging fits in shared memory (w <= 5 at dk = dv = 128). Falcon-2/2A return
+ * windows up to 8 whose staging fits in shared memory (w <= 5 at dk = dv = 128). Falcon-2/2A return
  * UNSUPPORTED.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  */

@@ -157,6 +157,7 @@ def _grads(**kw):
     (dict(dk=129), {}, 1 << 30, F.FALCON_ERR_UNSUPPORTED),
     (dict(dv=256), {}, 1 << 30, F.FALCON_ERR_UNSUPPORTED),
     (dict(rule=3, window=16), {}, 1 << 30, F.FALCON_ERR_UNSUPPORTED),   # window staging too large
+    (dict(rule=3, window=9, dk=16, dv=16), {}, 1 << 30, F.FALCON_ERR_UNSUPPORTED),   # above 8 pairs
     (dict(rule=3, window=0), {}, 1 << 30, F.FALCON_ERR_INVALID_ARG),
     (dict(q=None), {}, 1 << 30, F.FALCON_ERR_INVALID_ARG),
     (dict(eps=-1.0), {}, 1 << 30, F.FALCON_ERR_INVALID_ARG),
