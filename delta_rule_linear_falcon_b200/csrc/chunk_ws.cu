@@ -54,6 +54,13 @@
 // into that order for the solve and permute T back to m-major order for the MMAs. P~ masks
 // by token (a query reads the pairs of its own and earlier tokens); only the TB query rows
 // are loaded and only TB outputs are written per block.
+//
+// Two-pass path (regression rules, given a workspace of 16 KB per block and head). The solve
+// does not depend on the state, so chunk_local_kernel runs it for every block of every head
+// at once and writes T_f and T' (bf16, in the order the tensor cores read them) to the
+// workspace. The chain kernel then runs with PRE set: the feed warp brings each block's tiles
+// into a two-slot ring with one bulk copy, the helpers only prepare the decays and P~, and the
+// local warps, with no solve left, store the outputs of each block instead of the chain.
 #include <cuda.h>
 
 #include "chunk_mma.cuh"
