@@ -634,7 +634,10 @@ chunk_local_kernel(const __grid_constant__ CUtensorMap tmK, const ChunkParams p,
             // are zero, for W > 1 T is read in token-major order (row rr is token-major row
             // (rr % TB) W + rr / TB; the eight columns j0.. of a chunk share m' = j0 / TB and take
             // tokens j0 % TB + k, a stride of W)
-            const int rr = lt >> 1, h = lt & 1;
+            // for W > 1 a warp's 16 rows are taken from all W slots m (rr = m TB + s), so that their
+            // token-major rows s W + m fall on different banks
+            const int ix = lt >> 1, h = lt & 1;
+            const int rr = W == 1 ? ix : (ix % W) * TB + ix / W;
             const float fr = sFr[rr];
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
