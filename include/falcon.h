@@ -256,9 +256,13 @@ FALCON_API falcon_status_t falcon_fwd_recurrent(const falcon_args_t *args, falco
  *   args->k_prev is given.
  * Workspace: falcon_bwd_workspace_size(args) bytes, 16-byte aligned (the states at the
  * start of every segment of about sqrt(T) steps and one segment of recomputed states,
- * fp32, per head). fp32 state and arithmetic; one CTA of 512 threads per (b, h).
+ * fp32, per slice of 32 value rows of a head). fp32 state and arithmetic; one CTA of 128
+ * threads per slice of 32 value rows of a (b, h): the rows of S evolve independently, and the
+ * slices add their parts of dq, dk, dalpha, deta and dk_prev to the outputs with atomic adds
+ * (so those sums are taken in no fixed order, and their last bits can differ between runs);
+ * dv and dS0 rows are each written by one slice.
  * Supported: Falcon-1, 1A, 3, 3A (with or without FALCON_SAME_STEP); 1 <= dk, dv <= 128;
- * windows up to 8 whose staging fits in shared memory (w <= 5 at dk = dv = 128). Falcon-2/2A return
+ * windows of up to 8 pairs. Falcon-2/2A return
  * UNSUPPORTED.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  */

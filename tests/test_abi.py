@@ -156,7 +156,7 @@ def _grads(**kw):
     (dict(rule=6 | 0x100), {}, 1 << 30, F.FALCON_ERR_UNSUPPORTED),
     (dict(dk=129), {}, 1 << 30, F.FALCON_ERR_UNSUPPORTED),
     (dict(dv=256), {}, 1 << 30, F.FALCON_ERR_UNSUPPORTED),
-    (dict(rule=3, window=16), {}, 1 << 30, F.FALCON_ERR_UNSUPPORTED),   # window staging too large
+    (dict(rule=3, window=16), {}, 1 << 30, F.FALCON_ERR_UNSUPPORTED),   # more pairs than the step inputs hold
     (dict(rule=3, window=9, dk=16, dv=16), {}, 1 << 30, F.FALCON_ERR_UNSUPPORTED),   # above 8 pairs
     (dict(rule=3, window=0), {}, 1 << 30, F.FALCON_ERR_INVALID_ARG),
     (dict(q=None), {}, 1 << 30, F.FALCON_ERR_INVALID_ARG),
@@ -181,13 +181,14 @@ def test_backward_rejects_bad_arguments_on_host(L, akw, gkw, ws, expect):
 
 def test_backward_workspace_size(L):
     """Checkpoints every C = ceil(sqrt(T)) steps plus one segment of C + 1 recomputed states, fp32,
-    per head."""
+    per slice of 32 value rows (the last slice of a head padded to 32 rows)."""
     import math
-    for T, dk, dv in ((256, 32, 32), (100, 128, 64), (1, 16, 8), (4096, 128, 128)):
+    for T, dk, dv in ((256, 32, 32), (100, 128, 64), (1, 16, 8), (4096, 128, 128), (50, 24, 48)):
         a = _args(T=T, dk=dk, dv=dv, o=None)
         C = math.ceil(math.sqrt(T))
         nseg = -(-T // C)
-        assert L.falcon_bwd_workspace_size(ctypes.byref(a)) == 2 * 3 * (nseg + C + 1) * dv * dk * 4
+        rows = 32 * -(-dv // 32)
+        assert L.falcon_bwd_workspace_size(ctypes.byref(a)) == 2 * 3 * (nseg + C + 1) * rows * dk * 4
     assert L.falcon_bwd_workspace_size(ctypes.byref(_args(T=0))) == 0
     assert L.falcon_bwd_workspace_size(ctypes.byref(_args(rule=5))) == 0
     assert L.falcon_bwd_workspace_size(None) == 0
