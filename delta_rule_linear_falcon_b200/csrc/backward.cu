@@ -6,7 +6,7 @@
 // in fp32.
 //
 // The rows of S evolve independently given the keys, so each (b, h) is split into slices of
-// 32 value rows, one CTA of 128 threads each; every sum over value rows that the backward forms
+// 16 value rows, one CTA of 128 threads each; every sum over value rows that the backward forms
 // (dq, dx, dbeta, dalpha) feeds only an output gradient, so each slice adds its part to the
 // zeroed outputs with atomics. With U = dL/dS after step t (starting from dS_T),
 // step t (0-based, pairs j = t - m of window slot m, Sbar = alpha_t S_{t-1}) gives
@@ -39,8 +39,9 @@ namespace falcon {
 
 namespace {
 
-constexpr int kBwdRows = 32;                    // value rows per CTA (a slice of a head)
-constexpr int kBwdThreads = 4 * kBwdRows;       // four threads per row; one per key column (d_k <= 128)
+constexpr int kBwdRows = 16;                    // value rows per CTA (a slice of a head)
+constexpr int kBwdThreads = 128;                // row products: four threads per row (threads 0 .. 4 kBwdRows - 1);
+                                                // column products: one thread per key column (d_k <= 128)
 constexpr int kBwdWarps = kBwdThreads / 32;
 constexpr int kBwdMaxWindow = 8;                // pairs per step the register prefetch holds
 
