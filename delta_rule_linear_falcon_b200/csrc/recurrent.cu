@@ -6,9 +6,16 @@
 // DKMAX); keys and values of the last w pairs live in a ring of w + 1 slots in
 // shared memory, so a single barrier per step separates writing a slot from its
 // last read. The inputs of step t + A are loaded into registers while step t
-// computes (a register queue A = 3..8 steps deep), which keeps global-load latency off
-// the per-step path. The squared norm of each pair is reduced once, when the pair
-// is staged (one partial per warp), and the window sum reads those partials.
+// computes (a register queue A = 3..8 steps deep, held in the input type and
+// converted only when the step stages them, so that no instruction waits on a load
+// before that step), which keeps global-load latency off the per-step path. The
+// squared norm of each pair is reduced once, when the pair is staged (one partial
+// per warp), and the window sum reads those partials. The rows are kept as
+// S = sigma S' with one scale sigma per head: the decay multiplies sigma, and the
+// update, in units of sigma, is one fused multiply-add per entry,
+//   S' <- S' - (coef / sigma) x,   coef as below with Sbar . x = sigma (S' . x);
+// sigma is folded back into the rows whenever it leaves [2^-60, 2^60] (a zero decay
+// included).
 // Per step t (0-based, pair j = t - m for window slot m):
 //   Sbar = alpha_t S
 //   beta = eta_t / (sum_m ||x_{t-m}||^2 + eps)
@@ -46,6 +53,12 @@ __device__ __forceinline__ float row_dot(const float (&S)[DKMAX], const float *x
     return (a0 + a1) + (a2 + a3);
 }
 
+__device__ __forceinline__ float raw_f(float x) { return x; }
+__device__ __forceinline__ float raw_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename IO> __device__ __forceinline__ IO raw_zero();
+template <> __device__ __forceinline__ float raw_zero<float>() { return 0.f; }
+template <> __device__ __forceinline__ __nv_bfloat16 raw_zero<__nv_bfloat16>() { return __float2bfloat16(0.f); }
+
 template <typename IO, bool REGRESSION, int DKMAX, bool PERCOL>
 __global__ void __launch_bounds__(kRecThreads)
 recurrent_kernel(RecParams p) {
@@ -76,31 +89,34 @@ recurrent_kernel(RecParams p) {
     float ncol = (PERCOL && p.n0 && tid < dk) ? p.n0[bh * (size_t)dk + tid] : 0.f;
 
     const bool has_row = tid < dv;
+    float sigma = 1.f;                      // S = sigma S' (S' is the register row)
     float S[DKMAX];
 #pragma unroll
     for (int c = 0; c < DKMAX; ++c)
         S[c] = (has_row && p.S0 && c < dk) ? p.S0[(bh * (size_t)dv + tid) * dk + c] : 0.f;
 
-    auto load_x = [&](int t) -> float {   // key half of pair t, coordinate tid
-        if (tid >= dk) return 0.f;
-        if (p.same_step) return Io<IO>::ld(k, (size_t)t * dk + tid);
-        if (t >= 1) return Io<IO>::ld(k, (size_t)(t - 1) * dk + tid);
-        return kp ? Io<IO>::ld(kp, tid) : 0.f;
+    const IO z0 = raw_zero<IO>();
+    auto load_x = [&](int t) -> IO {   // key half of pair t, coordinate tid
+        if (tid >= dk) return z0;
+        if (p.same_step) return k[(size_t)t * dk + tid];
+        if (t >= 1) return k[(size_t)(t - 1) * dk + tid];
+        return kp ? kp[tid] : z0;
     };
-    // register queue: inputs of steps t .. t + kAhead - 1, slot t % kAhead
-    float xr[kAhead], qr[kAhead], yr[kAhead], ar[kAhead], er[kAhead];
-    auto fetch = [&](int t, float &x, float &qq, float &y, float &a, float &e) {
+    // register queue: inputs of steps t .. t + kAhead - 1, slot t % kAhead, in the input type
+    IO xr[kAhead], qr[kAhead], yr[kAhead];
+    float ar[kAhead], er[kAhead];
+    auto fetch = [&](int t, IO &x, IO &qq, IO &y, float &a, float &e) {
         if (t < T) {
             x = load_x(t);
-            qq = tid < dk ? Io<IO>::ld(q, (size_t)t * dk + tid) : 0.f;
-            y = has_row ? Io<IO>::ld(v, (size_t)t * dv + tid) : 0.f;
+            qq = tid < dk ? q[(size_t)t * dk + tid] : z0;
+            y = has_row ? v[(size_t)t * dv + tid] : z0;
             a = alpha[t];
             e = eta[t];
         }
     };
 #pragma unroll
     for (int i = 0; i < kAhead; ++i) {
-        xr[i] = 0.f; qr[i] = 0.f; yr[i] = 0.f; ar[i] = 1.f; er[i] = 0.f;
+        xr[i] = z0; qr[i] = z0; yr[i] = z0; ar[i] = 1.f; er[i] = 0.f;
         fetch(i, xr[i], qr[i], yr[i], ar[i], er[i]);
     }
     __syncthreads();
@@ -112,24 +128,25 @@ recurrent_kernel(RecParams p) {
             const int t = t0 + i;
             if (t >= T) break;
             // (A) stage pair t and q_t with the pair's squared-norm partial, refill the queue slot
+            const float xi = raw_f(xr[i]);
             {
-                float x2 = xr[i] * xr[i];
+                float x2 = xi * xi;
                 if (PERCOL) {   // x . z with z = D x: the D-weighted squared norm
                     ncol = ar[i] * ncol + x2;
                     const float den = ncol + p.eps;
-                    const float z = (tid < dk && den > 0.f) ? xr[i] / den : 0.f;
+                    const float z = (tid < dk && den > 0.f) ? xi / den : 0.f;
                     if (tid < dk) sZ[slot * DKMAX + tid] = z;   // entries dk.. stay zero
-                    x2 = z * xr[i];
+                    x2 = z * xi;
                 }
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) x2 += __shfl_xor_sync(0xffffffffu, x2, off);
                 if (lane == 0) sN[slot * kRecWarps + warp] = x2;
             }
             if (tid < dk) {
-                sX[slot * DKMAX + tid] = xr[i];
-                sQ[(t & 1) * DKMAX + tid] = qr[i];
+                sX[slot * DKMAX + tid] = xi;
+                sQ[(t & 1) * DKMAX + tid] = raw_f(qr[i]);
             }
-            if (has_row) sY[slot * DVP + tid] = yr[i];
+            if (has_row) sY[slot * DVP + tid] = raw_f(yr[i]);
             const float a = ar[i], e = er[i];
             fetch(t + kAhead, xr[i], qr[i], yr[i], ar[i], er[i]);
             __syncthreads();
@@ -148,14 +165,21 @@ recurrent_kernel(RecParams p) {
             const float beta = step_size(e, ns, p.eps);
 
             // (C) row update and the read after the write
-            if (has_row) {
+            // Sbar = (a sigma) S'; the block-uniform scale is folded into the rows if it would leave range
+            float sc = a * sigma;
+            if (!(sc >= 0x1p-60f && sc <= 0x1p60f)) {
 #pragma unroll
-                for (int c = 0; c < DKMAX; ++c) S[c] *= a;  // Sbar
+                for (int c = 0; c < DKMAX; ++c) S[c] *= sc;
+                sc = 1.f;
+            }
+            sigma = sc;
+            const float inv = 1.f / sc;
+            if (has_row) {
                 if (W == 1) {
                     const float *x = sX + slot * DKMAX;
                     const float *zw = PERCOL ? sZ + slot * DKMAX : x;   // write-key direction
-                    const float y = sY[slot * DVP + tid];
-                    const float coef = REGRESSION ? beta * (row_dot<DKMAX>(S, x) - y) : -beta * y;
+                    const float y = sY[slot * DVP + tid] * inv;
+                    const float coef = REGRESSION ? beta * (row_dot<DKMAX>(S, x) - y) : -beta * y;   // / sigma
 #pragma unroll
                     for (int c = 0; c < DKMAX; c += 4) {
                         const float4 xv = *reinterpret_cast<const float4 *>(zw + c);
@@ -168,7 +192,7 @@ recurrent_kernel(RecParams p) {
                     float coef[kRecMaxWindow];
                     int sl = slot;
                     for (int m = 0; m < nw; ++m) {
-                        const float y = sY[sl * DVP + tid];
+                        const float y = sY[sl * DVP + tid] * inv;
                         coef[m] = REGRESSION ? beta * (row_dot<DKMAX>(S, sX + sl * DKMAX) - y) : -beta * y;
                         sl = sl == 0 ? RS - 1 : sl - 1;
                     }
@@ -181,7 +205,7 @@ recurrent_kernel(RecParams p) {
                         sl = sl == 0 ? RS - 1 : sl - 1;
                     }
                 }
-                Io<IO>::st(o, (size_t)t * dv + tid, row_dot<DKMAX>(S, sQ + (t & 1) * DKMAX));
+                Io<IO>::st(o, (size_t)t * dv + tid, sigma * row_dot<DKMAX>(S, sQ + (t & 1) * DKMAX));
             }
             slot = slot + 1 == RS ? 0 : slot + 1;
         }
@@ -192,7 +216,7 @@ recurrent_kernel(RecParams p) {
         float *So = p.S_out + (bh * (size_t)dv + tid) * dk;
 #pragma unroll
         for (int c = 0; c < DKMAX; ++c)
-            if (c < dk) So[c] = S[c];
+            if (c < dk) So[c] = sigma * S[c];
     }
     if (p.k_last) {
         IO *kl = reinterpret_cast<IO *>(p.k_last) + bh * (size_t)dk;
