@@ -96,12 +96,13 @@ struct BwdCtx {
     const float *al, *et;
     int T, dk, dv, w;
     bool same;
-    // element c of the key row of pair j (0 for j < 0, or for the first pair without k_prev)
-    __device__ float key_elem(long j, int c) const {
-        if (j < 0) return 0.f;
-        if (same) return Io<IO>::ld(k, (size_t)j * dk + c);
-        if (j >= 1) return Io<IO>::ld(k, (size_t)(j - 1) * dk + c);
-        return kp ? Io<IO>::ld(kp, c) : 0.f;
+    // element c of the key row of pair j, in the input type (0 for j < 0, or for the first pair
+    // without k_prev)
+    __device__ IO key_raw(long j, int c) const {
+        if (j < 0) return Io<IO>::zero();
+        if (same) return k[(size_t)j * dk + c];
+        if (j >= 1) return k[(size_t)(j - 1) * dk + c];
+        return kp ? kp[c] : Io<IO>::zero();
     }
 };
 
@@ -194,26 +195,29 @@ bwd_recurrent_kernel(BwdParams p) {
     // The inputs of a step, loaded one step ahead into registers (thread tid < dk holds key and
     // query element tid, tid < R value and dO element r0 + tid of the slice's rows), so that their
     // memory latency overlaps the step before instead of sitting on the chain of steps.
+    // one step's inputs, the bf16 ones kept in the input type until commit converts them
     struct StepIn {
-        float a, e, q, g, x[kBwdMaxWindow], y[kBwdMaxWindow];
+        float a, e, g;
+        IO q, x[kBwdMaxWindow], y[kBwdMaxWindow];
     };
     auto fetch = [&](long t, StepIn &in, bool qg) {
-        in.a = 1.f; in.e = 0.f; in.q = 0.f; in.g = 0.f;
+        const IO z = Io<IO>::zero();
+        in.a = 1.f; in.e = 0.f; in.q = z; in.g = 0.f;
 #pragma unroll
-        for (int m = 0; m < kBwdMaxWindow; ++m) in.x[m] = in.y[m] = 0.f;
+        for (int m = 0; m < kBwdMaxWindow; ++m) in.x[m] = in.y[m] = z;
         if (t < 0 || t >= T) return;
         in.a = ctx.al[t];
         in.e = ctx.et[t];
         if (qg) {
-            if (tid < dk) in.q = Io<IO>::ld(q, (size_t)t * dk + tid);
+            if (tid < dk) in.q = q[(size_t)t * dk + tid];
             if (tid < R) in.g = dO[(size_t)t * dv + r0 + tid];
         }
 #pragma unroll
         for (int m = 0; m < kBwdMaxWindow; ++m) {
             if (m < w) {
                 const long j = t - m;
-                if (tid < dk) in.x[m] = ctx.key_elem(j, tid);
-                if (tid < R && j >= 0) in.y[m] = Io<IO>::ld(ctx.v, (size_t)j * dv + r0 + tid);
+                if (tid < dk) in.x[m] = ctx.key_raw(j, tid);
+                if (tid < R && j >= 0) in.y[m] = ctx.v[(size_t)j * dv + r0 + tid];
             }
         }
     };
@@ -221,12 +225,12 @@ bwd_recurrent_kernel(BwdParams p) {
 #pragma unroll
         for (int m = 0; m < kBwdMaxWindow; ++m) {
             if (m < w) {
-                if (tid < dk) sX[(size_t)m * dk + tid] = in.x[m];
-                if (tid < R) sY[m * RS + tid] = in.y[m];
+                if (tid < dk) sX[(size_t)m * dk + tid] = Io<IO>::cvt(in.x[m]);
+                if (tid < R) sY[m * RS + tid] = Io<IO>::cvt(in.y[m]);
             }
         }
         if (qg) {
-            if (tid < dk) sQ[tid] = in.q;
+            if (tid < dk) sQ[tid] = Io<IO>::cvt(in.q);
             if (tid < R) sG[tid] = in.g;
         }
     };

@@ -13,8 +13,12 @@ enum : int { kDevErrNone = 0, kDevErrGeometry = 1, kDevErrTimeout = 2 };
 // Element access for the two I/O dtypes. Values are widened to fp32.
 template <typename IO> struct Io;
 
+// ld/st convert at the access. cvt and zero serve code that keeps loaded values in the input
+// type until it needs them (a prefetch queue), so that no instruction waits on those loads early.
 template <> struct Io<float> {
     static __device__ __forceinline__ float ld(const float *p, size_t i) { return p[i]; }
+    static __device__ __forceinline__ float cvt(float x) { return x; }
+    static __device__ __forceinline__ float zero() { return 0.f; }
     static __device__ __forceinline__ void st(float *p, size_t i, float x) { p[i] = x; }
     // 8 consecutive elements starting at i (i multiple of 8, 16-byte aligned rows)
     static __device__ __forceinline__ void ld8(const float *p, size_t i, float (&x)[8]) {
@@ -32,6 +36,8 @@ template <> struct Io<__nv_bfloat16> {
     static __device__ __forceinline__ float ld(const __nv_bfloat16 *p, size_t i) {
         return __bfloat162float(p[i]);
     }
+    static __device__ __forceinline__ float cvt(__nv_bfloat16 x) { return __bfloat162float(x); }
+    static __device__ __forceinline__ __nv_bfloat16 zero() { return __float2bfloat16(0.f); }
     static __device__ __forceinline__ void st(__nv_bfloat16 *p, size_t i, float x) {
         p[i] = __float2bfloat16_rn(x);
     }

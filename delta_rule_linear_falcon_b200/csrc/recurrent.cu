@@ -53,12 +53,6 @@ __device__ __forceinline__ float row_dot(const float (&S)[DKMAX], const float *x
     return (a0 + a1) + (a2 + a3);
 }
 
-__device__ __forceinline__ float raw_f(float x) { return x; }
-__device__ __forceinline__ float raw_f(__nv_bfloat16 x) { return __bfloat162float(x); }
-template <typename IO> __device__ __forceinline__ IO raw_zero();
-template <> __device__ __forceinline__ float raw_zero<float>() { return 0.f; }
-template <> __device__ __forceinline__ __nv_bfloat16 raw_zero<__nv_bfloat16>() { return __float2bfloat16(0.f); }
-
 template <typename IO, bool REGRESSION, int DKMAX, bool PERCOL>
 __global__ void __launch_bounds__(kRecThreads)
 recurrent_kernel(RecParams p) {
@@ -95,7 +89,7 @@ recurrent_kernel(RecParams p) {
     for (int c = 0; c < DKMAX; ++c)
         S[c] = (has_row && p.S0 && c < dk) ? p.S0[(bh * (size_t)dv + tid) * dk + c] : 0.f;
 
-    const IO z0 = raw_zero<IO>();
+    const IO z0 = Io<IO>::zero();
     auto load_x = [&](int t) -> IO {   // key half of pair t, coordinate tid
         if (tid >= dk) return z0;
         if (p.same_step) return k[(size_t)t * dk + tid];
@@ -128,7 +122,7 @@ recurrent_kernel(RecParams p) {
             const int t = t0 + i;
             if (t >= T) break;
             // (A) stage pair t and q_t with the pair's squared-norm partial, refill the queue slot
-            const float xi = raw_f(xr[i]);
+            const float xi = Io<IO>::cvt(xr[i]);
             {
                 float x2 = xi * xi;
                 if (PERCOL) {   // x . z with z = D x: the D-weighted squared norm
@@ -144,9 +138,9 @@ recurrent_kernel(RecParams p) {
             }
             if (tid < dk) {
                 sX[slot * DKMAX + tid] = xi;
-                sQ[(t & 1) * DKMAX + tid] = raw_f(qr[i]);
+                sQ[(t & 1) * DKMAX + tid] = Io<IO>::cvt(qr[i]);
             }
-            if (has_row) sY[slot * DVP + tid] = raw_f(yr[i]);
+            if (has_row) sY[slot * DVP + tid] = Io<IO>::cvt(yr[i]);
             const float a = ar[i], e = er[i];
             fetch(t + kAhead, xr[i], qr[i], yr[i], ar[i], er[i]);
             __syncthreads();
