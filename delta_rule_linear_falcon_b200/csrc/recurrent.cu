@@ -16,6 +16,9 @@
 //   S' <- S' - (coef / sigma) x,   coef as below with Sbar . x = sigma (S' . x);
 // sigma is folded back into the rows whenever it leaves [2^-60, 2^60] (a zero decay
 // included).
+// Window 1 has an instantiation of its own, without the window loops; with 128 key
+// columns the row takes 128 registers, and both of these keep the rest of the kernel in
+// registers too (the state row spilled before, and a step took two to three times as long).
 // Per step t (0-based, pair j = t - m for window slot m):
 //   Sbar = alpha_t S
 //   beta = eta_t / (sum_m ||x_{t-m}||^2 + eps)
@@ -53,17 +56,23 @@ __device__ __forceinline__ float row_dot(const float (&S)[DKMAX], const float *x
     return (a0 + a1) + (a2 + a3);
 }
 
-template <typename IO, bool REGRESSION, int DKMAX, bool PERCOL>
+// ONE: the window is one pair (compiled without the window loops, whose per-pair coefficients
+// would otherwise take registers from the state row).
+template <typename IO, bool REGRESSION, int DKMAX, bool PERCOL, bool ONE>
 __global__ void __launch_bounds__(kRecThreads)
 recurrent_kernel(RecParams p) {
     extern __shared__ __align__(16) float smem[];
-    const int dk = p.dk, dv = p.dv, W = p.window, RS = W + 1;
+    const int dk = p.dk, dv = p.dv, W = ONE ? 1 : p.window, RS = W + 1;
     float *sX = smem;                        // RS x DKMAX key ring (zero padded)
     float *sY = sX + (size_t)RS * DKMAX;     // RS x DVP value ring
     const int DVP = (dv + 3) & ~3;
     float *sQ = sY + (size_t)RS * DVP;       // 2 x DKMAX queries (double buffered)
     float *sN = sQ + 2 * DKMAX;              // RS x kRecWarps partial squared norms of the pairs
-    float *sZ = sN + RS * kRecWarps;         // per-column rules: RS x DKMAX write-key directions
+    float *sZ = sN + RS * kRecWarps;         // RS x DKMAX write-key directions (a copy of the key for
+                                             // the other rules, so that the update and the dot product
+                                             // read different arrays: when they read one, the compiler
+                                             // keeps the dot product's loads for the update, 128 more
+                                             // live registers beside the row)
     constexpr int kAhead = ahead<DKMAX>();
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -77,7 +86,7 @@ recurrent_kernel(RecParams p) {
     const float *eta = p.eta + bh * (size_t)T;
     IO *o = reinterpret_cast<IO *>(p.o) + bh * (size_t)T * dv;
 
-    for (int idx = tid; idx < RS * (DKMAX + DVP + kRecWarps) + 2 * DKMAX + (PERCOL ? RS * DKMAX : 0); idx += kRecThreads)
+    for (int idx = tid; idx < RS * (DKMAX + DVP + kRecWarps) + 2 * DKMAX + RS * DKMAX; idx += kRecThreads)
         smem[idx] = 0.f;
     // running energy of key coordinate tid (per-column rules)
     float ncol = (PERCOL && p.n0 && tid < dk) ? p.n0[bh * (size_t)dk + tid] : 0.f;
@@ -138,6 +147,7 @@ recurrent_kernel(RecParams p) {
             }
             if (tid < dk) {
                 sX[slot * DKMAX + tid] = xi;
+                if (!PERCOL && ONE) sZ[slot * DKMAX + tid] = xi;
                 sQ[(t & 1) * DKMAX + tid] = Io<IO>::cvt(qr[i]);
             }
             if (has_row) sY[slot * DVP + tid] = Io<IO>::cvt(yr[i]);
@@ -169,9 +179,9 @@ recurrent_kernel(RecParams p) {
             sigma = sc;
             const float inv = 1.f / sc;
             if (has_row) {
-                if (W == 1) {
+                if (ONE || W == 1) {
                     const float *x = sX + slot * DKMAX;
-                    const float *zw = PERCOL ? sZ + slot * DKMAX : x;   // write-key direction
+                    const float *zw = sZ + slot * DKMAX;   // write-key direction
                     const float y = sY[slot * DVP + tid] * inv;
                     const float coef = REGRESSION ? beta * (row_dot<DKMAX>(S, x) - y) : -beta * y;   // / sigma
 #pragma unroll
@@ -234,7 +244,9 @@ size_t recurrent_smem_bytes(int dk, int dv, int window) {
 template <typename IO, bool REG, int DKMAX>
 static cudaError_t launch_rec(const RecParams &p, cudaStream_t s) {
     const size_t smem = recurrent_smem_bytes(p.dk, p.dv, p.window);
-    auto kern = p.per_column ? recurrent_kernel<IO, REG, DKMAX, true> : recurrent_kernel<IO, REG, DKMAX, false>;
+    auto kern = p.per_column      ? recurrent_kernel<IO, REG, DKMAX, true, true>
+                : p.window == 1 ? recurrent_kernel<IO, REG, DKMAX, false, true>
+                                : recurrent_kernel<IO, REG, DKMAX, false, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long grid = (long)p.B * p.H;
