@@ -40,9 +40,10 @@ namespace falcon {
 namespace {
 
 constexpr int kBwdRows = 16;                    // value rows per CTA (a slice of a head)
-constexpr int kBwdThreads = 128;                // row products: four threads per row (threads 0 .. 4 kBwdRows - 1);
+constexpr int kBwdThreads = 128;                // row products: kRowThr threads per row (all 128 for 16 rows);
                                                 // column products: one thread per key column (d_k <= 128)
 constexpr int kBwdWarps = kBwdThreads / 32;
+constexpr int kRowThr = kBwdThreads / kBwdRows; // threads per value row in the row products (8)
 constexpr int kBwdMaxWindow = 8;                // pairs per step the register prefetch holds
 
 struct BwdSmem {
@@ -53,7 +54,9 @@ struct BwdSmem {
 
 __host__ __device__ inline BwdSmem bwd_smem(int dk, int w) {
     BwdSmem s;
-    s.LD = ((dk + 27) / 32) * 32 + 4; s.dk = dk; s.w = w;
+    // row stride = 8 mod 32 floats: the four rows of a warp's row products (8 threads each) and a
+    // column phase fall on distinct banks
+    s.LD = ((dk + 31) / 32) * 32 + 8; s.dk = dk; s.w = w;
     constexpr int R = kBwdRows;
     const size_t mat = (size_t)R * s.LD;
     s.oU = 0; s.oP = mat; s.oA = 2 * mat;
@@ -82,10 +85,10 @@ __device__ __forceinline__ float block_sum(float x, float *red) {
     return s;
 }
 
-// Sum over the four threads of a value row (lanes 4i .. 4i + 3); all four get it.
-__device__ __forceinline__ float quad_sum(float x) {
-    x += __shfl_xor_sync(0xffffffffu, x, 1);
-    x += __shfl_xor_sync(0xffffffffu, x, 2);
+// Sum over the kRowThr threads of a value row (lanes kRowThr i ..); all of them get it.
+__device__ __forceinline__ float row_sum(float x) {
+#pragma unroll
+    for (int o = 1; o < kRowThr; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
     return x;
 }
 
@@ -121,7 +124,7 @@ bwd_recurrent_kernel(BwdParams p) {
     const int nsl = (dv + kBwdRows - 1) / kBwdRows;
     const size_t bh = blockIdx.x / nsl;
     const int sl = blockIdx.x % nsl, r0 = sl * kBwdRows, R = min(kBwdRows, dv - r0);   // the slice's rows
-    const int ri = tid >> 2, rq = tid & 3;          // row products: slice row ri, columns rq, rq + 4, ..
+    const int ri = tid / kRowThr, rq = tid % kRowThr;   // row products: slice row ri, columns rq, rq + kRowThr, ..
     const bool rok = ri < R;
     const int cc = tid;                             // column products: key column cc over the slice's rows
     const size_t DD = (size_t)dv * dk;              // a head's state in the caller's arrays
@@ -252,15 +255,15 @@ bwd_recurrent_kernel(BwdParams p) {
         const float a = in.a;
         float *Si = sP + (size_t)(rok ? ri : 0) * LD;
         if (rok)
-            for (int c = rq; c < dk; c += 4) Si[c] *= a;
+            for (int c = rq; c < dk; c += kRowThr) Si[c] *= a;
         if (REG) {
             // residuals at the decayed state first (every window pair), then the update
             for (int m = 0; m < w; ++m) {
                 const float *x = sX + (size_t)m * dk;
                 float r = 0.f;
                 if (rok)
-                    for (int c = rq; c < dk; c += 4) r = fmaf(Si[c], x[c], r);
-                r = quad_sum(r);
+                    for (int c = rq; c < dk; c += kRowThr) r = fmaf(Si[c], x[c], r);
+                r = row_sum(r);
                 if (rok && rq == 0) sR[m * RS + ri] = r - sY[m * RS + ri];
             }
             __syncwarp();
@@ -268,13 +271,13 @@ bwd_recurrent_kernel(BwdParams p) {
                 for (int m = 0; m < w; ++m) {
                     const float *x = sX + (size_t)m * dk;
                     const float br = beta * sR[m * RS + ri];
-                    for (int c = rq; c < dk; c += 4) Si[c] = fmaf(-br, x[c], Si[c]);
+                    for (int c = rq; c < dk; c += kRowThr) Si[c] = fmaf(-br, x[c], Si[c]);
                 }
         } else if (rok) {
             for (int m = 0; m < w; ++m) {
                 const float *x = sX + (size_t)m * dk;
                 const float by = beta * sY[m * RS + ri];
-                for (int c = rq; c < dk; c += 4) Si[c] = fmaf(by, x[c], Si[c]);
+                for (int c = rq; c < dk; c += kRowThr) Si[c] = fmaf(by, x[c], Si[c]);
             }
         }
     };
@@ -330,18 +333,18 @@ bwd_recurrent_kernel(BwdParams p) {
                 const float *Pi = sP + (size_t)(rok ? ri : 0) * LD;
                 if (rok) {
                     const float g = sG[ri];
-                    for (int c = rq; c < dk; c += 4) Ui[c] = fmaf(g, sQ[c], Ui[c]);
+                    for (int c = rq; c < dk; c += kRowThr) Ui[c] = fmaf(g, sQ[c], Ui[c]);
                 }
                 for (int m = 0; m < w; ++m) {
                     const float *x = sX + (size_t)m * dk;
                     float ux = 0.f, sx = 0.f;
                     if (rok)
-                        for (int c = rq; c < dk; c += 4) {
+                        for (int c = rq; c < dk; c += kRowThr) {
                             ux = fmaf(Ui[c], x[c], ux);
                             sx = fmaf(Pi[c], x[c], sx);
                         }
-                    ux = quad_sum(ux);
-                    sx = quad_sum(sx);
+                    ux = row_sum(ux);
+                    sx = row_sum(sx);
                     if (rok && rq == 0) {
                         sUx[m * RS + ri] = ux;
                         if (REG) {
@@ -360,7 +363,7 @@ bwd_recurrent_kernel(BwdParams p) {
             if (tid == 0 && has_den) atomicAdd(get + t, dbeta / den);
             // rows: dr_m, dy_m (scattered to the value row of pair j)
             if (rok)
-                for (int m = rq; m < w; m += 4) {
+                for (int m = rq; m < w; m += kRowThr) {
                     const float ux = sUx[m * RS + ri];
                     if (REG) sDr[m * RS + ri] = -beta * ux;
                     const long j = t - m;
@@ -403,7 +406,7 @@ bwd_recurrent_kernel(BwdParams p) {
             if (rok) {
                 float *Ui = sU + (size_t)ri * LD;
                 const float *Pi = sP + (size_t)ri * LD;
-                for (int c = rq; c < dk; c += 4) {
+                for (int c = rq; c < dk; c += kRowThr) {
                     float d = Ui[c];
                     if (REG)
                         for (int m = 0; m < w; ++m) d = fmaf(sDr[m * RS + ri], sX[(size_t)m * dk + c], d);
