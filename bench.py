@@ -453,7 +453,7 @@ def bench_backward(args, D: Dist):
     ms = t0.elapsed_time(t1) / 3
     return {"workload": f"falcon1_bwd_recurrent_bf16_B{B}H{H}T{T}d{d}", "ms_per_call": round(ms, 3),
             "tokens_per_s": round(B * T / (ms * 1e-3), 1), "workspace_bytes": int(ws.numel()),
-            "note": "latency bound: one CTA per 16 value rows of a head, forward to checkpoints, then "
+            "note": "latency bound: one CTA per 8 value rows of a head, forward to checkpoints, then "
                     "recompute and reverse per segment"}
 
 

@@ -39,11 +39,12 @@ namespace falcon {
 
 namespace {
 
-constexpr int kBwdRows = 16;                    // value rows per CTA (a slice of a head)
-constexpr int kBwdThreads = 128;                // row products: kRowThr threads per row (all 128 for 16 rows);
+constexpr int kBwdRows = 8;                     // value rows per CTA (a slice of a head)
+constexpr int kBwdThreads = 128;                // row products: kRowThr threads per row (all 128 threads);
                                                 // column products: one thread per key column (d_k <= 128)
 constexpr int kBwdWarps = kBwdThreads / 32;
-constexpr int kRowThr = kBwdThreads / kBwdRows; // threads per value row in the row products (8)
+constexpr int kRowThr = kBwdThreads / kBwdRows; // threads per value row in the row products (16)
+static_assert(32 % kRowThr == 0 && kRowThr % 4 == 0, "a warp holds whole rows; rows stay 16-byte aligned");
 constexpr int kBwdMaxWindow = 8;                // pairs per step the register prefetch holds
 
 struct BwdSmem {
@@ -54,9 +55,9 @@ struct BwdSmem {
 
 __host__ __device__ inline BwdSmem bwd_smem(int dk, int w) {
     BwdSmem s;
-    // row stride = 8 mod 32 floats: the four rows of a warp's row products (8 threads each) and a
-    // column phase fall on distinct banks
-    s.LD = ((dk + 31) / 32) * 32 + 8; s.dk = dk; s.w = w;
+    // row stride = kRowThr mod 32 floats: the rows of a warp's row products (kRowThr threads each)
+    // and a column phase fall on distinct banks
+    s.LD = ((dk + 31) / 32) * 32 + kRowThr; s.dk = dk; s.w = w;
     constexpr int R = kBwdRows;
     const size_t mat = (size_t)R * s.LD;
     s.oU = 0; s.oP = mat; s.oA = 2 * mat;

@@ -256,8 +256,8 @@ FALCON_API falcon_status_t falcon_fwd_recurrent(const falcon_args_t *args, falco
  *   args->k_prev is given.
  * Workspace: falcon_bwd_workspace_size(args) bytes, 16-byte aligned (the states at the
  * start of every segment of about sqrt(T) steps and one segment of recomputed states,
- * fp32, per slice of 16 value rows of a head). fp32 state and arithmetic; one CTA of 128
- * threads per slice of 16 value rows of a (b, h): the rows of S evolve independently, and the
+ * fp32, per slice of 8 value rows of a head). fp32 state and arithmetic; one CTA of 128
+ * threads per slice of 8 value rows of a (b, h): the rows of S evolve independently, and the
  * slices add their parts of dq, dk, dalpha, deta and dk_prev to the outputs with atomic adds
  * (so those sums are taken in no fixed order, and their last bits can differ between runs);
  * dv and dS0 rows are each written by one slice.

@@ -181,13 +181,13 @@ def test_backward_rejects_bad_arguments_on_host(L, akw, gkw, ws, expect):
 
 def test_backward_workspace_size(L):
     """Checkpoints every C = ceil(sqrt(T)) steps plus one segment of C + 1 recomputed states, fp32,
-    per slice of 16 value rows (the last slice of a head padded to 16 rows)."""
+    per slice of 8 value rows (the last slice of a head padded to 8 rows)."""
     import math
     for T, dk, dv in ((256, 32, 32), (100, 128, 64), (1, 16, 8), (4096, 128, 128), (50, 24, 48)):
         a = _args(T=T, dk=dk, dv=dv, o=None)
         C = math.ceil(math.sqrt(T))
         nseg = -(-T // C)
-        rows = 16 * -(-dv // 16)
+        rows = 8 * -(-dv // 8)
         assert L.falcon_bwd_workspace_size(ctypes.byref(a)) == 2 * 3 * (nseg + C + 1) * rows * dk * 4
     assert L.falcon_bwd_workspace_size(ctypes.byref(_args(T=0))) == 0
     assert L.falcon_bwd_workspace_size(ctypes.byref(_args(rule=5))) == 0
