@@ -45,6 +45,7 @@ constexpr int kBwdThreads = 128;                // row products: kRowThr threads
 constexpr int kBwdWarps = kBwdThreads / 32;
 constexpr int kRowThr = kBwdThreads / kBwdRows; // threads per value row in the row products (16)
 static_assert(32 % kRowThr == 0 && kRowThr % 4 == 0, "a warp holds whole rows; rows stay 16-byte aligned");
+static_assert(kBwdRows % 2 == 0, "the column products take the rows in pairs");
 constexpr int kBwdMaxWindow = 8;                // pairs per step the register prefetch holds
 
 struct BwdSmem {
@@ -130,6 +131,10 @@ bwd_recurrent_kernel(BwdParams p) {
     const int cc = tid;                             // column products: key column cc over the slice's rows
     const size_t DD = (size_t)dv * dk;              // a head's state in the caller's arrays
     const size_t DS = (size_t)kBwdRows * dk;        // a slice's state in the workspace
+    // Shared memory starts at zero: rows R .. kBwdRows - 1 of every row array then stay zero (each
+    // writer of a row is guarded by its row), so the column products run over all kBwdRows rows.
+    for (int i = tid; i < (int)L.total; i += kBwdThreads) smem[i] = 0.f;
+    __syncthreads();
 
     BwdCtx<IO> ctx{p,
                    reinterpret_cast<const IO *>(p.q) + bh * T * dk,
@@ -378,20 +383,33 @@ bwd_recurrent_kernel(BwdParams p) {
             __syncthreads();
             // columns: dq_t = S_t^T dO_t; dx_m (scattered to the key row of pair j): this slice's rows
             if (cc < dk) {
-                float acc = 0.f;
-                for (int i = 0; i < R; ++i) acc = fmaf(sA[i * LD + cc], sG[i], acc);
-                atomicAdd(gq + (size_t)t * dk + cc, acc);
+                float acc0 = 0.f, acc1 = 0.f;   // two chains over the slice's rows (zero beyond R)
+#pragma unroll
+                for (int i = 0; i < kBwdRows; i += 2) {
+                    acc0 = fmaf(sA[i * LD + cc], sG[i], acc0);
+                    acc1 = fmaf(sA[(i + 1) * LD + cc], sG[i + 1], acc1);
+                }
+                atomicAdd(gq + (size_t)t * dk + cc, acc0 + acc1);
                 for (int m = 0; m < w; ++m) {
-                    float dx = 0.f;
-                    if (REG) {
+                    float dx;
+                    if (REG) {   // -beta U^T r + alpha S^T dr, each sum its own chain
                         const float *r = sR + m * RS, *dr = sDr + m * RS;
-                        for (int i = 0; i < R; ++i) {
-                            dx = fmaf(-beta * sU[i * LD + cc], r[i], dx);
-                            dx = fmaf(a * sP[i * LD + cc], dr[i], dx);
+                        float ur = 0.f, pd = 0.f;
+#pragma unroll
+                        for (int i = 0; i < kBwdRows; ++i) {
+                            ur = fmaf(sU[i * LD + cc], r[i], ur);
+                            pd = fmaf(sP[i * LD + cc], dr[i], pd);
                         }
+                        dx = fmaf(-beta, ur, a * pd);
                     } else {
                         const float *y = sY + m * RS;
-                        for (int i = 0; i < R; ++i) dx = fmaf(beta * sU[i * LD + cc], y[i], dx);
+                        float u0 = 0.f, u1 = 0.f;
+#pragma unroll
+                        for (int i = 0; i < kBwdRows; i += 2) {
+                            u0 = fmaf(sU[i * LD + cc], y[i], u0);
+                            u1 = fmaf(sU[(i + 1) * LD + cc], y[i + 1], u1);
+                        }
+                        dx = beta * (u0 + u1);
                     }
                     dx = fmaf(2.f * dN, sX[(size_t)m * dk + cc], dx);
                     const long j = t - m;
