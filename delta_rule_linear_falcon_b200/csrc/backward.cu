@@ -261,6 +261,7 @@ bwd_recurrent_kernel(BwdParams p) {
         const float a = in.a;
         float *Si = sP + (size_t)(rok ? ri : 0) * LD;
         if (rok)
+#pragma unroll 4
             for (int c = rq; c < dk; c += kRowThr) Si[c] *= a;
         if (REG) {
             // residuals at the decayed state first (every window pair), then the update
@@ -268,6 +269,7 @@ bwd_recurrent_kernel(BwdParams p) {
                 const float *x = sX + (size_t)m * dk;
                 float r = 0.f;
                 if (rok)
+#pragma unroll 4
                     for (int c = rq; c < dk; c += kRowThr) r = fmaf(Si[c], x[c], r);
                 r = row_sum(r);
                 if (rok && rq == 0) sR[m * RS + ri] = r - sY[m * RS + ri];
@@ -277,12 +279,14 @@ bwd_recurrent_kernel(BwdParams p) {
                 for (int m = 0; m < w; ++m) {
                     const float *x = sX + (size_t)m * dk;
                     const float br = beta * sR[m * RS + ri];
+#pragma unroll 4
                     for (int c = rq; c < dk; c += kRowThr) Si[c] = fmaf(-br, x[c], Si[c]);
                 }
         } else if (rok) {
             for (int m = 0; m < w; ++m) {
                 const float *x = sX + (size_t)m * dk;
                 const float by = beta * sY[m * RS + ri];
+#pragma unroll 4
                 for (int c = rq; c < dk; c += kRowThr) Si[c] = fmaf(by, x[c], Si[c]);
             }
         }
@@ -339,12 +343,14 @@ bwd_recurrent_kernel(BwdParams p) {
                 const float *Pi = sP + (size_t)(rok ? ri : 0) * LD;
                 if (rok) {
                     const float g = sG[ri];
+#pragma unroll 4
                     for (int c = rq; c < dk; c += kRowThr) Ui[c] = fmaf(g, sQ[c], Ui[c]);
                 }
                 for (int m = 0; m < w; ++m) {
                     const float *x = sX + (size_t)m * dk;
                     float ux = 0.f, sx = 0.f;
                     if (rok)
+#pragma unroll 4
                         for (int c = rq; c < dk; c += kRowThr) {
                             ux = fmaf(Ui[c], x[c], ux);
                             sx = fmaf(Pi[c], x[c], sx);
@@ -425,6 +431,7 @@ bwd_recurrent_kernel(BwdParams p) {
             if (rok) {
                 float *Ui = sU + (size_t)ri * LD;
                 const float *Pi = sP + (size_t)ri * LD;
+#pragma unroll 4
                 for (int c = rq; c < dk; c += kRowThr) {
                     float d = Ui[c];
                     if (REG)
