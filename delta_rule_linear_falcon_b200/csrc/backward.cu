@@ -6,7 +6,7 @@
 // in fp32.
 //
 // The rows of S evolve independently given the keys, so each (b, h) is split into slices of
-// 16 value rows, one CTA of 128 threads each; every sum over value rows that the backward forms
+// 8 value rows, one CTA of 128 threads each; every sum over value rows that the backward forms
 // (dq, dx, dbeta, dalpha) feeds only an output gradient, so each slice adds its part to the
 // zeroed outputs with atomics. With U = dL/dS after step t (starting from dS_T),
 // step t (0-based, pairs j = t - m of window slot m, Sbar = alpha_t S_{t-1}) gives
@@ -26,10 +26,10 @@
 // C steps in the workspace, and the reverse sweep re-runs each segment forward from its
 // checkpoint into a buffer of C + 1 states before walking it backwards. The slice's rows of U
 // and of the two states a step needs (before and after it) sit in shared memory. Row products
-// (U x, Sbar x, the state update) take four threads per value row i, each every fourth column,
-// reduced with two shuffles; the row stride is 4 more than a multiple of 32 floats, so the 32
-// threads of a warp (8 rows x 4 column phases) hit 32 different banks. Column products (S^T dO,
-// U^T r, Sbar^T dr) take one thread per key column over the slice's rows.
+// (U x, Sbar x, the state update) take sixteen threads per value row i, each every sixteenth
+// column, reduced with four shuffles; the row stride is 16 more than a multiple of 32 floats, so
+// the 32 threads of a warp (2 rows x 16 column phases) hit 32 different banks. Column products
+// (S^T dO, U^T r, Sbar^T dr) take one thread per key column over the slice's rows.
 #include <math.h>
 
 #include "common.cuh"
